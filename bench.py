@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark of the OrbitQuant quantized linear layer forward on B200.
+
+One step is one pass of the hot path over one batch of synthetic tokens:
+rotate + quantize (norm, permutation gather, block Walsh-Hadamard, Lloyd-Max
+codes) followed by the codebook contraction with the s*r epilogue.  The
+weights are prepared once beforehand (offline in the method).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) shard tokens: every
+rank processes its own batch of the workload with replicated weights (weak
+scaling, no collective on the data path).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantized-linear tokens/s at d=3072; RPBH+quant HBM GB/s; GEMM % TC peak"
+UNIT = "tokens/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="dit_image")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+            "bf16_tflops_sustained": None, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            v = [t.strip() for t in ln.split(",")]
+            if len(v) < 9:
+                continue
+            try:
+                sm.append(float(v[1]))
+                smax.append(float(v[2]))
+                power.append(float(v[3]))
+            except ValueError:
+                continue
+            for n, flag in zip(names, v[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle timing (host)
+def oracle_cpu_rate(wl, lay, seconds: float, chunk: int = 32):
+    """Tokens/s of the fp64 oracle (as it stands) on this host's cores, on a
+    bounded sample of the workload: chunks of `chunk` tokens, until `seconds`
+    of work have run.  Weight rows are prepared by the oracle beforehand
+    (offline in the method, not timed)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle as O
+    from quantized_linear_token_b200 import workloads as W
+
+    d = lay.d_in
+    h = O.hadamard_block_size(d)
+    perm = O.rpbh_permutation(d, W.ROTATION_SEED)
+    cb_a, cb_w = O.lloyd_max(d, lay.a_bits), O.lloyd_max(d, lay.w_bits)
+    Wm = W.weights(wl, lay).astype(np.float64)
+    wc, r, _ = O.weight_prepare(Wm, perm, h, cb_w)
+    x = W.activations(wl, d, tokens=min(wl.tokens, 1024))
+    x64 = O.bf16_bits_to_f64(x) if x.dtype == np.uint16 else x.astype(np.float64)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        i0 = (done % x64.shape[0])
+        xs = x64[i0:i0 + chunk]
+        codes, s, _ = O.rotate_quantize(xs, perm, h, cb_a)
+        O.linear_from_codes(codes, s, wc, r, cb_a.levels, cb_w.levels)
+        done += xs.shape[0]
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return done / el, el, done, threads
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from quantized_linear_token_b200 import binding as B
+    from quantized_linear_token_b200 import build as Bld
+    from quantized_linear_token_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        Bld.build()
+    if world > 1:
+        dist.barrier()
+    B.load_library()
+
+    wl = W.WORKLOADS[args.workload]
+    lay = wl.layers[0]
+    T, d, dout = wl.tokens, lay.d_in, lay.d_out
+    x_np = W.activations(wl, d)
+    Wm = W.weights(wl, lay)
+    x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
+    layer = B.oq_layer_create(d, dout, W.ROTATION_SEED, lay.a_bits, lay.w_bits)
+    Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(Wm).to(dev))
+    codes = torch.empty((T, layer.a_words_per_row), dtype=torch.int32, device=dev)
+    s = torch.empty((T,), dtype=torch.float32, device=dev)
+    y = torch.empty((T, dout), dtype=torch.float32, device=dev)
+    ws = torch.empty((B.oq_linear_fused_workspace_size(layer, T),), dtype=torch.uint8, device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        B.oq_rotate_quantize(layer, x, codes, s)
+        B.oq_linear(layer, codes, s, Wc, r, y)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()                                  # L2 flushed, outside the events
+        ev[i][0].record(stream)
+        B.oq_rotate_quantize(layer, x, codes, s)
+        ev[i][1].record(stream)
+        B.oq_linear(layer, codes, s, Wc, r, y)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    clk = clocks.stop() if clocks else None
+    t_rq = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_mm = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    t_step = [a + b for a, b in zip(t_rq, t_mm)]
+    total_ms = sum(t_step)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    B.oq_poll_error(layer)
+
+    # fused call, same workload (one C call, both kernels)
+    for _ in range(2):
+        B.oq_linear_fused(layer, x, Wc, r, y, ws)
+    evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(K):
+        flush.zero_()
+        evf[i][0].record(stream)
+        B.oq_linear_fused(layer, x, Wc, r, y, ws)
+        evf[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_fused = [evf[i][0].elapsed_time(evf[i][1]) for i in range(K)]
+
+    # end to end through the public API with host buffers: pinned x -> device,
+    # fused call, y -> pinned host, all inside the events
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty((T, dout), dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    eve = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(max(2, args.warmup // 2)):
+        x_dev.copy_(x_host, non_blocking=True)
+        B.oq_linear_fused(layer, x_dev, Wc, r, y, ws)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    for i in range(K):
+        eve[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        B.oq_linear_fused(layer, x_dev, Wc, r, y, ws)
+        y_host.copy_(y, non_blocking=True)
+        eve[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = [eve[i][0].elapsed_time(eve[i][1]) for i in range(K)]
+    e2e_ms = sum(t_e2e)
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    B.oq_poll_error(layer)
+
+    peaks = load_peaks()
+    flops = 2.0 * T * d * dout
+    mm_ms = statistics.mean(t_mm)
+    rq_ms = statistics.mean(t_rq)
+    rq_bytes = T * (2 * d + d * lay.a_bits / 8 + 4)
+    gemm_tf = flops / (mm_ms * 1e-3) / 1e12
+    rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": world * T * K / (total_ms * 1e-3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{args.workload}: {wl.title}",
+            "tokens_per_gpu": T, "d_in": d, "d_out": dout, "a_bits": lay.a_bits, "w_bits": lay.w_bits,
+            "h": d & -d, "x_dtype": "bf16", "y_dtype": "fp32",
+            "parallelism": f"token-sharded x{world}, weights replicated",
+            "l2": "flushed (256 MiB write) before every step, outside the timed events",
+            "step": "oq_rotate_quantize + oq_linear (weights prepared once, offline)",
+        },
+        "roofline": {
+            "kernel": "codebook GEMM (tcgen05, decode to fp16, fp32 TMEM accumulate)",
+            "bound": "tensor", "achieved": gemm_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": gemm_tf / peaks["bf16_tflops"], "traffic": None,
+            "peak_source": f"{peaks['source']} bf16 dense burst (fp16 has the same tensor rate)",
+            "flops_per_launch": flops, "ms_per_launch": mm_ms,
+        },
+        "roofline_rotate_quantize": {
+            "kernel": "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes, pack)",
+            "bound": "hbm", "achieved": rq_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": rq_gbs / peaks["hbm_gbs"], "traffic": None,
+            "peak_source": f"{peaks['source']} HBM copy bandwidth",
+            "bytes_per_launch": rq_bytes, "ms_per_launch": rq_ms,
+        },
+        "fused": {"value": T / (statistics.mean(t_fused) * 1e-3), "unit": UNIT,
+                  "ms_per_call": statistics.mean(t_fused)},
+        "e2e": {"value": world * T * K / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(y.numel() * y.element_size()),
+                "path": "pinned host x -> device, oq_linear_fused, y -> pinned host"},
+        "gpu_launches": 2 * K,
+        "wall_s_timed_region": wall,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, el, done, threads = oracle_cpu_rate(wl, lay, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                               "sample": f"{done} tokens of {args.workload} in chunks of 32 "
+                                         f"({el:.1f} s): oracle rotate_quantize + linear_from_codes, "
+                                         f"fp64 numpy; weight rows prepared beforehand"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The oracle timed on the host cores, on this arm's workload/metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from quantized_linear_token_b200 import workloads as W
+    wl = W.WORKLOADS[args.workload]
+    lay = wl.layers[0]
+    per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_cpu_rate(wl, lay, min(per_step, 2.0))
+    rates, total_tok, total_s, threads = [], 0, 0.0, 1
+    for _ in range(args.steps):
+        rate, el, done, threads = oracle_cpu_rate(wl, lay, per_step)
+        rates.append(rate)
+        total_tok += done
+        total_s += el
+    value = total_tok / total_s
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {wl.title}", "d_in": lay.d_in, "d_out": lay.d_out,
+                   "a_bits": lay.a_bits, "w_bits": lay.w_bits},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{total_tok} tokens, {args.steps} steps of ~{per_step:.1f} s, chunks of 32"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,204 @@
+/*
+ * orbitquant.h -- C ABI of the OrbitQuant quantized linear layer on B200.
+ *
+ * The method ("OrbitQuant: Data-Agnostic Quantization for Image and Video
+ * Diffusion Transformers", arXiv 2607.02461), as described by the web pages
+ * cited below:
+ *   - per token, split the activation into its norm s and direction x/s
+ *     (paper.gecl.asia reading notes, Method 1);
+ *   - rotate the direction with the randomized permuted block-Hadamard
+ *     (RPBH) rotation R = blockdiag(H_h/sqrt(h)) P_pi, h the largest power of
+ *     two dividing d (gecl notes Method 4 and Key Insight; pith.science
+ *     Supplementary A);
+ *   - code every rotated coordinate with the Lloyd-Max codebook C_{d,b}
+ *     designed for the fixed marginal f_d ~ N(0, 1/d) (gecl notes Method 3;
+ *     pith Figure 2);
+ *   - weight rows get the same rotation, norm split and quantizer offline, so
+ *     the rotation cancels inside the layer (hotpaper.ai abstract; gecl notes
+ *     Method 2; llmdb.app Mathematical Formulation y = Q_w(W R^-1) Q_a(R x)).
+ *   y[t, o] = s_t r_o sum_i C_w[Wc[o, i]] C_a[Xc[t, i]].
+ *
+ * Conventions for every call below:
+ *   - Pointers named "device" must point to CUDA device memory of the current
+ *     device, be 16-byte aligned and be contiguous row-major.  The caller owns
+ *     them.  The library owns only what an oq_layer holds (the permutation,
+ *     codebook tables, an error word).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; the return value reports
+ *     argument checks and launch errors only.  No call allocates memory except
+ *     oq_layer_create.
+ *   - Faults the kernels detect themselves (a bounded wait that ran out, an
+ *     index out of range) set the layer's device error word, read back by
+ *     oq_poll_error.
+ *   - Supported shapes: d_in % 32 == 0 with h = (largest power of two dividing
+ *     d_in) in [32, 4096]; d_out % 16 == 0; a_bits in {2,3,4,8}; w_bits in
+ *     {2,3,4}.  Anything else returns OQ_ERR_UNSUPPORTED.  T = 0 is a no-op.
+ *   - Codes are packed per group of 32 consecutive rotated coordinates: the
+ *     group is a little-endian bit stream of 32*b bits stored as b uint32
+ *     words, low word first; code i of the group sits at bits [i*b, (i+1)*b).
+ *     A row of d codes takes d*b/32 words.  Codes are unsigned and ascend with
+ *     the level value.
+ */
+#ifndef ORBITQUANT_H
+#define ORBITQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  OQ_OK = 0,
+  OQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer     */
+  OQ_ERR_UNSUPPORTED = 2,   /* shape or bit width outside the supported set  */
+  OQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed          */
+  OQ_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out (device word) */
+  OQ_ERR_NOMEM = 5,         /* oq_layer_create could not allocate            */
+  OQ_ERR_DEVICE = 6         /* a kernel's own bounds check fired             */
+} oq_status;
+
+enum { OQ_DTYPE_F32 = 0, OQ_DTYPE_BF16 = 1 };
+
+/* Layer / codebook flags. */
+enum {
+  OQ_FLAG_SIGNS = 1,              /* Rademacher signs D_j before each block
+                                     Hadamard (pith Supplementary A);
+                                     off by default                          */
+  OQ_FLAG_GAUSSIAN_MARGINAL = 2   /* design the codebook on N(0, 1/d) (pith
+                                     Figure 2) instead of the exact sphere
+                                     marginal f_d                            */
+};
+
+/*
+ * oq_codebook_build -- the Lloyd-Max codebook C_{d,b} (gecl notes Method 3;
+ * pith Figure 2: one codebook per input dimension and bit width, built
+ * offline without data).  Host-only; needs no GPU.
+ *   d      input dimension (>= 3); the marginal is that of one coordinate of
+ *          a uniform point on the unit sphere S^{d-1},
+ *          f_d(t) = Gamma(d/2)/(sqrt(pi) Gamma((d-1)/2)) (1-t^2)^((d-3)/2),
+ *          or N(0, 1/d) with OQ_FLAG_GAUSSIAN_MARGINAL.
+ *   bits   1..8; the codebook has L = 2^bits levels.
+ *   out    caller-owned; receives ascending levels[0..L), the L-1 midpoint
+ *          thresholds, the designed MSE per coordinate (units of the unit-norm
+ *          coordinate) and the solver's iteration count.
+ * Deterministic.  Results are cached per (d, bits, flags) inside the library.
+ * Errors: OQ_ERR_INVALID_ARG for a null `out` or d < 3; OQ_ERR_UNSUPPORTED for
+ * bits outside 1..8.
+ */
+typedef struct {
+  int32_t d, bits, flags, iterations;
+  double levels[256];
+  double thresholds[255];
+  double mse;
+} oq_codebook;
+
+oq_status oq_codebook_build(int32_t d, int32_t bits, int32_t flags, oq_codebook* out);
+
+/*
+ * oq_rotation_build -- the seeded rotation's random parts, host-only (needs no
+ * GPU).  The permutation pi of RPBH (gecl notes Method 4; pith Supplementary
+ * A, y = P_pi x) as a gather: rotated position i takes input channel perm[i].
+ * Drawn with SplitMix64(seed) driving a descending Fisher-Yates shuffle
+ * (j = high 64 bits of next() * (i + 1), i = d-1 .. 1); the pages fix no
+ * generator.  With OQ_FLAG_SIGNS in `flags` and a non-null `signs`, also the
+ * Rademacher signs D_j of pith Supplementary A by rotated position (+1/-1,
+ * -1 when bit 63 of the next draw is set), drawn after the shuffle.
+ *   perm   caller-owned host array of d entries.
+ *   signs  caller-owned host array of d entries, or NULL.
+ * Errors: OQ_ERR_INVALID_ARG for d < 1 or a null perm.
+ */
+oq_status oq_rotation_build(int32_t d, uint64_t seed, int32_t flags, uint32_t* perm, int8_t* signs);
+
+/*
+ * oq_layer_create -- a layer's shared rotation and codebooks.  Builds the
+ * seeded permutation pi (SplitMix64(seed) driving a descending Fisher-Yates
+ * shuffle; the pages fix no generator), optional signs, both codebooks, and
+ * uploads the device tables.  Allocates device memory on the current device.
+ * `*out` is library-owned; release it with oq_layer_destroy.
+ * Errors: OQ_ERR_INVALID_ARG (null out), OQ_ERR_UNSUPPORTED (shape/bits),
+ * OQ_ERR_NOMEM / OQ_ERR_CUDA (allocation or upload failed).
+ */
+typedef struct oq_layer oq_layer;
+
+oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_bits,
+                          int32_t w_bits, int32_t flags, oq_layer** out);
+void oq_layer_destroy(oq_layer* layer);
+
+typedef struct {
+  int32_t d_in, d_out, h, k, a_bits, w_bits, flags, reserved;
+  uint64_t seed;
+  int64_t a_words_per_row;   /* d_in * a_bits / 32 */
+  int64_t w_words_per_row;   /* d_in * w_bits / 32 */
+  double a_scale, w_scale;   /* fp16 decode scale of each codebook's levels */
+} oq_layer_info;
+
+oq_status oq_layer_get_info(const oq_layer* layer, oq_layer_info* out);
+
+/* Host copy of the permutation as a gather: rotated position i takes input
+ * channel perm[i].  `perm` is a caller-owned host array of d_in entries. */
+oq_status oq_layer_get_perm(const oq_layer* layer, uint32_t* perm);
+
+/*
+ * oq_rotate_quantize -- online activation codec (gecl notes Method 1, 2, 4):
+ *   s[t] = ||x[t]||_2,  u = R x[t] / s[t],  codes[t, i] = #{j : t_j < u_i}.
+ *   x      device [T, d_in], bf16 (OQ_DTYPE_BF16) or fp32 (OQ_DTYPE_F32).
+ *   codes  device [T, d_in*a_bits/32] uint32, packed as described above.
+ *   s      device [T] fp32.
+ * A token of zeros gets s = 0 and every code = 2^(a_bits-1) - 1.
+ */
+oq_status oq_rotate_quantize(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
+                             uint32_t* codes, float* s, void* stream);
+
+/*
+ * oq_weight_prepare -- offline weight rows (hotpaper.ai abstract: the same
+ * quantizer extended to weight rows, rotation absorbed; gecl notes Method 2):
+ *   r[o] = ||W[o]||_2, Wcodes[o] = codes of R W[o] / r[o] with the weight
+ *   codebook C_{d_in, w_bits}.
+ *   W       device [d_out, d_in], fp32 or bf16.
+ *   Wcodes  device [d_out, d_in*w_bits/32] uint32.
+ *   r       device [d_out] fp32.
+ */
+oq_status oq_weight_prepare(const oq_layer* layer, const void* W, int32_t W_dtype,
+                            uint32_t* Wcodes, float* r, void* stream);
+
+/*
+ * oq_linear -- codebook contraction in the shared rotated basis with the
+ * magnitudes restored (llmdb.app Mathematical Formulation; gecl notes
+ * Method 1-2; pith Figure 2):
+ *   y[t, o] = s[t] r[o] sum_i C_w[Wcodes[o, i]] C_a[codes[t, i]]
+ *   codes, s   from oq_rotate_quantize; Wcodes, r from oq_weight_prepare.
+ *   y          device [T, d_out] fp32.
+ * Runs on the tcgen05 tensor cores: both operands are decoded to fp16 levels
+ * (scaled per codebook for exact-as-possible fp16 values), accumulated in
+ * fp32 in tensor memory, and rescaled in the epilogue.
+ */
+oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s, int64_t T,
+                    const uint32_t* Wcodes, const float* r, float* y, void* stream);
+
+/*
+ * oq_linear_fused -- x -> y in one call: the rotate-quantize step produces
+ * the A operand of the contraction (same results as oq_rotate_quantize
+ * followed by oq_linear).  `workspace` is caller-owned device scratch of at
+ * least oq_linear_fused_workspace_size(layer, T) bytes (the packed
+ * activation codes and norms); it may be reused between calls on one stream.
+ */
+size_t oq_linear_fused_workspace_size(const oq_layer* layer, int64_t T);
+oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
+                          const uint32_t* Wcodes, const float* r, float* y,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Reads and clears the layer's device error word.  Synchronizes the device.
+ * Returns OQ_OK, OQ_ERR_TIMEOUT or OQ_ERR_DEVICE. */
+oq_status oq_poll_error(const oq_layer* layer);
+
+/* Message for the last error on the calling thread ("" if none). */
+const char* oq_last_error(void);
+const char* oq_status_string(oq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ORBITQUANT_H */

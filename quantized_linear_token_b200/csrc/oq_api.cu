@@ -1,0 +1,308 @@
+// C-ABI entry points of liborbitquant (declared in include/orbitquant.h):
+// argument checks, the layer object (permutation, codebooks, device tables)
+// and dispatch to the kernels.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "oq_internal.h"
+
+namespace oq {
+
+static thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+static oq_status fail(oq_status st, const std::string& msg) {
+  set_error(msg);
+  return st;
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static oq_status cuda_check(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return OQ_OK;
+  return fail(e == cudaErrorMemoryAllocation ? OQ_ERR_NOMEM : OQ_ERR_CUDA,
+              std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+static void scaled_thresholds(const oq_codebook& cb, int h, float* thr) {
+  const int n = 1 << (cb.bits - 1);
+  const double sh = std::sqrt((double)h);
+  for (int k = 0; k < 128; ++k) thr[k] = INFINITY;
+  // positive thresholds tau_1..tau_{n-1} = thresholds[n .. 2n-2]
+  for (int k = 1; k < n; ++k) thr[k - 1] = (float)(sh * cb.thresholds[n - 1 + k]);
+}
+
+}  // namespace oq
+
+using namespace oq;
+
+extern "C" {
+
+const char* oq_last_error(void) { return g_last_error.c_str(); }
+
+const char* oq_status_string(oq_status st) {
+  switch (st) {
+    case OQ_OK: return "ok";
+    case OQ_ERR_INVALID_ARG: return "invalid argument";
+    case OQ_ERR_UNSUPPORTED: return "unsupported shape or bit width";
+    case OQ_ERR_CUDA: return "CUDA error";
+    case OQ_ERR_TIMEOUT: return "device wait timed out";
+    case OQ_ERR_NOMEM: return "out of memory";
+    case OQ_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+oq_status oq_codebook_build(int32_t d, int32_t bits, int32_t flags, oq_codebook* out) {
+  if (!out) return fail(OQ_ERR_INVALID_ARG, "oq_codebook_build: out is null");
+  if (d < 3) return fail(OQ_ERR_INVALID_ARG, "oq_codebook_build: d must be >= 3");
+  if (bits < 1 || bits > 8) return fail(OQ_ERR_UNSUPPORTED, "oq_codebook_build: bits must be 1..8");
+  return get_codebook(d, bits, flags, out);
+}
+
+oq_status oq_rotation_build(int32_t d, uint64_t seed, int32_t flags, uint32_t* perm, int8_t* signs) {
+  if (d < 1 || !perm) return fail(OQ_ERR_INVALID_ARG, "oq_rotation_build: d < 1 or perm is null");
+  std::vector<uint32_t> p;
+  std::vector<int8_t> sg;
+  const bool want_signs = (flags & OQ_FLAG_SIGNS) && signs;
+  make_permutation(d, seed, p, want_signs ? &sg : nullptr);
+  std::memcpy(perm, p.data(), (size_t)d * sizeof(uint32_t));
+  if (want_signs) std::memcpy(signs, sg.data(), (size_t)d);
+  return OQ_OK;
+}
+
+static oq_status check_shape(int32_t d_in, int32_t d_out, int32_t a_bits, int32_t w_bits) {
+  if (d_in <= 0 || d_out <= 0) return fail(OQ_ERR_INVALID_ARG, "dimensions must be positive");
+  if (d_in % 32) return fail(OQ_ERR_UNSUPPORTED, "d_in must be a multiple of 32");
+  if (d_in > 65535) return fail(OQ_ERR_UNSUPPORTED, "d_in must be < 65536");
+  const int h = d_in & -d_in;
+  if (h < 32 || h > 4096) return fail(OQ_ERR_UNSUPPORTED, "block size h must be in [32, 4096]");
+  if (d_out % 16) return fail(OQ_ERR_UNSUPPORTED, "d_out must be a multiple of 16");
+  if (!(a_bits == 2 || a_bits == 3 || a_bits == 4 || a_bits == 8))
+    return fail(OQ_ERR_UNSUPPORTED, "a_bits must be 2, 3, 4 or 8");
+  if (!(w_bits == 2 || w_bits == 3 || w_bits == 4)) return fail(OQ_ERR_UNSUPPORTED, "w_bits must be 2, 3 or 4");
+  return OQ_OK;
+}
+
+void oq_layer_destroy(oq_layer* L) {
+  if (!L) return;
+  cudaFree(L->d_gather_a);
+  cudaFree(L->d_signmask);
+  cudaFree(L->d_levels_a);
+  cudaFree(L->d_levels_w);
+  cudaFree(L->d_error);
+  delete L;
+}
+
+oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_bits, int32_t w_bits,
+                          int32_t flags, oq_layer** out) {
+  if (!out) return fail(OQ_ERR_INVALID_ARG, "oq_layer_create: out is null");
+  *out = nullptr;
+  oq_status st = check_shape(d_in, d_out, a_bits, w_bits);
+  if (st != OQ_OK) return st;
+  if (flags & ~(OQ_FLAG_SIGNS | OQ_FLAG_GAUSSIAN_MARGINAL)) return fail(OQ_ERR_INVALID_ARG, "unknown flag bits");
+
+  oq_layer* L = new (std::nothrow) oq_layer();
+  if (!L) return fail(OQ_ERR_NOMEM, "host allocation failed");
+  L->d_in = d_in;
+  L->d_out = d_out;
+  L->h = d_in & -d_in;
+  L->k = d_in / L->h;
+  L->log_h = 0;
+  while ((1 << L->log_h) < L->h) ++L->log_h;
+  L->a_bits = a_bits;
+  L->w_bits = w_bits;
+  L->flags = flags;
+  L->seed = seed;
+  cudaGetDevice(&L->device);
+
+  if ((st = get_codebook(d_in, a_bits, flags, &L->cb_a)) != OQ_OK ||
+      (st = get_codebook(d_in, w_bits, flags, &L->cb_w)) != OQ_OK) {
+    delete L;
+    return st;
+  }
+  const bool signed_rot = (flags & OQ_FLAG_SIGNS) != 0;
+  make_permutation(d_in, seed, L->perm_host, signed_rot ? &L->signs_host : nullptr);
+  std::vector<uint16_t> gather;
+  std::vector<uint32_t> signmask;
+  rq_build_gather(d_in, L->h, L->perm_host, signed_rot ? &L->signs_host : nullptr, gather, signmask);
+
+  L->a_scale = choose_fp16_scale(L->cb_a);
+  L->w_scale = choose_fp16_scale(L->cb_w);
+  uint16_t lv_a[256] = {0}, lv_w[256] = {0};
+  for (int i = 0; i < (1 << a_bits); ++i) lv_a[i] = f64_to_f16_bits(L->a_scale * L->cb_a.levels[i]);
+  for (int i = 0; i < (1 << w_bits); ++i) lv_w[i] = f64_to_f16_bits(L->w_scale * L->cb_w.levels[i]);
+  scaled_thresholds(L->cb_a, L->h, L->thr_a);
+  scaled_thresholds(L->cb_w, L->h, L->thr_w);
+
+  st = cuda_check(cudaMalloc(&L->d_gather_a, gather.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
+  if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_gather_a, gather.data(), gather.size() * sizeof(uint16_t),
+                                              cudaMemcpyHostToDevice), "upload gather");
+  if (st == OQ_OK && signed_rot) {
+    st = cuda_check(cudaMalloc(&L->d_signmask, signmask.size() * sizeof(uint32_t)), "cudaMalloc(signs)");
+    if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_signmask, signmask.data(), signmask.size() * sizeof(uint32_t),
+                                                cudaMemcpyHostToDevice), "upload signs");
+  }
+  if (st == OQ_OK) st = cuda_check(cudaMalloc(&L->d_levels_a, sizeof(lv_a)), "cudaMalloc(levels)");
+  if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_levels_a, lv_a, sizeof(lv_a), cudaMemcpyHostToDevice), "upload levels");
+  if (st == OQ_OK) st = cuda_check(cudaMalloc(&L->d_levels_w, sizeof(lv_w)), "cudaMalloc(levels)");
+  if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_levels_w, lv_w, sizeof(lv_w), cudaMemcpyHostToDevice), "upload levels");
+  if (st == OQ_OK) st = cuda_check(cudaMalloc(&L->d_error, sizeof(int)), "cudaMalloc(error word)");
+  if (st == OQ_OK) st = cuda_check(cudaMemset(L->d_error, 0, sizeof(int)), "clear error word");
+  if (st != OQ_OK) {
+    oq_layer_destroy(L);
+    return st;
+  }
+  *out = L;
+  return OQ_OK;
+}
+
+oq_status oq_layer_get_info(const oq_layer* L, oq_layer_info* out) {
+  if (!L || !out) return fail(OQ_ERR_INVALID_ARG, "oq_layer_get_info: null argument");
+  std::memset(out, 0, sizeof(*out));
+  out->d_in = L->d_in;
+  out->d_out = L->d_out;
+  out->h = L->h;
+  out->k = L->k;
+  out->a_bits = L->a_bits;
+  out->w_bits = L->w_bits;
+  out->flags = L->flags;
+  out->seed = L->seed;
+  out->a_words_per_row = (int64_t)L->d_in * L->a_bits / 32;
+  out->w_words_per_row = (int64_t)L->d_in * L->w_bits / 32;
+  out->a_scale = L->a_scale;
+  out->w_scale = L->w_scale;
+  return OQ_OK;
+}
+
+oq_status oq_layer_get_perm(const oq_layer* L, uint32_t* perm) {
+  if (!L || !perm) return fail(OQ_ERR_INVALID_ARG, "oq_layer_get_perm: null argument");
+  std::memcpy(perm, L->perm_host.data(), L->perm_host.size() * sizeof(uint32_t));
+  return OQ_OK;
+}
+
+static oq_status check_rows_input(const void* x, int32_t dtype, const char* who) {
+  if (!x) return fail(OQ_ERR_INVALID_ARG, std::string(who) + ": input is null");
+  if (dtype != OQ_DTYPE_BF16 && dtype != OQ_DTYPE_F32)
+    return fail(OQ_ERR_INVALID_ARG, std::string(who) + ": dtype must be OQ_DTYPE_BF16 or OQ_DTYPE_F32");
+  if (!aligned(x, 16)) return fail(OQ_ERR_INVALID_ARG, std::string(who) + ": input must be 16-byte aligned");
+  return OQ_OK;
+}
+
+static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t rows, int bits, const float* thr,
+                    uint32_t* codes, float* norms, void* stream) {
+  RQArgs a;
+  a.src = x;
+  a.src_dtype = dtype;
+  a.rows = rows;
+  a.d = L->d_in;
+  a.h = L->h;
+  a.log_h = L->log_h;
+  a.bits = bits;
+  a.gather = L->d_gather_a;
+  a.signmask = L->d_signmask;
+  a.thr = thr;
+  a.codes = codes;
+  a.norms = norms;
+  a.err = L->d_error;
+  return rq_launch(a, stream);
+}
+
+oq_status oq_rotate_quantize(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint32_t* codes,
+                             float* s, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize: layer is null");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize: T < 0");
+  if (T == 0) return OQ_OK;
+  oq_status st = check_rows_input(x, x_dtype, "oq_rotate_quantize");
+  if (st != OQ_OK) return st;
+  if (!codes || !s || !aligned(codes, 16) || !aligned(s, 4))
+    return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize: codes (16-byte) / s (4-byte) pointers invalid");
+  return rq(L, x, x_dtype, T, L->a_bits, L->thr_a, codes, s, stream);
+}
+
+oq_status oq_weight_prepare(const oq_layer* L, const void* W, int32_t W_dtype, uint32_t* Wcodes, float* r,
+                            void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_weight_prepare: layer is null");
+  oq_status st = check_rows_input(W, W_dtype, "oq_weight_prepare");
+  if (st != OQ_OK) return st;
+  if (!Wcodes || !r || !aligned(Wcodes, 16) || !aligned(r, 4))
+    return fail(OQ_ERR_INVALID_ARG, "oq_weight_prepare: Wcodes (16-byte) / r (4-byte) pointers invalid");
+  return rq(L, W, W_dtype, L->d_out, L->w_bits, L->thr_w, Wcodes, r, stream);
+}
+
+static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T,
+                             const uint32_t* Wcodes, const float* r, float* y, void* stream) {
+  GemmArgs g;
+  g.a_codes = codes;
+  g.b_codes = Wcodes;
+  g.a_scale = s;
+  g.b_scale = r;
+  g.a_levels = L->d_levels_a;
+  g.b_levels = L->d_levels_w;
+  g.out_scale = (float)(1.0 / (L->a_scale * L->w_scale));
+  g.y = y;
+  g.M = T;
+  g.N = L->d_out;
+  g.K = L->d_in;
+  g.a_bits = L->a_bits;
+  g.b_bits = L->w_bits;
+  g.err = L->d_error;
+  return gemm_launch(g, stream);
+}
+
+oq_status oq_linear(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T, const uint32_t* Wcodes,
+                    const float* r, float* y, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear: layer is null");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear: T < 0");
+  if (T == 0) return OQ_OK;
+  if (!codes || !s || !Wcodes || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear: null pointer");
+  if (!aligned(codes, 16) || !aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(s, 4) || !aligned(r, 16))
+    return fail(OQ_ERR_INVALID_ARG, "oq_linear: misaligned pointer");
+  return linear_impl(L, codes, s, T, Wcodes, r, y, stream);
+}
+
+size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
+  if (!L || T <= 0) return 0;
+  const size_t codes = (size_t)T * ((size_t)L->d_in * L->a_bits / 32) * 4;
+  return ((codes + 255) & ~(size_t)255) + (size_t)T * 4;
+}
+
+oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                          const float* r, float* y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: layer is null");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: T < 0");
+  if (T == 0) return OQ_OK;
+  oq_status st = check_rows_input(x, x_dtype, "oq_linear_fused");
+  if (st != OQ_OK) return st;
+  if (!Wcodes || !r || !y || !workspace) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: null pointer");
+  if (!aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(r, 16) || !aligned(workspace, 256))
+    return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: misaligned pointer (workspace needs 256 bytes)");
+  if (workspace_bytes < oq_linear_fused_workspace_size(L, T))
+    return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
+  uint32_t* codes = static_cast<uint32_t*>(workspace);
+  const size_t cbytes = (size_t)T * ((size_t)L->d_in * L->a_bits / 32) * 4;
+  float* s = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + ((cbytes + 255) & ~(size_t)255));
+  st = rq(L, x, x_dtype, T, L->a_bits, L->thr_a, codes, s, stream);
+  if (st != OQ_OK) return st;
+  return linear_impl(L, codes, s, T, Wcodes, r, y, stream);
+}
+
+oq_status oq_poll_error(const oq_layer* L) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_poll_error: layer is null");
+  oq_status st = cuda_check(cudaDeviceSynchronize(), "oq_poll_error: synchronize");
+  if (st != OQ_OK) return st;
+  int word = 0;
+  st = cuda_check(cudaMemcpy(&word, L->d_error, sizeof(int), cudaMemcpyDeviceToHost), "oq_poll_error: read");
+  if (st != OQ_OK) return st;
+  if (word) cudaMemset(L->d_error, 0, sizeof(int));
+  if (word & OQ_DEVERR_TIMEOUT) return fail(OQ_ERR_TIMEOUT, "a kernel's bounded wait ran out");
+  if (word & OQ_DEVERR_BOUNDS) return fail(OQ_ERR_DEVICE, "a kernel's bounds check fired");
+  return OQ_OK;
+}
+
+}  // extern "C"

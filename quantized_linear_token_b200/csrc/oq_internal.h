@@ -1,0 +1,79 @@
+// Internal declarations shared by the library's host and device sources.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "orbitquant.h"
+
+// error word bits written by kernels into the layer's device word
+#define OQ_DEVERR_TIMEOUT 1
+#define OQ_DEVERR_BOUNDS 2
+
+struct oq_layer {
+  int d_in, d_out, h, k, log_h, a_bits, w_bits, flags;
+  uint64_t seed;
+  int device;
+  oq_codebook cb_a, cb_w;
+  double a_scale, w_scale;            // fp16 decode scale per codebook
+  std::vector<uint32_t> perm_host;    // gather: rotated position i <- channel perm[i]
+  std::vector<int8_t> signs_host;     // +-1 by rotated position (OQ_FLAG_SIGNS)
+  // device tables (owned)
+  uint16_t* d_gather_a;               // rotate-quantize gather offsets, kernel order
+  uint32_t* d_signmask;               // sign bits in kernel order, or null
+  uint16_t* d_levels_a;               // fp16 bits of a_scale * activation levels
+  uint16_t* d_levels_w;               // fp16 bits of w_scale * weight levels
+  int* d_error;                       // device error word
+  float thr_a[128];                   // sqrt(h) * positive thresholds, +inf padded
+  float thr_w[128];
+};
+
+namespace oq {
+
+void set_error(const std::string& msg);
+
+// host math (oq_host.cpp)
+void make_permutation(int d, uint64_t seed, std::vector<uint32_t>& perm, std::vector<int8_t>* signs);
+oq_status design_codebook(int d, int bits, int flags, oq_codebook* out);
+oq_status get_codebook(int d, int bits, int flags, oq_codebook* out);
+uint16_t f64_to_f16_bits(double v);
+double f16_bits_to_f64(uint16_t h);
+double choose_fp16_scale(const oq_codebook& cb);
+
+// rotate + quantize launch (oq_rotate_quantize.cu): rows of `src` -> packed codes + norms
+struct RQArgs {
+  const void* src;       // [rows, d] bf16 or fp32
+  int src_dtype;
+  int64_t rows;
+  int d, h, log_h, bits;
+  const uint16_t* gather;    // per-thread gather offsets (kernel order)
+  const uint32_t* signmask;  // or null
+  const float* thr;          // host array of 128 scaled thresholds
+  uint32_t* codes;           // [rows, d*bits/32]
+  float* norms;              // [rows]
+  int* err;
+};
+int rq_elems_per_thread(int h);
+// kernel-order gather table for a permutation (and optional signs)
+void rq_build_gather(int d, int h, const std::vector<uint32_t>& perm, const std::vector<int8_t>* signs,
+                     std::vector<uint16_t>& gather, std::vector<uint32_t>& signmask);
+oq_status rq_launch(const RQArgs& a, void* stream);
+
+// codebook contraction launch (oq_gemm.cu)
+struct GemmArgs {
+  const uint32_t* a_codes;   // [M, K*a_bits/32]
+  const uint32_t* b_codes;   // [N, K*b_bits/32]
+  const float* a_scale;      // [M] per-row magnitude s
+  const float* b_scale;      // [N] per-row magnitude r
+  const uint16_t* a_levels;  // fp16 bits, 2^a_bits
+  const uint16_t* b_levels;  // fp16 bits, 2^b_bits
+  float out_scale;           // 1 / (alpha_a alpha_w)
+  float* y;                  // [M, N] fp32
+  int64_t M;
+  int N, K, a_bits, b_bits;
+  int* err;
+};
+oq_status gemm_launch(const GemmArgs& g, void* stream);
+
+}  // namespace oq

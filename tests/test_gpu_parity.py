@@ -1,0 +1,182 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle on the
+same seeded inputs (bounds in tests/parity.py).  Needs a B200."""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle as O
+from quantized_linear_token_b200 import workloads as W
+
+from parity import check_codes, check_linear, to_numpy_u32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def env():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_linear_token_b200 import build
+    build.build()
+    from quantized_linear_token_b200 import binding as B
+    B.load_library()
+    return torch, B
+
+
+def _x_tensor(torch, x_np):
+    if x_np.dtype == np.uint16:
+        return torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).cuda(), O.bf16_bits_to_f64(x_np)
+    return torch.from_numpy(x_np).cuda(), x_np.astype(np.float64)
+
+
+def _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, flags=0, seed=0, w_rows=None, y_rows=None,
+               label=""):
+    torch, B = env
+    layer = B.oq_layer_create(d_in, d_out, seed, a_bits, w_bits, flags)
+    gauss = bool(flags & B.OQ_FLAG_GAUSSIAN_MARGINAL)
+    cb_a, cb_w = O.lloyd_max(d_in, a_bits, gauss), O.lloyd_max(d_in, w_bits, gauss)
+    h = O.hadamard_block_size(d_in)
+    perm = O.rpbh_permutation(d_in, seed)
+    signs = O.rademacher_signs(d_in, seed) if flags & B.OQ_FLAG_SIGNS else None
+    np.testing.assert_array_equal(layer.perm().astype(np.int64), perm)
+
+    x_t, x64 = _x_tensor(torch, x_np)
+    W_t = torch.from_numpy(Wm).cuda()
+    Wc, r = B.oq_weight_prepare(layer, W_t)
+    codes, s = B.oq_rotate_quantize(layer, x_t)
+    y = B.oq_linear(layer, codes, s, Wc, r)
+    yf = B.oq_linear_fused(layer, x_t, Wc, r)
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+
+    # weight rows (sampled for large layers)
+    wr = np.arange(d_out) if w_rows is None else w_rows
+    Wc_np, r_np = to_numpy_u32(Wc), r.cpu().numpy()
+    check_codes(Wc_np[wr], Wm[wr].astype(np.float64), perm, h, cb_w, w_bits, signs, r_np[wr], label + " W")
+    # activations, all rows
+    codes_np, s_np = to_numpy_u32(codes), s.cpu().numpy()
+    _, _, st = check_codes(codes_np, x64, perm, h, cb_a, a_bits, signs, s_np, label + " x")
+    # contraction on the GPU's own codes
+    y_np, yf_np = y.cpu().numpy(), yf.cpu().numpy()
+    lin = check_linear(y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, label + " y", rows=y_rows)
+    # the fused call computes the same codes, so the same y
+    np.testing.assert_array_equal(yf_np, y_np)
+    return st, lin
+
+
+CASES = [
+    # key,        d_in,  d_out, a, w, T,   recipe source
+    ("pr1", 256, 256, 4, 4, 64),
+    ("dit_image", 3072, 3072, 4, 4, 300),
+    ("dit_mlp_up", 3072, 12288, 4, 2, 200),
+    ("dit_mlp_down", 12288, 3072, 4, 2, 130),
+    ("video_w4a4", 5120, 5120, 4, 4, 150),
+    ("video_w3a3", 5120, 5120, 3, 3, 150),
+    ("stress_w2a4", 13824, 5120, 4, 2, 129),
+    ("stress_w3a3", 13824, 5120, 3, 3, 129),
+    ("stress_w4a4", 13824, 5120, 4, 4, 129),
+    ("stress_w4a8", 13824, 5120, 8, 4, 129),
+]
+
+
+def _inputs(key, d_in, d_out, T):
+    if key == "pr1":
+        wl = W.WORKLOADS["pr1"]
+        return W.activations(wl, d_in, T), W.weights(wl, wl.layers[0])
+    if key.startswith("dit_image"):
+        wl = W.WORKLOADS["dit_image"]
+        return W.activations(wl, d_in, T), W.weights(wl, wl.layers[0])
+    if key.startswith("dit_mlp"):
+        wl = W.WORKLOADS["dit_mlp"]
+        lay = wl.layers[0] if key.endswith("up") else wl.layers[1]
+        return W.activations(wl, d_in, T, gelu=key.endswith("down"), stream=int(key.endswith("down"))), \
+            W.weights(wl, lay)
+    if key.startswith("video"):
+        wl = W.WORKLOADS["video_dit"]
+        lay = wl.layers[0] if key.endswith("w4a4") else wl.layers[1]
+        return W.activations(wl, d_in, T), W.weights(wl, lay)
+    wl = W.WORKLOADS["stress"]
+    lay = [l for l in wl.layers if key.endswith(l.name)][0]
+    return W.activations(wl, d_in, T), W.weights(wl, lay)
+
+
+@pytest.mark.parametrize("key,d_in,d_out,a_bits,w_bits,T", CASES, ids=[c[0] for c in CASES])
+def test_workload_parity(env, key, d_in, d_out, a_bits, w_bits, T):
+    x_np, Wm = _inputs(key, d_in, d_out, T)
+    rng = np.random.default_rng(7)
+    w_rows = None if d_out <= 1024 else np.unique(np.concatenate(
+        [np.arange(64), np.arange(d_out - 64, d_out), rng.choice(d_out, 128, replace=False)]))
+    st, lin = _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, w_rows=w_rows, label=key)
+    print(key, st, lin)
+
+
+EDGE = [
+    # d_in, d_out, a, w, T, flags
+    (32, 16, 4, 4, 1, 0),          # h = 32, one block, one token
+    (96, 48, 2, 2, 37, 0),         # h = 32, k = 3, single-pass kernel, ragged everything
+    (192, 80, 3, 3, 129, 0),       # h = 64, k = 3, ragged N (80)
+    (128, 128, 8, 4, 5, 0),        # h = 128, 8-bit activations
+    (640, 272, 4, 3, 257, 1),      # h = 128, k = 5, Rademacher signs
+    (1024, 256, 4, 4, 130, 2),     # Gaussian-marginal codebook
+    (2048, 128, 4, 2, 70, 0),      # h = 2048 (64 per thread, two passes)
+    (6144, 512, 3, 4, 33, 0),      # h = 2048, k = 3
+]
+
+
+@pytest.mark.parametrize("d_in,d_out,a_bits,w_bits,T,flags", EDGE)
+def test_edge_shapes(env, d_in, d_out, a_bits, w_bits, T, flags):
+    x_np = W.custom_activations(T, d_in, seed=d_in + T, outliers=min(4, d_in // 8))
+    Wm = W.custom_weights(d_out, d_in, seed=d_out)
+    _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, flags=flags, seed=3, label=f"edge{d_in}x{d_out}")
+
+
+def test_degenerate_tokens(env):
+    # a zero token (s = 0, every code L/2 - 1, y = 0) and tokens with very
+    # small and very large norms
+    torch, B = env
+    d_in, d_out, T = 256, 128, 6
+    x = W.bf16_bits_to_f32(W.custom_activations(T, d_in, seed=5))
+    x[1] = 0.0
+    x[2] *= 1e-12
+    x[3] *= 1e12
+    x[4] = 0.0
+    x[4, 17] = -3.0                      # one-hot token
+    x_np = W.f32_to_bf16_bits(x)
+    Wm = W.custom_weights(d_out, d_in, seed=9)
+    _run_layer(env, d_in, d_out, 4, 4, x_np, Wm, label="degenerate")
+    layer = B.oq_layer_create(d_in, d_out, 0, 4, 4, 0)
+    xt = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).cuda()
+    codes, s = B.oq_rotate_quantize(layer, xt)
+    c = O.unpack_codes(to_numpy_u32(codes), 4, d_in)
+    assert float(s[1]) == 0.0 and np.all(c[1] == 7)
+
+
+def test_empty_batch(env):
+    torch, B = env
+    layer = B.oq_layer_create(256, 256, 0, 4, 4, 0)
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    Wc, r = B.oq_weight_prepare(layer, torch.zeros((256, 256), device="cuda"))
+    codes, s = B.oq_rotate_quantize(layer, x)
+    y = B.oq_linear(layer, codes, s, Wc, r)
+    assert codes.shape == (0, 32) and y.shape == (0, 256)
+    B.oq_poll_error(layer)
+
+
+def test_bench_config_full_size(env):
+    """The image-DiT projection at its full size (9216 tokens, 3072 -> 3072,
+    W4A4), in the launch configuration the benchmark times: every code and
+    norm checked, y checked on 256 sampled rows."""
+    torch, B = env
+    wl = W.WORKLOADS["dit_image"]
+    lay = wl.layers[0]
+    x_np = W.activations(wl, lay.d_in)
+    Wm = W.weights(wl, lay)
+    rows = np.random.default_rng(0).choice(wl.tokens, 256, replace=False)
+    rows.sort()
+    w_rows = np.arange(0, lay.d_out, 7)
+    st, lin = _run_layer(env, lay.d_in, lay.d_out, lay.a_bits, lay.w_bits, x_np, Wm, w_rows=w_rows,
+                         y_rows=rows, label="dit_image full")
+    print("full", st, lin)
