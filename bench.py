@@ -42,6 +42,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_image")
+    ap.add_argument("--tokens", type=int, default=0, help="override the workload's token count (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -170,8 +171,8 @@ def run_ours(args):
 
     wl = W.WORKLOADS[args.workload]
     lay = wl.layers[0]
-    T, d, dout = wl.tokens, lay.d_in, lay.d_out
-    x_np = W.activations(wl, d)
+    T, d, dout = (args.tokens or wl.tokens), lay.d_in, lay.d_out
+    x_np = W.activations(wl, d, tokens=T)
     Wm = W.weights(wl, lay)
     x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
     layer = B.oq_layer_create(d, dout, W.ROTATION_SEED, lay.a_bits, lay.w_bits)

@@ -137,6 +137,8 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   uint16_t lv_a[256] = {0}, lv_w[256] = {0};
   for (int i = 0; i < (1 << a_bits); ++i) lv_a[i] = f64_to_f16_bits(L->a_scale * L->cb_a.levels[i]);
   for (int i = 0; i < (1 << w_bits); ++i) lv_w[i] = f64_to_f16_bits(L->w_scale * L->cb_w.levels[i]);
+  std::memcpy(L->lv_a, lv_a, sizeof(lv_a));
+  std::memcpy(L->lv_w, lv_w, sizeof(lv_w));
   scaled_thresholds(L->cb_a, L->h, L->thr_a);
   scaled_thresholds(L->cb_w, L->h, L->thr_w);
 
@@ -244,6 +246,8 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
   g.b_scale = r;
   g.a_levels = L->d_levels_a;
   g.b_levels = L->d_levels_w;
+  g.a_levels_host = L->lv_a;
+  g.b_levels_host = L->lv_w;
   g.out_scale = (float)(1.0 / (L->a_scale * L->w_scale));
   g.y = y;
   g.M = T;

@@ -2,19 +2,22 @@
 // Takeaway 3: a native non-uniform low-bit GEMM in the shared rotated basis):
 //   y[m, n] = a_scale[m] b_scale[n] out_scale sum_k LA[A[m, k]] LB[B[n, k]]
 // A and B are packed code matrices (K-major rows); LA, LB are the two
-// codebooks as fp16 (pre-scaled, see oq_host.cpp).
+// codebooks as fp16 values (pre-scaled, see oq_host.cpp).
 //
-// One CTA computes a BM x BN tile of y:
-//   * warps 0-3 decode the codes of each K block (BK = 64) through small
-//     shared-memory tables straight into fp16 operand tiles laid out in the
-//     128-byte-swizzled K-major form that tcgen05 reads (8 codes -> one
-//     16-byte chunk per store);
-//   * warp 4 allocates the tensor-memory accumulator, and one of its threads
-//     issues tcgen05.mma (M = 128, N = BN, K = 16 per instruction) for every
-//     full stage, releasing the stage with tcgen05.commit;
-//   * warps 0-3 then read the fp32 accumulator back (tcgen05.ld) and write
-//     y with the per-row and per-column magnitudes applied.
-// Every mbarrier wait is bounded (see oq_ptx.cuh).
+// Persistent kernel, one CTA per SM, tiles of BM x BN outputs, K blocks of 64:
+//   * warps 0-7 ("decoders") stream the codes of each K block straight from
+//     global memory (one 16-byte load per 32-64 codes, prefetched one K block
+//     ahead) and expand them in registers into fp16 operand tiles in the
+//     128-byte-swizzled K-major layout tcgen05 reads.  The expansion uses
+//     byte-permute (prmt) lookups into codebook tables held in registers:
+//     4-bit codes use the codebook's symmetry (magnitude table + sign byte),
+//     2- and 3-bit codes a full table; 8-bit codes a shared-memory table;
+//   * warp 12 allocates 2 x BN columns of tensor memory (two accumulators)
+//     and one of its threads issues tcgen05.mma (M=128, N=BN, K=16) for each
+//     decoded stage, releasing it with tcgen05.commit;
+//   * warps 8-11 drain the other accumulator (tcgen05.ld), apply
+//     s[m] r[n] / (alpha_a alpha_w) and store y, overlapping the next tile.
+// All mbarrier waits are bounded (oq_ptx.cuh).
 #include <algorithm>
 #include <cstring>
 
@@ -25,65 +28,115 @@ namespace oq {
 namespace {
 
 constexpr int BM = 128, BK = 64, UMMA_K = 16;
+constexpr int NDEC = 256;          // decoder threads (warps 0-7)
+constexpr int EPI_WARP0 = 8;       // epilogue warps 8-11
+constexpr int MMA_WARP = 12;
+constexpr int NTHREADS = 13 * 32;
+constexpr int OS = 4;              // operand stages
 
 struct GemmKParams {
   const uint32_t* a_codes;
   const uint32_t* b_codes;
   const float* a_scale;
   const float* b_scale;
-  const uint16_t* a_levels;
-  const uint16_t* b_levels;
   float out_scale;
   float* y;
   int64_t M;
   int N, K, a_wpr, b_wpr;
+  int n_tiles, nkb;
+  int64_t tiles;
+  uint32_t a_tab[4], b_tab[4];
+  const uint16_t* a_lut8;
   int* err;
 };
 
-// decode tables: one entry per byte of codes (2/4/8 bits) or per 6 bits (3 bits)
-template <int BITS> struct Lut;
-template <> struct Lut<2> { static constexpr int ENTRIES = 256; using T = uint2; };
-template <> struct Lut<3> { static constexpr int ENTRIES = 64; using T = uint32_t; };
-template <> struct Lut<4> { static constexpr int ENTRIES = 256; using T = uint32_t; };
-template <> struct Lut<8> { static constexpr int ENTRIES = 256; using T = uint32_t; };
+// per bit width: 16-byte code parts per row per K block and 8-code chunks per part
+template <int BITS> struct Fmt;
+template <> struct Fmt<2> { static constexpr int QP = 1, CPP = 8; };
+template <> struct Fmt<3> { static constexpr int QP = 2, CPP = 4; };
+template <> struct Fmt<4> { static constexpr int QP = 2, CPP = 4; };
+template <> struct Fmt<8> { static constexpr int QP = 4, CPP = 2; };
 
+// the codes of part q of K block kb of a row (zeros past K)
 template <int BITS>
-__device__ void build_lut(typename Lut<BITS>::T* lut, const uint16_t* lv, int tid, int nthreads) {
-  for (int e = tid; e < Lut<BITS>::ENTRIES; e += nthreads) {
-    if constexpr (BITS == 4) {
-      lut[e] = (uint32_t)lv[e & 15] | ((uint32_t)lv[e >> 4] << 16);
-    } else if constexpr (BITS == 2) {
-      lut[e] = make_uint2((uint32_t)lv[e & 3] | ((uint32_t)lv[(e >> 2) & 3] << 16),
-                          (uint32_t)lv[(e >> 4) & 3] | ((uint32_t)lv[e >> 6] << 16));
-    } else if constexpr (BITS == 3) {
-      lut[e] = (uint32_t)lv[e & 7] | ((uint32_t)lv[e >> 3] << 16);
-    } else {
-      lut[e] = (uint32_t)lv[e];
-    }
+__device__ __forceinline__ uint4 load_part(const uint32_t* row, int kb, int q, int K) {
+  const int k0 = kb * BK + q * (BK / Fmt<BITS>::QP);
+  if (k0 >= K) return make_uint4(0u, 0u, 0u, 0u);
+  if constexpr (BITS == 3) {
+    const uint32_t* p = row + kb * 6 + q * 3;
+    return make_uint4(__ldg(p), __ldg(p + 1), __ldg(p + 2), 0u);
+  } else if constexpr (BITS == 2) {
+    // rows are only 8-byte aligned when K % 64 == 32
+    const uint2* p = reinterpret_cast<const uint2*>(row + kb * 4);
+    const uint2 lo = __ldg(p);
+    const uint2 hi = (k0 + 32 < K) ? __ldg(p + 1) : make_uint2(0u, 0u);
+    return make_uint4(lo.x, lo.y, hi.x, hi.y);
+  } else {
+    return __ldg(reinterpret_cast<const uint4*>(row) + kb * (BITS / 2) + q);
   }
 }
 
-// 8 codes of a row starting at element k (k % 8 == 0) -> 8 fp16 values
+// ---- 8 codes -> 8 fp16 (one 16-byte chunk of the operand tile)
+__device__ __forceinline__ uint4 dec4(uint32_t w, const uint32_t (&t)[4]) {
+  // symmetric codebook: code c >= 8 -> +P[c-8], c < 8 -> -P[7-c]
+  const uint32_t n = ((~w) & 0x88888888u) >> 3;            // 1 per negative code
+  const uint32_t m = (w & 0x77777777u) ^ (n * 7u);         // magnitude index
+  const uint32_t mh = m >> 16, nh = n >> 16;
+  const uint32_t lo_a = __byte_perm(t[0], t[1], m), hi_a = __byte_perm(t[2], t[3], m) | __byte_perm(0x8000u, 0u, n);
+  const uint32_t lo_b = __byte_perm(t[0], t[1], mh), hi_b = __byte_perm(t[2], t[3], mh) | __byte_perm(0x8000u, 0u, nh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+__device__ __forceinline__ uint4 dec2(uint32_t x, const uint32_t (&t)[4]) {
+  // 2-bit fields -> one selector nibble per code; 4-entry table in one register
+  uint32_t y = (x | (x << 8)) & 0x00FF00FFu;
+  y = (y | (y << 4)) & 0x0F0F0F0Fu;
+  y = (y | (y << 2)) & 0x33333333u;
+  const uint32_t yh = y >> 16;
+  const uint32_t lo_a = __byte_perm(t[0], t[0], y), hi_a = __byte_perm(t[1], t[1], y);
+  const uint32_t lo_b = __byte_perm(t[0], t[0], yh), hi_b = __byte_perm(t[1], t[1], yh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+__device__ __forceinline__ uint4 dec3(uint32_t x, const uint32_t (&t)[4]) {
+  // 3-bit fields -> one selector nibble per code; 8-entry table in two registers
+  uint32_t y = (x & 0xFFFu) | ((x & 0xFFF000u) << 4);
+  y = (y & 0x003F003Fu) | ((y & 0x0FC00FC0u) << 2);
+  y = (y & 0x07070707u) | ((y & 0x38383838u) << 1);
+  const uint32_t yh = y >> 16;
+  const uint32_t lo_a = __byte_perm(t[0], t[1], y), hi_a = __byte_perm(t[2], t[3], y);
+  const uint32_t lo_b = __byte_perm(t[0], t[1], yh), hi_b = __byte_perm(t[2], t[3], yh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+__device__ __forceinline__ uint4 dec8(uint32_t w0, uint32_t w1, const uint16_t* lut) {
+  auto pr = [&](uint32_t w, int b) {
+    return (uint32_t)lut[(w >> (8 * b)) & 0xFF] | ((uint32_t)lut[(w >> (8 * b + 8)) & 0xFF] << 16);
+  };
+  return make_uint4(pr(w0, 0), pr(w0, 2), pr(w1, 0), pr(w1, 2));
+}
+
+// chunk j of a part -> 8 fp16
 template <int BITS>
-__device__ __forceinline__ uint4 decode8(const uint32_t* row, int k, const typename Lut<BITS>::T* lut) {
+__device__ __forceinline__ uint4 decode_chunk(const uint4& v, int j, const uint32_t (&t)[4], const uint16_t* lut8) {
   if constexpr (BITS == 4) {
-    const uint32_t w = __ldg(row + (k >> 3));
-    return make_uint4(lut[w & 0xFF], lut[(w >> 8) & 0xFF], lut[(w >> 16) & 0xFF], lut[w >> 24]);
+    const uint32_t w = j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+    return dec4(w, t);
   } else if constexpr (BITS == 2) {
-    const uint32_t w = __ldg(row + (k >> 4)) >> ((k & 15) * 2);
-    const uint2 a = lut[w & 0xFF], b = lut[(w >> 8) & 0xFF];
-    return make_uint4(a.x, a.y, b.x, b.y);
-  } else if constexpr (BITS == 8) {
-    const uint2 w = __ldg(reinterpret_cast<const uint2*>(row + (k >> 2)));
-    return make_uint4(lut[w.x & 0xFF] | (lut[(w.x >> 8) & 0xFF] << 16),
-                      lut[(w.x >> 16) & 0xFF] | (lut[w.x >> 24] << 16),
-                      lut[w.y & 0xFF] | (lut[(w.y >> 8) & 0xFF] << 16),
-                      lut[(w.y >> 16) & 0xFF] | (lut[w.y >> 24] << 16));
+    const uint32_t w = (j < 2) ? v.x : (j < 4 ? v.y : (j < 6 ? v.z : v.w));
+    return dec2((j & 1) ? (w >> 16) : (w & 0xFFFFu), t);
+  } else if constexpr (BITS == 3) {
+    uint32_t x;
+    if (j == 0) x = v.x & 0xFFFFFFu;
+    else if (j == 1) x = ((v.x >> 24) | (v.y << 8)) & 0xFFFFFFu;
+    else if (j == 2) x = ((v.y >> 16) | (v.z << 16)) & 0xFFFFFFu;
+    else x = v.z >> 8;
+    return dec3(x, t);
   } else {
-    const int bit = k * 3, wi = bit >> 5, sh = bit & 31;
-    uint32_t v = __ldg(row + wi) >> sh;
-    if (sh > 8) v |= __ldg(row + wi + 1) << (32 - sh);
-    return make_uint4(lut[v & 63], lut[(v >> 6) & 63], lut[(v >> 12) & 63], lut[(v >> 18) & 63]);
+    return j == 0 ? dec8(v.x, v.y, lut8) : dec8(v.z, v.w, lut8);
   }
 }
 
@@ -92,39 +145,45 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int ch) {
   return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4));
 }
 
-template <int A_BITS, int B_BITS, int BN, int STAGES>
-__global__ void __launch_bounds__(160, 1) gemm_kernel(const __grid_constant__ GemmKParams p) {
+template <int A_BITS, int B_BITS, int BN>
+__global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant__ GemmKParams p) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   constexpr int A_TILE = BM * BK * 2;
   constexpr int B_TILE = BN * BK * 2;
   constexpr int STAGE_BYTES = A_TILE + B_TILE;
-  using LA = typename Lut<A_BITS>::T;
-  using LB = typename Lut<B_BITS>::T;
-  LA* lutA = reinterpret_cast<LA*>(smem + STAGES * STAGE_BYTES);
-  LB* lutB = reinterpret_cast<LB*>(smem + STAGES * STAGE_BYTES + 2048);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + 4096);
-  uint64_t* empty = full + STAGES;
-  uint64_t* accf = empty + STAGES;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  constexpr int QA = Fmt<A_BITS>::QP, QB = Fmt<B_BITS>::QP;
+  constexpr int ITEMS_A = BM * QA, ITEMS = BM * QA + BN * QB;
+  constexpr int IPT = (ITEMS + NDEC - 1) / NDEC;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+
+  uint16_t* lut8 = reinterpret_cast<uint16_t*>(smem + OS * STAGE_BYTES);
+  uint64_t* op_full = reinterpret_cast<uint64_t*>(smem + OS * STAGE_BYTES + 512);
+  uint64_t* op_empty = op_full + OS;
+  uint64_t* acc_full = op_empty + OS;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
-  const int64_t m0 = (int64_t)blockIdx.y * BM;
-  const int num_kb = (p.K + BK - 1) / BK;
+  const int nkb = p.nkb;
+  const int64_t my_tiles = (p.tiles > (int64_t)blockIdx.x) ? (p.tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 
-  build_lut<A_BITS>(lutA, p.a_levels, threadIdx.x, blockDim.x);
-  build_lut<B_BITS>(lutB, p.b_levels, threadIdx.x, blockDim.x);
+  if (A_BITS == 8 && p.a_lut8)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = p.a_lut8[i];
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 128);
-      mbar_init(&empty[s], 1);
+    for (int s = 0; s < OS; ++s) {
+      mbar_init(&op_full[s], NDEC);
+      mbar_init(&op_empty[s], 1);
     }
-    mbar_init(accf, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 128);
+    }
     fence_mbar_init();
   }
-  if (warp == 4) {
-    tmem_alloc(tmem_slot, BN);
+  if (warp == MMA_WARP) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -132,112 +191,224 @@ __global__ void __launch_bounds__(160, 1) gemm_kernel(const __grid_constant__ Ge
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp < 4) {
-    // ------------------------------------------------ decode producers
-    const int pt = threadIdx.x;
-    for (int kb = 0; kb < num_kb; ++kb) {
-      const int s = kb % STAGES;
-      const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-      if (kb >= STAGES && !mbar_wait(&empty[s], ph ^ 1u, p.err)) break;
-      unsigned char* At = smem + s * STAGE_BYTES;
-      unsigned char* Bt = At + A_TILE;
-      const int kbase = kb * BK;
-#pragma unroll 4
-      for (int i = 0; i < (BM * 8) / 128; ++i) {
-        const int id = pt + 128 * i, r = id >> 3, ch = id & 7;
-        const int64_t row = m0 + r;
-        const int k = kbase + ch * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row < p.M && k < p.K) v = decode8<A_BITS>(p.a_codes + row * p.a_wpr, k, lutA);
-        *reinterpret_cast<uint4*>(At + sw128_offset(r, ch)) = v;
-      }
-#pragma unroll 4
-      for (int i = 0; i < (BN * 8) / 128; ++i) {
-        const int id = pt + 128 * i, r = id >> 3, ch = id & 7;
-        const int row = n0 + r;
-        const int k = kbase + ch * 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row < p.N && k < p.K) v = decode8<B_BITS>(p.b_codes + (int64_t)row * p.b_wpr, k, lutB);
-        *reinterpret_cast<uint4*>(Bt + sw128_offset(r, ch)) = v;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(&full[s]);
+  if (warp < NDEC / 32) {
+    // ------------------------------------------------ decoders
+    uint32_t ta[4], tb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ta[i] = p.a_tab[i];
+      tb[i] = p.b_tab[i];
     }
-
-    // ------------------------------------------------ epilogue
-    mbar_wait(accf, 0u, p.err);
-    tc_fence_after();
-    const int rl = warp * 32 + lane;
-    const int64_t row = m0 + rl;
-    const float srow = (row < p.M) ? __ldg(p.a_scale + row) * p.out_scale : 0.f;
-#pragma unroll 1
-    for (int cc = 0; cc < BN / 32; ++cc) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
-      tmem_wait_ld();
-      const int nb = n0 + cc * 32;
-      if (row < p.M && nb < p.N) {
-        float* dst = p.y + row * p.N + nb;
-        if (nb + 32 <= p.N) {
+    const int64_t total = my_tiles * nkb;
+    uint4 cur[IPT], nxt[IPT];
+    // rows past M or N only feed outputs the epilogue never stores, so their
+    // loads are skipped and their (arbitrary) decoded values left in place;
+    // K past the end must contribute zero and is cleared on the A side.
+    auto fetch = [&](int64_t m0, int n0, int kb, uint4 (&dst)[IPT]) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 rr = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + q);
-            float4 o;
-            o.x = __uint_as_float(v[4 * q + 0]) * srow * rr.x;
-            o.y = __uint_as_float(v[4 * q + 1]) * srow * rr.y;
-            o.z = __uint_as_float(v[4 * q + 2]) * srow * rr.z;
-            o.w = __uint_as_float(v[4 * q + 3]) * srow * rr.w;
-            reinterpret_cast<float4*>(dst)[q] = o;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (nb + i < p.N) dst[i] = __uint_as_float(v[i]) * srow * __ldg(p.b_scale + nb + i);
+      for (int it = 0; it < IPT; ++it) {
+        const int id = threadIdx.x + NDEC * it;
+        dst[it] = make_uint4(0u, 0u, 0u, 0u);
+        if (id < ITEMS_A) {
+          const int64_t row = m0 + id / QA;
+          if (row < p.M) dst[it] = load_part<A_BITS>(p.a_codes + row * p.a_wpr, kb, id % QA, p.K);
+        } else if (id < ITEMS) {
+          const int row = n0 + (id - ITEMS_A) / QB;
+          if (row < p.N) dst[it] = load_part<B_BITS>(p.b_codes + (int64_t)row * p.b_wpr, kb, (id - ITEMS_A) % QB, p.K);
         }
       }
+    };
+    auto tile_origin = [&](int64_t tile_i, int64_t& m0, int& n0) {
+      const int64_t tt = blockIdx.x + tile_i * gridDim.x;
+      m0 = (tt / p.n_tiles) * BM;
+      n0 = (int)(tt % p.n_tiles) * BN;
+    };
+    int64_t m0 = 0, m0n = 0;
+    int n0 = 0, n0n = 0;
+    int64_t tile_i = 0;
+    int kb = 0;
+    if (total > 0) {
+      tile_origin(0, m0, n0);
+      fetch(m0, n0, 0, cur);
     }
-  } else if (warp == 4) {
+    for (int64_t g = 0; g < total; ++g) {
+      // position of the next K block (no divisions on the per-block path)
+      int kbn = kb + 1;
+      int64_t tile_n = tile_i;
+      m0n = m0;
+      n0n = n0;
+      if (kbn == nkb) {
+        kbn = 0;
+        ++tile_n;
+        if (g + 1 < total) tile_origin(tile_n, m0n, n0n);
+      }
+      if (g + 1 < total) fetch(m0n, n0n, kbn, nxt);
+      const int s = (int)(g & (OS - 1));
+      const uint32_t n = (uint32_t)(g / OS);
+      if (n > 0 && !mbar_wait(&op_empty[s], (n - 1) & 1u, p.err)) break;
+      unsigned char* At = smem + s * STAGE_BYTES;
+      unsigned char* Bt = At + A_TILE;
+      const bool kfull = (kb + 1) * BK <= p.K;
+#pragma unroll
+      for (int it = 0; it < IPT; ++it) {
+        const int id = threadIdx.x + NDEC * it;
+        if (id < ITEMS_A) {
+          const int r = id / QA, q = id % QA;
+#pragma unroll
+          for (int j = 0; j < Fmt<A_BITS>::CPP; ++j) {
+            uint4 o = decode_chunk<A_BITS>(cur[it], j, ta, lut8);
+            if (!kfull && kb * BK + (q * Fmt<A_BITS>::CPP + j) * 8 >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(At + sw128_offset(r, q * Fmt<A_BITS>::CPP + j)) = o;
+          }
+        } else if (id < ITEMS) {
+          const int r = (id - ITEMS_A) / QB, q = (id - ITEMS_A) % QB;
+#pragma unroll
+          for (int j = 0; j < Fmt<B_BITS>::CPP; ++j)
+            *reinterpret_cast<uint4*>(Bt + sw128_offset(r, q * Fmt<B_BITS>::CPP + j)) =
+                decode_chunk<B_BITS>(cur[it], j, tb, lut8);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&op_full[s]);
+#pragma unroll
+      for (int it = 0; it < IPT; ++it) cur[it] = nxt[it];
+      kb = kbn;
+      tile_i = tile_n;
+      m0 = m0n;
+      n0 = n0n;
+    }
+  } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;
+    for (int64_t i = 0; i < my_tiles; ++i) {
+      const int a = (int)(i & 1);
+      const uint32_t u = (uint32_t)(i >> 1);
+      if (!mbar_wait(&acc_full[a], u & 1u, p.err)) break;
+      tc_fence_after();
+      const int64_t tt = blockIdx.x + i * gridDim.x;
+      const int64_t row = (tt / p.n_tiles) * BM + q * 32 + lane;
+      const int n0 = (int)(tt % p.n_tiles) * BN;
+      const float srow = (row < p.M) ? __ldg(p.a_scale + row) * p.out_scale : 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN + cc * 32), v);
+        tmem_wait_ld();
+        const int nb = n0 + cc * 32;
+        if (row < p.M && nb < p.N) {
+          float* dst = p.y + row * p.N + nb;
+          if (nb + 32 <= p.N) {
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 rr = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + k4);
+              float4 o;
+              o.x = __uint_as_float(v[4 * k4 + 0]) * srow * rr.x;
+              o.y = __uint_as_float(v[4 * k4 + 1]) * srow * rr.y;
+              o.z = __uint_as_float(v[4 * k4 + 2]) * srow * rr.z;
+              o.w = __uint_as_float(v[4 * k4 + 3]) * srow * rr.w;
+              reinterpret_cast<float4*>(dst)[k4] = o;
+            }
+          } else {
+#pragma unroll
+            for (int k1 = 0; k1 < 32; ++k1)
+              if (nb + k1 < p.N) dst[k1] = __uint_as_float(v[k1]) * srow * __ldg(p.b_scale + nb + k1);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[a]);
+    }
+  } else if (warp == MMA_WARP) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_f16_f32(BM, BN);
-      const uint32_t tiles = smem_u32(smem);
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
-        if (!mbar_wait(&full[s], ph, p.err)) break;
+      const uint32_t tiles_base = smem_u32(smem);
+      int64_t g = 0;
+      bool ok = true;
+      for (int64_t i = 0; i < my_tiles && ok; ++i) {
+        const int a = (int)(i & 1);
+        const uint32_t u = (uint32_t)(i >> 1);
+        if (u > 0 && !mbar_wait(&acc_empty[a], (u - 1) & 1u, p.err)) break;
         tc_fence_after();
-        const uint32_t a_addr = tiles + s * STAGE_BYTES, b_addr = a_addr + A_TILE;
+        const uint32_t d_tmem = tmem + (uint32_t)(a * BN);
+        for (int kb = 0; kb < nkb; ++kb, ++g) {
+          const int s = (int)(g % OS);
+          const uint32_t n = (uint32_t)(g / OS);
+          if (!mbar_wait(&op_full[s], n & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = tiles_base + s * STAGE_BYTES, b_addr = a_addr + A_TILE;
 #pragma unroll
-        for (int kk = 0; kk < BK / UMMA_K; ++kk)
-          tc_mma_f16_ss(tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
-                        (kb > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&empty[s]);
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            tc_mma_f16_ss(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
+                          (kb > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(&op_empty[s]);
+        }
+        tc_commit(&acc_full[a]);
       }
-      tc_commit(accf);
     }
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// register tables for the prmt decoders
+void make_tables(int bits, const uint16_t* lv, uint32_t* t) {
+  auto pack = [](const uint8_t* b) {
+    return (uint32_t)b[0] | ((uint32_t)b[1] << 8) | ((uint32_t)b[2] << 16) | ((uint32_t)b[3] << 24);
+  };
+  uint8_t lo[8] = {0}, hi[8] = {0};
+  t[0] = t[1] = t[2] = t[3] = 0;
+  if (bits == 4) {
+    for (int m = 0; m < 8; ++m) {  // positive magnitudes, ascending
+      lo[m] = (uint8_t)(lv[8 + m] & 0xFF);
+      hi[m] = (uint8_t)(lv[8 + m] >> 8);
+    }
+  } else if (bits == 3 || bits == 2) {
+    for (int c = 0; c < (1 << bits); ++c) {
+      lo[c] = (uint8_t)(lv[c] & 0xFF);
+      hi[c] = (uint8_t)(lv[c] >> 8);
+    }
+  } else {
+    return;
+  }
+  if (bits == 2) {
+    t[0] = pack(lo);
+    t[1] = pack(hi);
+  } else {
+    t[0] = pack(lo);
+    t[1] = pack(lo + 4);
+    t[2] = pack(hi);
+    t[3] = pack(hi + 4);
   }
 }
 
 template <int A_BITS, int B_BITS, int BN>
-oq_status launch(const GemmKParams& kp, void* stream) {
-  constexpr int STAGES = (BN == 256) ? 4 : 6;
-  auto kern = gemm_kernel<A_BITS, B_BITS, BN, STAGES>;
-  const size_t smem = 1024 + (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 4096 + 8 * (2 * STAGES + 1) + 16;
+oq_status launch(const GemmKParams& kp_in, void* stream) {
+  GemmKParams kp = kp_in;
+  auto kern = gemm_kernel<A_BITS, B_BITS, BN>;
+  const size_t smem = 1024 + (size_t)OS * (BM * BK * 2 + BN * BK * 2) + 512 + 8 * (2 * OS + 4) + 16;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
     set_error(std::string("cudaFuncSetAttribute(gemm): ") + cudaGetErrorString(e));
     return OQ_ERR_CUDA;
   }
-  const dim3 grid((unsigned)((kp.N + BN - 1) / BN), (unsigned)((kp.M + BM - 1) / BM));
-  kern<<<grid, 160, smem, static_cast<cudaStream_t>(stream)>>>(kp);
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  kp.n_tiles = (kp.N + BN - 1) / BN;
+  kp.nkb = (kp.K + BK - 1) / BK;
+  kp.tiles = ((kp.M + BM - 1) / BM) * (int64_t)kp.n_tiles;
+  const int grid = (int)std::min<int64_t>(kp.tiles, sms);
+  kern<<<grid, NTHREADS, smem, static_cast<cudaStream_t>(stream)>>>(kp);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("gemm launch: ") + cudaGetErrorString(e));
@@ -272,8 +443,6 @@ oq_status gemm_launch(const GemmArgs& g, void* stream) {
   kp.b_codes = g.b_codes;
   kp.a_scale = g.a_scale;
   kp.b_scale = g.b_scale;
-  kp.a_levels = g.a_levels;
-  kp.b_levels = g.b_levels;
   kp.out_scale = g.out_scale;
   kp.y = g.y;
   kp.M = g.M;
@@ -281,8 +450,10 @@ oq_status gemm_launch(const GemmArgs& g, void* stream) {
   kp.K = g.K;
   kp.a_wpr = g.K * g.a_bits / 32;
   kp.b_wpr = g.K * g.b_bits / 32;
+  make_tables(g.a_bits, g.a_levels_host, kp.a_tab);
+  make_tables(g.b_bits, g.b_levels_host, kp.b_tab);
+  kp.a_lut8 = g.a_levels;
   kp.err = g.err;
-  if (g.M > (int64_t)65535 * BM) return OQ_ERR_UNSUPPORTED;
   switch (g.a_bits) {
     case 2: return launch_b<2>(kp, g.b_bits, stream);
     case 3: return launch_b<3>(kp, g.b_bits, stream);

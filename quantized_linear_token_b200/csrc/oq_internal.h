@@ -24,6 +24,7 @@ struct oq_layer {
   uint32_t* d_signmask;               // sign bits in kernel order, or null
   uint16_t* d_levels_a;               // fp16 bits of a_scale * activation levels
   uint16_t* d_levels_w;               // fp16 bits of w_scale * weight levels
+  uint16_t lv_a[256], lv_w[256];      // host copies of the two level tables
   int* d_error;                       // device error word
   float thr_a[128];                   // sqrt(h) * positive thresholds, +inf padded
   float thr_w[128];
@@ -66,8 +67,10 @@ struct GemmArgs {
   const uint32_t* b_codes;   // [N, K*b_bits/32]
   const float* a_scale;      // [M] per-row magnitude s
   const float* b_scale;      // [N] per-row magnitude r
-  const uint16_t* a_levels;  // fp16 bits, 2^a_bits
-  const uint16_t* b_levels;  // fp16 bits, 2^b_bits
+  const uint16_t* a_levels;       // device fp16 bits, 2^a_bits (8-bit table)
+  const uint16_t* b_levels;       // device fp16 bits, 2^b_bits
+  const uint16_t* a_levels_host;  // host copies (register decode tables)
+  const uint16_t* b_levels_host;
   float out_scale;           // 1 / (alpha_a alpha_w)
   float* y;                  // [M, N] fp32
   int64_t M;
