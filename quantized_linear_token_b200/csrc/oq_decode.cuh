@@ -1,0 +1,108 @@
+// Code decoding shared by the codebook-contraction kernels: loading the packed
+// codes of one K block of a row and expanding 8 codes into 8 fp16 values (one
+// 16-byte chunk of a 128B-swizzled K-major operand tile) with byte-permute
+// lookups into codebook tables held in registers.
+#pragma once
+
+#include <cstdint>
+
+namespace oq {
+
+constexpr int DEC_BK = 64;   // K elements per operand block (128 bytes of fp16)
+
+// per bit width: 16-byte code parts per row per K block and 8-code chunks per part
+template <int BITS> struct Fmt;
+template <> struct Fmt<2> { static constexpr int QP = 1, CPP = 8; };
+template <> struct Fmt<3> { static constexpr int QP = 2, CPP = 4; };
+template <> struct Fmt<4> { static constexpr int QP = 2, CPP = 4; };
+template <> struct Fmt<8> { static constexpr int QP = 4, CPP = 2; };
+
+// the codes of part q of K block kb of a row (zeros past K)
+template <int BITS>
+__device__ __forceinline__ uint4 load_part(const uint32_t* row, int kb, int q, int K) {
+  const int k0 = kb * DEC_BK + q * (DEC_BK / Fmt<BITS>::QP);
+  if (k0 >= K) return make_uint4(0u, 0u, 0u, 0u);
+  if constexpr (BITS == 3) {
+    const uint32_t* p = row + kb * 6 + q * 3;
+    return make_uint4(__ldg(p), __ldg(p + 1), __ldg(p + 2), 0u);
+  } else if constexpr (BITS == 2) {
+    // rows are only 8-byte aligned when K % 64 == 32
+    const uint2* p = reinterpret_cast<const uint2*>(row + kb * 4);
+    const uint2 lo = __ldg(p);
+    const uint2 hi = (k0 + 32 < K) ? __ldg(p + 1) : make_uint2(0u, 0u);
+    return make_uint4(lo.x, lo.y, hi.x, hi.y);
+  } else {
+    return __ldg(reinterpret_cast<const uint4*>(row) + kb * (BITS / 2) + q);
+  }
+}
+
+// ---- 8 codes -> 8 fp16 (one 16-byte chunk of the operand tile)
+__device__ __forceinline__ uint4 dec4(uint32_t w, const uint32_t (&t)[4]) {
+  // symmetric codebook: code c >= 8 -> +P[c-8], c < 8 -> -P[7-c]
+  const uint32_t n = ((~w) & 0x88888888u) >> 3;            // 1 per negative code
+  const uint32_t m = (w & 0x77777777u) ^ (n * 7u);         // magnitude index
+  const uint32_t mh = m >> 16, nh = n >> 16;
+  const uint32_t lo_a = __byte_perm(t[0], t[1], m), hi_a = __byte_perm(t[2], t[3], m) | __byte_perm(0x8000u, 0u, n);
+  const uint32_t lo_b = __byte_perm(t[0], t[1], mh), hi_b = __byte_perm(t[2], t[3], mh) | __byte_perm(0x8000u, 0u, nh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+__device__ __forceinline__ uint4 dec2(uint32_t x, const uint32_t (&t)[4]) {
+  // 2-bit fields -> one selector nibble per code; 4-entry table in one register
+  uint32_t y = (x | (x << 8)) & 0x00FF00FFu;
+  y = (y | (y << 4)) & 0x0F0F0F0Fu;
+  y = (y | (y << 2)) & 0x33333333u;
+  const uint32_t yh = y >> 16;
+  const uint32_t lo_a = __byte_perm(t[0], t[0], y), hi_a = __byte_perm(t[1], t[1], y);
+  const uint32_t lo_b = __byte_perm(t[0], t[0], yh), hi_b = __byte_perm(t[1], t[1], yh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+__device__ __forceinline__ uint4 dec3(uint32_t x, const uint32_t (&t)[4]) {
+  // 3-bit fields -> one selector nibble per code; 8-entry table in two registers
+  uint32_t y = (x & 0xFFFu) | ((x & 0xFFF000u) << 4);
+  y = (y & 0x003F003Fu) | ((y & 0x0FC00FC0u) << 2);
+  y = (y & 0x07070707u) | ((y & 0x38383838u) << 1);
+  const uint32_t yh = y >> 16;
+  const uint32_t lo_a = __byte_perm(t[0], t[1], y), hi_a = __byte_perm(t[2], t[3], y);
+  const uint32_t lo_b = __byte_perm(t[0], t[1], yh), hi_b = __byte_perm(t[2], t[3], yh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+__device__ __forceinline__ uint4 dec8(uint32_t w0, uint32_t w1, const uint16_t* lut) {
+  auto pr = [&](uint32_t w, int b) {
+    return (uint32_t)lut[(w >> (8 * b)) & 0xFF] | ((uint32_t)lut[(w >> (8 * b + 8)) & 0xFF] << 16);
+  };
+  return make_uint4(pr(w0, 0), pr(w0, 2), pr(w1, 0), pr(w1, 2));
+}
+
+// chunk j of a part -> 8 fp16
+template <int BITS>
+__device__ __forceinline__ uint4 decode_chunk(const uint4& v, int j, const uint32_t (&t)[4], const uint16_t* lut8) {
+  if constexpr (BITS == 4) {
+    const uint32_t w = j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+    return dec4(w, t);
+  } else if constexpr (BITS == 2) {
+    const uint32_t w = (j < 2) ? v.x : (j < 4 ? v.y : (j < 6 ? v.z : v.w));
+    return dec2((j & 1) ? (w >> 16) : (w & 0xFFFFu), t);
+  } else if constexpr (BITS == 3) {
+    uint32_t x;
+    if (j == 0) x = v.x & 0xFFFFFFu;
+    else if (j == 1) x = ((v.x >> 24) | (v.y << 8)) & 0xFFFFFFu;
+    else if (j == 2) x = ((v.y >> 16) | (v.z << 16)) & 0xFFFFFFu;
+    else x = v.z >> 8;
+    return dec3(x, t);
+  } else {
+    return j == 0 ? dec8(v.x, v.y, lut8) : dec8(v.z, v.w, lut8);
+  }
+}
+
+// byte offset of 16-byte chunk `ch` of row `r` in a 128B-swizzled K-major tile
+__device__ __forceinline__ uint32_t sw128_offset(int r, int ch) {
+  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4));
+}
+
+}  // namespace oq

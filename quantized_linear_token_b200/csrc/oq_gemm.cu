@@ -21,6 +21,7 @@
 #include <algorithm>
 #include <cstring>
 
+#include "oq_decode.cuh"
 #include "oq_internal.h"
 #include "oq_ptx.cuh"
 
@@ -49,101 +50,6 @@ struct GemmKParams {
   const uint16_t* a_lut8;
   int* err;
 };
-
-// per bit width: 16-byte code parts per row per K block and 8-code chunks per part
-template <int BITS> struct Fmt;
-template <> struct Fmt<2> { static constexpr int QP = 1, CPP = 8; };
-template <> struct Fmt<3> { static constexpr int QP = 2, CPP = 4; };
-template <> struct Fmt<4> { static constexpr int QP = 2, CPP = 4; };
-template <> struct Fmt<8> { static constexpr int QP = 4, CPP = 2; };
-
-// the codes of part q of K block kb of a row (zeros past K)
-template <int BITS>
-__device__ __forceinline__ uint4 load_part(const uint32_t* row, int kb, int q, int K) {
-  const int k0 = kb * BK + q * (BK / Fmt<BITS>::QP);
-  if (k0 >= K) return make_uint4(0u, 0u, 0u, 0u);
-  if constexpr (BITS == 3) {
-    const uint32_t* p = row + kb * 6 + q * 3;
-    return make_uint4(__ldg(p), __ldg(p + 1), __ldg(p + 2), 0u);
-  } else if constexpr (BITS == 2) {
-    // rows are only 8-byte aligned when K % 64 == 32
-    const uint2* p = reinterpret_cast<const uint2*>(row + kb * 4);
-    const uint2 lo = __ldg(p);
-    const uint2 hi = (k0 + 32 < K) ? __ldg(p + 1) : make_uint2(0u, 0u);
-    return make_uint4(lo.x, lo.y, hi.x, hi.y);
-  } else {
-    return __ldg(reinterpret_cast<const uint4*>(row) + kb * (BITS / 2) + q);
-  }
-}
-
-// ---- 8 codes -> 8 fp16 (one 16-byte chunk of the operand tile)
-__device__ __forceinline__ uint4 dec4(uint32_t w, const uint32_t (&t)[4]) {
-  // symmetric codebook: code c >= 8 -> +P[c-8], c < 8 -> -P[7-c]
-  const uint32_t n = ((~w) & 0x88888888u) >> 3;            // 1 per negative code
-  const uint32_t m = (w & 0x77777777u) ^ (n * 7u);         // magnitude index
-  const uint32_t mh = m >> 16, nh = n >> 16;
-  const uint32_t lo_a = __byte_perm(t[0], t[1], m), hi_a = __byte_perm(t[2], t[3], m) | __byte_perm(0x8000u, 0u, n);
-  const uint32_t lo_b = __byte_perm(t[0], t[1], mh), hi_b = __byte_perm(t[2], t[3], mh) | __byte_perm(0x8000u, 0u, nh);
-  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
-                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
-}
-
-__device__ __forceinline__ uint4 dec2(uint32_t x, const uint32_t (&t)[4]) {
-  // 2-bit fields -> one selector nibble per code; 4-entry table in one register
-  uint32_t y = (x | (x << 8)) & 0x00FF00FFu;
-  y = (y | (y << 4)) & 0x0F0F0F0Fu;
-  y = (y | (y << 2)) & 0x33333333u;
-  const uint32_t yh = y >> 16;
-  const uint32_t lo_a = __byte_perm(t[0], t[0], y), hi_a = __byte_perm(t[1], t[1], y);
-  const uint32_t lo_b = __byte_perm(t[0], t[0], yh), hi_b = __byte_perm(t[1], t[1], yh);
-  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
-                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
-}
-
-__device__ __forceinline__ uint4 dec3(uint32_t x, const uint32_t (&t)[4]) {
-  // 3-bit fields -> one selector nibble per code; 8-entry table in two registers
-  uint32_t y = (x & 0xFFFu) | ((x & 0xFFF000u) << 4);
-  y = (y & 0x003F003Fu) | ((y & 0x0FC00FC0u) << 2);
-  y = (y & 0x07070707u) | ((y & 0x38383838u) << 1);
-  const uint32_t yh = y >> 16;
-  const uint32_t lo_a = __byte_perm(t[0], t[1], y), hi_a = __byte_perm(t[2], t[3], y);
-  const uint32_t lo_b = __byte_perm(t[0], t[1], yh), hi_b = __byte_perm(t[2], t[3], yh);
-  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
-                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
-}
-
-__device__ __forceinline__ uint4 dec8(uint32_t w0, uint32_t w1, const uint16_t* lut) {
-  auto pr = [&](uint32_t w, int b) {
-    return (uint32_t)lut[(w >> (8 * b)) & 0xFF] | ((uint32_t)lut[(w >> (8 * b + 8)) & 0xFF] << 16);
-  };
-  return make_uint4(pr(w0, 0), pr(w0, 2), pr(w1, 0), pr(w1, 2));
-}
-
-// chunk j of a part -> 8 fp16
-template <int BITS>
-__device__ __forceinline__ uint4 decode_chunk(const uint4& v, int j, const uint32_t (&t)[4], const uint16_t* lut8) {
-  if constexpr (BITS == 4) {
-    const uint32_t w = j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
-    return dec4(w, t);
-  } else if constexpr (BITS == 2) {
-    const uint32_t w = (j < 2) ? v.x : (j < 4 ? v.y : (j < 6 ? v.z : v.w));
-    return dec2((j & 1) ? (w >> 16) : (w & 0xFFFFu), t);
-  } else if constexpr (BITS == 3) {
-    uint32_t x;
-    if (j == 0) x = v.x & 0xFFFFFFu;
-    else if (j == 1) x = ((v.x >> 24) | (v.y << 8)) & 0xFFFFFFu;
-    else if (j == 2) x = ((v.y >> 16) | (v.z << 16)) & 0xFFFFFFu;
-    else x = v.z >> 8;
-    return dec3(x, t);
-  } else {
-    return j == 0 ? dec8(v.x, v.y, lut8) : dec8(v.z, v.w, lut8);
-  }
-}
-
-// byte offset of 16-byte chunk `ch` of row `r` in a 128B-swizzled K-major tile
-__device__ __forceinline__ uint32_t sw128_offset(int r, int ch) {
-  return (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((ch ^ (r & 7)) << 4));
-}
 
 template <int A_BITS, int B_BITS, int BN>
 __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant__ GemmKParams p) {
@@ -360,37 +266,6 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
   }
 }
 
-// register tables for the prmt decoders
-void make_tables(int bits, const uint16_t* lv, uint32_t* t) {
-  auto pack = [](const uint8_t* b) {
-    return (uint32_t)b[0] | ((uint32_t)b[1] << 8) | ((uint32_t)b[2] << 16) | ((uint32_t)b[3] << 24);
-  };
-  uint8_t lo[8] = {0}, hi[8] = {0};
-  t[0] = t[1] = t[2] = t[3] = 0;
-  if (bits == 4) {
-    for (int m = 0; m < 8; ++m) {  // positive magnitudes, ascending
-      lo[m] = (uint8_t)(lv[8 + m] & 0xFF);
-      hi[m] = (uint8_t)(lv[8 + m] >> 8);
-    }
-  } else if (bits == 3 || bits == 2) {
-    for (int c = 0; c < (1 << bits); ++c) {
-      lo[c] = (uint8_t)(lv[c] & 0xFF);
-      hi[c] = (uint8_t)(lv[c] >> 8);
-    }
-  } else {
-    return;
-  }
-  if (bits == 2) {
-    t[0] = pack(lo);
-    t[1] = pack(hi);
-  } else {
-    t[0] = pack(lo);
-    t[1] = pack(lo + 4);
-    t[2] = pack(hi);
-    t[3] = pack(hi + 4);
-  }
-}
-
 template <int A_BITS, int B_BITS, int BN>
 oq_status launch(const GemmKParams& kp_in, void* stream) {
   GemmKParams kp = kp_in;
@@ -435,8 +310,44 @@ oq_status launch_b(const GemmKParams& kp, int b_bits, void* stream) {
 
 }  // namespace
 
+// register tables for the prmt decoders
+void make_decode_tables(int bits, const uint16_t* lv, uint32_t* t) {
+  auto pack = [](const uint8_t* b) {
+    return (uint32_t)b[0] | ((uint32_t)b[1] << 8) | ((uint32_t)b[2] << 16) | ((uint32_t)b[3] << 24);
+  };
+  uint8_t lo[8] = {0}, hi[8] = {0};
+  t[0] = t[1] = t[2] = t[3] = 0;
+  if (bits == 4) {
+    for (int m = 0; m < 8; ++m) {  // positive magnitudes, ascending
+      lo[m] = (uint8_t)(lv[8 + m] & 0xFF);
+      hi[m] = (uint8_t)(lv[8 + m] >> 8);
+    }
+  } else if (bits == 3 || bits == 2) {
+    for (int c = 0; c < (1 << bits); ++c) {
+      lo[c] = (uint8_t)(lv[c] & 0xFF);
+      hi[c] = (uint8_t)(lv[c] >> 8);
+    }
+  } else {
+    return;
+  }
+  if (bits == 2) {
+    t[0] = pack(lo);
+    t[1] = pack(hi);
+  } else {
+    t[0] = pack(lo);
+    t[1] = pack(lo + 4);
+    t[2] = pack(hi);
+    t[3] = pack(hi + 4);
+  }
+}
+
 oq_status gemm_launch(const GemmArgs& g, void* stream) {
   if (g.M == 0) return OQ_OK;
+  // CTA-pair tiles (256 x 256) whenever the output width allows them
+  if (g.N % 256 == 0) {
+    const oq_status st = gemm_pair_launch(g, stream);
+    if (st != OQ_ERR_UNSUPPORTED) return st;
+  }
   GemmKParams kp;
   std::memset(&kp, 0, sizeof(kp));
   kp.a_codes = g.a_codes;
@@ -450,8 +361,8 @@ oq_status gemm_launch(const GemmArgs& g, void* stream) {
   kp.K = g.K;
   kp.a_wpr = g.K * g.a_bits / 32;
   kp.b_wpr = g.K * g.b_bits / 32;
-  make_tables(g.a_bits, g.a_levels_host, kp.a_tab);
-  make_tables(g.b_bits, g.b_levels_host, kp.b_tab);
+  make_decode_tables(g.a_bits, g.a_levels_host, kp.a_tab);
+  make_decode_tables(g.b_bits, g.b_levels_host, kp.b_tab);
   kp.a_lut8 = g.a_levels;
   kp.err = g.err;
   switch (g.a_bits) {

@@ -1,0 +1,413 @@
+// Codebook contraction on CTA pairs (tcgen05 cta_group::2), the main path for
+// d_out % 256 == 0:
+//   y[m, n] = a_scale[m] b_scale[n] out_scale sum_k LA[A[m, k]] LB[B[n, k]]
+// (gecl notes Method 2 and Takeaway 3: a native non-uniform low-bit GEMM in
+// the shared rotated basis).
+//
+// A cluster of two CTAs computes a 256 x 256 tile of y.  Each CTA decodes 128
+// rows of activation codes and 128 rows of weight codes per K block of 64
+// into fp16 operand tiles (128B-swizzled, K-major) in its own shared memory;
+// one thread of the even CTA issues the paired MMA (M = 256, N = 256, K = 16),
+// which reads A rows and B rows from both CTAs and leaves each CTA's 128 output
+// rows in its own tensor memory.  Compared with one-SM 128 x 256 tiles this
+// halves the weight decode per SM, and each SM still holds two accumulators,
+// so the epilogue of one tile overlaps the next tile's main loop.
+//
+// Warps: 0-15 decode (codes prefetched two K blocks ahead into registers),
+// 16-19 epilogue, 20 allocates tensor memory and (even CTA) issues the MMAs
+// (odd CTA: forwards the decoders' arrivals to the even CTA).
+// Synchronisation: decoders of both CTAs arrive (one thread per warp, release
+// at cluster scope) on the even CTA's `full` barrier; the MMA completion is
+// multicast by tcgen05.commit to both CTAs' `empty` / `acc_full` barriers;
+// epilogue warps of both CTAs arrive on the even CTA's `acc_empty`.  Every
+// wait is bounded (oq_ptx.cuh).
+#include <algorithm>
+#include <cstring>
+
+#include "oq_decode.cuh"
+#include "oq_internal.h"
+#include "oq_ptx.cuh"
+
+namespace oq {
+namespace {
+
+constexpr int RM = 128;            // activation rows per CTA (pair M = 256)
+constexpr int PN = 256;            // output columns per pair tile
+constexpr int RN = 128;            // weight rows per CTA
+constexpr int BK = DEC_BK, UMMA_K = 16;
+constexpr int NDEC = 512;          // decoder threads (warps 0-15)
+constexpr int EPI_WARP0 = 16;      // epilogue warps 16-19 (TMEM lane quarters 0-3)
+constexpr int MMA_WARP = 20;
+constexpr int NTHREADS = 21 * 32;
+constexpr int OS = 6;              // operand stages
+constexpr int A_TILE = RM * BK * 2;
+constexpr int B_TILE = RN * BK * 2;
+constexpr int STAGE_BYTES = A_TILE + B_TILE;
+constexpr uint32_t TMEM_COLS = 2 * PN;
+constexpr uint32_t FULL_LOCAL = NDEC / 32;           // one arrival per decoder warp
+constexpr uint32_t ACC_EMPTY_COUNT = 2 * 4;           // one per epilogue warp, both CTAs
+
+struct PairParams {
+  const uint32_t* a_codes;
+  const uint32_t* b_codes;
+  const float* a_scale;
+  const float* b_scale;
+  float out_scale;
+  float* y;
+  int64_t M;
+  int N, K, a_wpr, b_wpr;
+  int n_tiles, nkb;
+  int64_t tiles;
+  uint32_t a_tab[4], b_tab[4];
+  const uint16_t* a_lut8;
+  int* err;
+};
+
+template <int A_BITS, int B_BITS>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ PairParams p) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  constexpr int QA = Fmt<A_BITS>::QP, QB = Fmt<B_BITS>::QP;
+  constexpr int ITEMS_A = RM * QA, ITEMS = RM * QA + RN * QB;
+  constexpr int IPT = (ITEMS + NDEC - 1) / NDEC;
+
+  uint16_t* lut8 = reinterpret_cast<uint16_t*>(smem + OS * STAGE_BYTES);
+  uint64_t* op_full = reinterpret_cast<uint64_t*>(smem + OS * STAGE_BYTES + 512);
+  uint64_t* op_empty = op_full + OS;
+  uint64_t* acc_full = op_empty + OS;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nkb = p.nkb;
+  const int64_t my_tiles = (p.tiles > pair) ? (p.tiles - 1 - pair) / npairs + 1 : 0;
+
+  if (A_BITS == 8 && p.a_lut8)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = p.a_lut8[i];
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < OS; ++s) {
+      // the even CTA also counts the odd CTA's forwarded arrival
+      mbar_init(&op_full[s], rank == 0 ? FULL_LOCAL + 1 : FULL_LOCAL);
+      mbar_init(&op_empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], ACC_EMPTY_COUNT);
+    }
+    fence_mbar_init();
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers of both CTAs initialised before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (warp < NDEC / 32) {
+    // ------------------------------------------------ decoders
+    uint32_t ta[4], tb[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ta[i] = p.a_tab[i];
+      tb[i] = p.b_tab[i];
+    }
+    // fixed per-thread items: operand row r, 16-byte code part q; the row's
+    // byte offset inside a stage and its swizzle pattern do not change
+    uint32_t row_off[IPT], xs[IPT];
+    int item_r[IPT], item_q[IPT];
+#pragma unroll
+    for (int it = 0; it < IPT; ++it) {
+      const int id = threadIdx.x + NDEC * it;
+      const bool is_a = id < ITEMS_A;
+      const int r = is_a ? id / QA : (id - ITEMS_A) / QB;
+      item_r[it] = r;
+      item_q[it] = is_a ? id % QA : (id - ITEMS_A) % QB;
+      row_off[it] = (is_a ? 0u : (uint32_t)A_TILE) + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+      xs[it] = (uint32_t)(r & 7) << 4;
+    }
+    // code-row pointers of the tile the fetch cursor is in (null: the row is
+    // outside the matrix; its decoded values only reach discarded outputs)
+    const uint32_t* frow[IPT];
+    auto origin = [&](int64_t tile_i) {
+      const int64_t tt = pair + tile_i * npairs;
+      const int64_t m0 = (tt / p.n_tiles) * (2 * RM) + rank * RM;
+      const int n0 = (int)(tt % p.n_tiles) * PN + (int)rank * RN;
+#pragma unroll
+      for (int it = 0; it < IPT; ++it) {
+        const int id = threadIdx.x + NDEC * it;
+        frow[it] = nullptr;
+        if (id < ITEMS_A) {
+          const int64_t row = m0 + item_r[it];
+          if (row < p.M) frow[it] = p.a_codes + row * p.a_wpr;
+        } else if (id < ITEMS) {
+          const int row = n0 + item_r[it];
+          if (row < p.N) frow[it] = p.b_codes + (int64_t)row * p.b_wpr;
+        }
+      }
+    };
+    auto fetch = [&](int kb, uint4 (&dst)[IPT]) {
+#pragma unroll
+      for (int it = 0; it < IPT; ++it) {
+        const int id = threadIdx.x + NDEC * it;
+        dst[it] = make_uint4(0u, 0u, 0u, 0u);
+        if (frow[it] != nullptr) {
+          if (id < ITEMS_A) dst[it] = load_part<A_BITS>(frow[it], kb, item_q[it], p.K);
+          else dst[it] = load_part<B_BITS>(frow[it], kb, item_q[it], p.K);
+        }
+      }
+    };
+    // decode one K block into stage `st`; `tail`: the block runs past K and
+    // the A chunks beyond it must be zero
+    auto decode = [&](const uint4 (&cur)[IPT], int st, bool tail, int kb) {
+      const uint32_t st_base = smem_base + (uint32_t)(st * STAGE_BYTES);
+#pragma unroll
+      for (int it = 0; it < IPT; ++it) {
+        const int id = threadIdx.x + NDEC * it;
+        const uint32_t rb = st_base + row_off[it];
+        if (id < ITEMS_A) {
+#pragma unroll
+          for (int j = 0; j < Fmt<A_BITS>::CPP; ++j) {
+            const int cj = item_q[it] * Fmt<A_BITS>::CPP + j;
+            uint4 o = decode_chunk<A_BITS>(cur[it], j, ta, lut8);
+            if (tail && kb * BK + cj * 8 >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
+            st_shared_v4(rb | (((uint32_t)cj << 4) ^ xs[it]), o);
+          }
+        } else if (id < ITEMS) {
+#pragma unroll
+          for (int j = 0; j < Fmt<B_BITS>::CPP; ++j) {
+            const int cj = item_q[it] * Fmt<B_BITS>::CPP + j;
+            st_shared_v4(rb | (((uint32_t)cj << 4) ^ xs[it]), decode_chunk<B_BITS>(cur[it], j, tb, lut8));
+          }
+        }
+      }
+    };
+    const int64_t total = my_tiles * nkb;
+    // the fetch cursor runs two K blocks ahead of the decode cursor; the three
+    // register buffers rotate by unrolling (no copies of registers whose loads
+    // are still in flight)
+    int64_t f_tile = 0;
+    int f_kb = 0;
+    origin(0);
+    auto advance = [&]() {
+      if (++f_kb == nkb) {
+        f_kb = 0;
+        ++f_tile;
+        origin(f_tile);
+      }
+    };
+    uint4 c0[IPT], c1[IPT], c2[IPT];
+    if (total > 0) {
+      fetch(f_kb, c0);
+      advance();
+    }
+    if (total > 1) {
+      fetch(f_kb, c1);
+      advance();
+    }
+    int s = 0, d_kb = 0;
+    uint32_t n = 0;
+    int64_t g = 0;
+    auto step = [&](const uint4 (&cur)[IPT], uint4 (&fut)[IPT]) -> bool {
+      if (g + 2 < total) {
+        fetch(f_kb, fut);
+        advance();
+      }
+      if (n > 0 && !mbar_wait(&op_empty[s], (n - 1) & 1u, p.err)) return false;
+      if ((d_kb + 1) * BK > p.K) decode(cur, s, true, d_kb);
+      else decode(cur, s, false, d_kb);
+      // this warp's tiles -> visible to the async proxy, then one arrival
+      // per warp on this CTA's `full` barrier (the odd CTA forwards it)
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&op_full[s]);
+      if (++s == OS) {
+        s = 0;
+        ++n;
+      }
+      if (++d_kb == nkb) d_kb = 0;
+      ++g;
+      return true;
+    };
+    while (g < total) {
+      if (!step(c0, c2) || g >= total) break;
+      if (!step(c1, c0) || g >= total) break;
+      if (!step(c2, c1)) break;
+    }
+  } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
+    // ------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    for (int64_t i = 0; i < my_tiles; ++i) {
+      const int a = (int)(i & 1);
+      const uint32_t u = (uint32_t)(i >> 1);
+      if (!mbar_wait(&acc_full[a], u & 1u, p.err)) break;
+      tc_fence_after();
+      const int64_t tt = pair + i * npairs;
+      const int64_t row = (tt / p.n_tiles) * (2 * RM) + rank * RM + q * 32 + lane;
+      const int n0 = (int)(tt % p.n_tiles) * PN;
+      const float srow = (row < p.M) ? __ldg(p.a_scale + row) * p.out_scale : 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < PN / 32; ++cc) {
+        const int nb = n0 + cc * 32;
+        float4 rr[8];
+#pragma unroll
+        for (int k4 = 0; k4 < 8; ++k4) rr[k4] = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + k4);
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * PN + cc * 32), v);
+        tmem_wait_ld();
+        if (row < p.M) {
+          float* dst = p.y + row * p.N + nb;
+#pragma unroll
+          for (int k4 = 0; k4 < 8; ++k4) {
+            float4 o;
+            o.x = __uint_as_float(v[4 * k4 + 0]) * srow * rr[k4].x;
+            o.y = __uint_as_float(v[4 * k4 + 1]) * srow * rr[k4].y;
+            o.z = __uint_as_float(v[4 * k4 + 2]) * srow * rr[k4].z;
+            o.w = __uint_as_float(v[4 * k4 + 3]) * srow * rr[k4].w;
+            reinterpret_cast<float4*>(dst)[k4] = o;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[a]), 0));
+    }
+  } else if (warp == MMA_WARP && rank == 0) {
+    // ------------------------------------------------ paired MMA issuer (even CTA)
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16_f32(2 * RM, PN);
+      int s = 0;
+      uint32_t n = 0;
+      bool ok = true;
+      for (int64_t i = 0; i < my_tiles && ok; ++i) {
+        const int a = (int)(i & 1);
+        const uint32_t u = (uint32_t)(i >> 1);
+        if (u > 0 && !mbar_wait_cluster(&acc_empty[a], (u - 1) & 1u, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(a * PN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait_cluster(&op_full[s], n & 1u, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_base + (uint32_t)(s * STAGE_BYTES), b_addr = a_addr + A_TILE;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            tc_mma_f16_ss_pair(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
+                               (kb > 0 || kk > 0) ? 1u : 0u);
+          tc_commit_pair_mc(&op_empty[s], (uint16_t)0x3);
+          if (++s == OS) {
+            s = 0;
+            ++n;
+          }
+        }
+        tc_commit_pair_mc(&acc_full[a], (uint16_t)0x3);
+      }
+    }
+    __syncwarp();
+  }
+
+  if (warp == MMA_WARP && rank == 1) {
+    // ------------------------------------------------ forwarder (odd CTA)
+    // one cluster-scope release per stage instead of one per decoder warp
+    if (lane == 0) {
+      const int64_t total = my_tiles * nkb;
+      int s = 0;
+      uint32_t n = 0;
+      for (int64_t g = 0; g < total; ++g) {
+        if (!mbar_wait(&op_full[s], n & 1u, p.err)) break;
+        mbar_arrive_cluster(mapa_shared(smem_u32(&op_full[s]), 0));
+        if (++s == OS) {
+          s = 0;
+          ++n;
+        }
+      }
+    }
+    __syncwarp();
+  }
+
+  // neither CTA may leave while its peer can still read its tiles or arrive
+  // on its barriers
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+template <int A_BITS, int B_BITS>
+oq_status launch_pair(const PairParams& kp_in, void* stream) {
+  PairParams kp = kp_in;
+  auto kern = gemm_pair_kernel<A_BITS, B_BITS>;
+  const size_t smem = 1024 + (size_t)OS * STAGE_BYTES + 512 + 8 * (2 * OS + 4) + 16;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) {
+    set_error(std::string("cudaFuncSetAttribute(gemm pair): ") + cudaGetErrorString(e));
+    return OQ_ERR_CUDA;
+  }
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  kp.n_tiles = kp.N / PN;
+  kp.nkb = (kp.K + BK - 1) / BK;
+  kp.tiles = ((kp.M + 2 * RM - 1) / (2 * RM)) * (int64_t)kp.n_tiles;
+  const int64_t grid = std::min<int64_t>(2 * kp.tiles, (int64_t)(sms & ~1));
+  kern<<<(unsigned)grid, NTHREADS, smem, static_cast<cudaStream_t>(stream)>>>(kp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error(std::string("gemm pair launch: ") + cudaGetErrorString(e));
+    return OQ_ERR_CUDA;
+  }
+  return OQ_OK;
+}
+
+template <int A_BITS>
+oq_status launch_pair_b(const PairParams& kp, int b_bits, void* stream) {
+  switch (b_bits) {
+    case 2: return launch_pair<A_BITS, 2>(kp, stream);
+    case 3: return launch_pair<A_BITS, 3>(kp, stream);
+    case 4: return launch_pair<A_BITS, 4>(kp, stream);
+    default: return OQ_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace
+
+oq_status gemm_pair_launch(const GemmArgs& g, void* stream) {
+  if (g.M == 0) return OQ_OK;
+  if (g.N % PN != 0) return OQ_ERR_UNSUPPORTED;
+  PairParams kp;
+  std::memset(&kp, 0, sizeof(kp));
+  kp.a_codes = g.a_codes;
+  kp.b_codes = g.b_codes;
+  kp.a_scale = g.a_scale;
+  kp.b_scale = g.b_scale;
+  kp.out_scale = g.out_scale;
+  kp.y = g.y;
+  kp.M = g.M;
+  kp.N = g.N;
+  kp.K = g.K;
+  kp.a_wpr = g.K * g.a_bits / 32;
+  kp.b_wpr = g.K * g.b_bits / 32;
+  make_decode_tables(g.a_bits, g.a_levels_host, kp.a_tab);
+  make_decode_tables(g.b_bits, g.b_levels_host, kp.b_tab);
+  kp.a_lut8 = g.a_levels;
+  kp.err = g.err;
+  switch (g.a_bits) {
+    case 2: return launch_pair_b<2>(kp, g.b_bits, stream);
+    case 3: return launch_pair_b<3>(kp, g.b_bits, stream);
+    case 4: return launch_pair_b<4>(kp, g.b_bits, stream);
+    case 8: return launch_pair_b<8>(kp, g.b_bits, stream);
+    default: return OQ_ERR_UNSUPPORTED;
+  }
+}
+
+}  // namespace oq

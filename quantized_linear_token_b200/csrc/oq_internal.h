@@ -78,5 +78,9 @@ struct GemmArgs {
   int* err;
 };
 oq_status gemm_launch(const GemmArgs& g, void* stream);
+// paired-CTA contraction (oq_gemm_pair.cu); OQ_ERR_UNSUPPORTED unless N % 256 == 0
+oq_status gemm_pair_launch(const GemmArgs& g, void* stream);
+// prmt decode tables of a codebook's fp16 levels (oq_gemm.cu)
+void make_decode_tables(int bits, const uint16_t* levels, uint32_t* t);
 
 }  // namespace oq
