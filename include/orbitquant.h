@@ -189,6 +189,29 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
                           const uint32_t* Wcodes, const float* r, float* y,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * oq_linear_fused_static -- the same computation as oq_linear_fused for
+ * callers that cannot allocate device memory: code running inside a CUDA
+ * graph capture, runtimes that give plug-ins no allocator, loops where an
+ * allocation or the synchronisation it implies is not allowed.  (The pages
+ * have no counterpart; this is an interface for such callers.)
+ *   The scratch that oq_linear_fused takes as `workspace` comes instead from a
+ *   fixed array of OQ_STATIC_SCRATCH_BYTES bytes in device memory that the
+ *   library reserves on every GPU that loads it, until the process exits.
+ *   No call allocates or frees memory.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   Every call shares the array: calls that overlap on the GPU (different
+ *   streams or host threads) race and give wrong results.
+ *   Arguments as for oq_linear_fused.  Errors: OQ_ERR_INVALID_ARG when the
+ *   batch needs more scratch than the array holds, i.e. when
+ *   oq_linear_fused_workspace_size(layer, T) > OQ_STATIC_SCRATCH_BYTES
+ *   (at d_in = 3072 and 4-bit activations about 10900 tokens).
+ */
+#define OQ_STATIC_SCRATCH_BYTES (16u << 20)
+oq_status oq_linear_fused_static(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
+                                 const uint32_t* Wcodes, const float* r, float* y, void* stream);
+
 /* Reads and clears the layer's device error word.  Synchronizes the device.
  * Returns OQ_OK, OQ_ERR_TIMEOUT or OQ_ERR_DEVICE. */
 oq_status oq_poll_error(const oq_layer* layer);

@@ -26,7 +26,7 @@ OQ_FLAG_GAUSSIAN_MARGINAL = 2
 EXPORTS = (
     "oq_codebook_build", "oq_rotation_build", "oq_layer_create", "oq_layer_destroy", "oq_layer_get_info", "oq_layer_get_perm",
     "oq_rotate_quantize", "oq_weight_prepare", "oq_linear", "oq_linear_fused_workspace_size",
-    "oq_linear_fused", "oq_poll_error", "oq_last_error", "oq_status_string",
+    "oq_linear_fused", "oq_linear_fused_static", "oq_poll_error", "oq_last_error", "oq_status_string",
 )
 
 
@@ -79,6 +79,7 @@ def load_library(path: str = LIB_PATH):
         "oq_linear": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_linear_fused_workspace_size": (sz, [vp, i64]),
         "oq_linear_fused": (i32, [vp, vp, i32, i64, vp, vp, vp, vp, sz, vp]),
+        "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
         "oq_poll_error": (i32, [vp]),
         "oq_last_error": (ctypes.c_char_p, []),
         "oq_status_string": (ctypes.c_char_p, [i32]),
@@ -242,6 +243,20 @@ def oq_linear_fused(layer: Layer, x, Wcodes, r, y=None, workspace=None):
                                           _dev(r, "r"), _dev(y, "y"), _dev(workspace, "workspace"),
                                           workspace.numel() * workspace.element_size(), _stream(x)),
            "oq_linear_fused")
+    return y
+
+
+def oq_linear_fused_static(layer: Layer, x, Wcodes, r, y=None):
+    """x [T, d_in] -> y [T, d_out] fp32 without any device allocation by the
+    library: its scratch is a fixed array the library reserves per GPU (see
+    include/orbitquant.h).  Calls that overlap on the GPU race on it."""
+    torch = _torch()
+    T = x.shape[0]
+    if y is None:
+        y = torch.empty((T, layer.d_out), dtype=torch.float32, device=x.device)
+    _check(load_library().oq_linear_fused_static(layer.handle, _dev(x, "x"), _dtype_code(x), T,
+                                                 _dev(Wcodes, "Wcodes"), _dev(r, "r"), _dev(y, "y"), _stream(x)),
+           "oq_linear_fused_static")
     return y
 
 
