@@ -146,6 +146,31 @@ def oracle_cpu_rate(wl, lay, seconds: float, chunk: int = 32):
     return done / el, el, done, threads
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+def rank_batch(wl, d: int, tokens: int, rank: int):
+    """This rank's own batch: weak scaling gives every rank `tokens` tokens of
+    the workload's recipe, drawn from the rank's own seeded stream."""
+    from quantized_linear_token_b200 import workloads as W
+    return W.activations(wl, d, tokens=tokens, stream=rank)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank number over all ranks (a no-op on one process)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, tokens_per_rank: int, steps: int, max_total_ms: float) -> float:
+    """Tokens per second of the whole job: all ranks' tokens over the slowest
+    rank's timed total."""
+    return world * tokens_per_rank * steps / (max_total_ms * 1e-3)
+
+
 # ------------------------------------------------------------------ our arm
 def run_ours(args):
     import numpy as np
@@ -172,7 +197,7 @@ def run_ours(args):
     wl = W.WORKLOADS[args.workload]
     lay = wl.layers[0]
     T, d, dout = (args.tokens or wl.tokens), lay.d_in, lay.d_out
-    x_np = W.activations(wl, d, tokens=T)
+    x_np = rank_batch(wl, d, T, rank)
     Wm = W.weights(wl, lay)
     x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(dev)
     layer = B.oq_layer_create(d, dout, W.ROTATION_SEED, lay.a_bits, lay.w_bits)
@@ -219,11 +244,7 @@ def run_ours(args):
     t_rq = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     t_mm = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     t_step = [a + b for a, b in zip(t_rq, t_mm)]
-    total_ms = sum(t_step)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(t_step), dev)
     B.oq_poll_error(layer)
 
     # fused call, same workload (one C call, both kernels)
@@ -257,11 +278,7 @@ def run_ours(args):
         eve[i][1].record(stream)
     torch.cuda.synchronize()
     t_e2e = [eve[i][0].elapsed_time(eve[i][1]) for i in range(K)]
-    e2e_ms = sum(t_e2e)
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(sum(t_e2e), dev)
     B.oq_poll_error(layer)
 
     peaks = load_peaks()
@@ -273,7 +290,7 @@ def run_ours(args):
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
     out = {
         "metric": METRIC,
-        "value": world * T * K / (total_ms * 1e-3),
+        "value": whole_job_rate(world, T, K, total_ms),
         "unit": UNIT,
         "n_gpus": world,
         "steps": K,
@@ -308,7 +325,7 @@ def run_ours(args):
         },
         "fused": {"value": T / (statistics.mean(t_fused) * 1e-3), "unit": UNIT,
                   "ms_per_call": statistics.mean(t_fused)},
-        "e2e": {"value": world * T * K / (e2e_ms * 1e-3), "unit": UNIT,
+        "e2e": {"value": whole_job_rate(world, T, K, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()),
                 "path": "pinned host x -> device, oq_linear_fused, y -> pinned host"},
