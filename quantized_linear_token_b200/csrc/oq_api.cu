@@ -198,7 +198,7 @@ static oq_status check_rows_input(const void* x, int32_t dtype, const char* who)
 
 static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t rows, int bits, const float* thr,
                     uint32_t* codes, float* norms, void* stream) {
-  RQArgs a;
+  RQArgs a{};
   a.src = x;
   a.src_dtype = dtype;
   a.rows = rows;

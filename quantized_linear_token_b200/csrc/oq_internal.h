@@ -51,7 +51,10 @@ struct RQArgs {
   const uint16_t* gather;    // per-thread gather offsets (kernel order)
   const uint32_t* signmask;  // or null
   const float* thr;          // host array of 128 scaled thresholds
-  uint32_t* codes;           // [rows, d*bits/32]
+  uint32_t* codes;           // [rows, d*bits/32], or
+  uint16_t* out16;           // fp16 levels [rows, d] (fused layer call); null otherwise
+  uint32_t dtab[4];          // prmt decode tables for out16
+  const uint16_t* lut8;      // device 8-bit level table for out16
   float* norms;              // [rows]
   int* err;
 };

@@ -5,24 +5,30 @@
 //   code_i = #{k : t_k < z_i / (s sqrt(h))}   (t = Lloyd-Max thresholds),
 // codes packed b bits each, 32 per group of b words, little-endian.
 //
-// Layout of the work, for one row ("token slot", d/E threads):
+// Layout of the work, for one row ("token slot", d/E threads; the block size
+// h is a compile-time constant so that every index below is fixed):
 //   * the row is copied into shared memory with one bulk async copy (double
 //     buffered: the next row streams in while this one is processed);
 //   * pass A: thread (j, c) of block j gathers the E rotated positions
 //     c + r (h/E), r = 0..E-1, through pi (gather offsets held in registers)
 //     and applies the butterflies of the high log2(E) bits in registers;
 //   * the values go through shared memory in a layout where every thread of
-//     pass B owns E consecutive positions (16-byte sub-chunks rotated by
-//     chunk index, so both the scattered writes and the vector reads are free
-//     of bank conflicts);
+//     pass B owns E consecutive positions (the 16-byte sub-chunks of chunk q
+//     are XOR-swizzled by q, so both the scattered writes -- one LOP3 of a
+//     compile-time offset per value -- and the vector reads are free of bank
+//     conflicts);
 //   * pass B applies the remaining low bits, compares with the thresholds
-//     scaled by s sqrt(h), packs and stores the codes with vector stores.
+//     scaled by s sqrt(h), packs and stores the codes with vector stores (or,
+//     for the fused layer call, stores the codes' fp16 levels: the operand
+//     the tensor-core contraction reads).
+// Butterflies with stride >= 2 use the paired fp32 adds of sm_100 (f32x2).
 // When h <= 64 a thread holds a whole block and pass B is skipped.
 #include <cuda_bf16.h>
 
 #include <algorithm>
 #include <cstring>
 
+#include "oq_decode.cuh"
 #include "oq_internal.h"
 #include "oq_ptx.cuh"
 
@@ -52,41 +58,73 @@ namespace {
 struct RQKParams {
   const void* src;
   int64_t rows;
-  int d, h, log_h, NT, S, e;
+  int d, NT, S;
   int work_words;      // per slot
   int stage_bytes;     // per buffer per slot
+  int has_signs;
   const uint16_t* gather;
   const uint32_t* signmask;
-  uint32_t* codes;
+  uint32_t* codes;     // packed codes, or
+  uint16_t* out16;     // fp16 levels [rows, d] (fused layer call)
   float* norms;
   int* err;
+  uint32_t dtab[4];    // prmt decode tables of the levels (out16)
+  const uint16_t* lut8;  // 8-bit levels (out16)
   float thr[128];      // sqrt(h) * positive thresholds tau_1.., +inf padded
 };
 
 template <typename XT>
-__device__ __forceinline__ float load_x(const unsigned char* stage, uint32_t idx) {
+__device__ __forceinline__ float load_x(uint32_t stage_addr, uint32_t idx) {
   if constexpr (sizeof(XT) == 2) {
-    const unsigned short v = *reinterpret_cast<const unsigned short*>(stage + 2u * idx);
+    uint16_t v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(stage_addr + 2u * idx));
     return __uint_as_float(((uint32_t)v) << 16);
   } else {
-    return *reinterpret_cast<const float*>(stage + 4u * idx);
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(stage_addr + 4u * idx));
+    return v;
   }
 }
 
-// in-register Walsh-Hadamard butterflies over register-index bits [lo, hi)
+// (a0, a1) <- (a0 + b0, a1 + b1), (b0, b1) <- (a0 - b0, a1 - b1) with the
+// paired fp32 adds of sm_100
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
+  asm("{\n\t.reg .b64 A, B, S, D;\n\t"
+      "mov.b64 A, {%0, %1};\n\tmov.b64 B, {%2, %3};\n\t"
+      "add.rn.f32x2 S, A, B;\n\tsub.rn.f32x2 D, A, B;\n\t"
+      "mov.b64 {%0, %1}, S;\n\tmov.b64 {%2, %3}, D;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+
+// in-register Walsh-Hadamard butterflies over register-index bits [LO, HI)
 template <int E, int LO, int HI>
 __device__ __forceinline__ void fwht_regs(float (&v)[E]) {
 #pragma unroll
   for (int s = (1 << LO); s < (1 << HI); s <<= 1) {
+    if (s == 1) {
 #pragma unroll
-    for (int r = 0; r < E; ++r) {
-      if ((r & s) == 0) {
-        const float a = v[r], b = v[r + s];
+      for (int r = 0; r < E; r += 2) {
+        const float a = v[r], b = v[r + 1];
         v[r] = a + b;
-        v[r + s] = a - b;
+        v[r + 1] = a - b;
       }
+    } else {
+#pragma unroll
+      for (int r = 0; r < E; r += 2)
+        if ((r & s) == 0) bfly2(v[r], v[r + 1], v[r + s], v[r + s + 1]);
     }
   }
+}
+
+// Word offset (inside its block) of the value that thread c of a block holds
+// in register r after pass A, minus the thread-dependent part: the value at
+// in-block position pos = c + r*HE lives in chunk q = pos / E, sub-chunk
+// v = (pos % E) / 4 stored at slot v ^ (q mod E/4).  With cb = c / 4 and
+// pos % E = A_r + c (A_r a multiple of HE), the offset is
+//   (scatter_imm(r) ^ 4 cb) | (c & 3).
+template <int E, int HE>
+__host__ __device__ constexpr uint32_t scatter_imm(int r) {
+  return (uint32_t)(E * ((r * HE) / E) + 4 * ((((r * HE) % E) / 4) ^ (((r * HE) / E) & (E / 4 - 1))));
 }
 
 // number of thresholds strictly below `a` among th[0..n-1] (sorted, last = +inf)
@@ -110,32 +148,47 @@ __device__ __forceinline__ int count_below(const float* th, float a) {
   }
 }
 
-template <int BITS, int E, int PASSES, typename XT, bool SIGNS>
-__global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_constant__ RQKParams p) {
-  constexpr int N_HALF = 1 << (BITS - 1);   // levels on each side of 0
+__host__ __device__ constexpr int elems_per_thread(int h) { return h <= 64 ? h : (h <= 1024 ? 32 : 64); }
+__host__ __device__ constexpr int log2i(int x) { return x <= 1 ? 0 : 1 + log2i(x / 2); }
+
+// register budget: 112 for 32 values per thread (3 CTAs of 192 per SM),
+// 168 for 64 values per thread
+template <int BITS, int LOG_H, typename XT, bool OUT16>
+__global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
+    rq_kernel(const __grid_constant__ RQKParams p) {
+  constexpr int H = 1 << LOG_H;
+  constexpr int E = elems_per_thread(H);
+  constexpr int LOGE = log2i(E);
+  constexpr int HE = H / E;
+  constexpr int PASSES = (H <= 64) ? 1 : 2;
+  constexpr int PAD = (PASSES == 2 && HE < 32) ? HE : 0;   // words between blocks
+  constexpr int N_HALF = 1 << (BITS - 1);
   constexpr int NTH = (BITS <= 4) ? N_HALF : 1;
   extern __shared__ __align__(1024) unsigned char smem[];
 
-  const int S = p.S, NT = p.NT, d = p.d, h = p.h;
-  const int HE = h / E;
+  const int S = p.S, NT = p.NT, d = p.d;
   const int slot_raw = threadIdx.x / NT;
   const bool active = slot_raw < S;
   const int slot = active ? slot_raw : 0;
   const int tid = active ? (int)threadIdx.x - slot * NT : 0;
-  const int j = tid / HE, c = tid - (tid / HE) * HE;
+  const int j = tid / HE, c = tid % HE;
 
-  // shared memory: mbarriers | reduction partials | 8-bit thresholds | slots
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem);                      // [S][2]
-  float* red = reinterpret_cast<float*>(smem + 16 * S);                    // [blockDim]
-  float* thr8 = red + blockDim.x;                                          // [S][128] (8-bit)
-  unsigned char* slots = smem + (((16 * S + 4 * blockDim.x + (BITS == 8 ? 512 * S : 0)) + 1023) & ~1023);
+  // shared memory: mbarriers | reduction partials | 8-bit thresholds | 8-bit
+  // levels | slots (two row buffers + exchange area each)
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem);
+  float* red = reinterpret_cast<float*>(smem + 16 * S);
+  float* thr8 = red + blockDim.x;
+  uint16_t* lut8 = reinterpret_cast<uint16_t*>(thr8 + (BITS == 8 ? 128 * S : 0));
+  unsigned char* slots =
+      smem + (((16 * S + 4 * blockDim.x + (BITS == 8 ? 512 * S + 512 : 0)) + 1023) & ~1023);
   const int slot_bytes = 2 * p.stage_bytes + 4 * p.work_words;
   unsigned char* stage0 = slots + (size_t)slot * slot_bytes;
   float* work = reinterpret_cast<float*>(stage0 + 2 * p.stage_bytes);
+  const uint32_t stage0_addr = smem_u32(stage0);
 
-  // gather offsets and sign bits of this thread, kept in registers
+  // this thread's gather offsets (pairs of 16-bit channel indices) and signs
   uint32_t gidx[E / 2];
-  uint32_t smask[E / 32];
+  uint32_t smask[E / 32 > 0 ? E / 32 : 1];
   {
     const uint4* g4 = reinterpret_cast<const uint4*>(p.gather + (size_t)tid * E);
 #pragma unroll
@@ -147,12 +200,13 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
       gidx[4 * q + 3] = v.w;
     }
 #pragma unroll
-    for (int q = 0; q < E / 32; ++q) smask[q] = (SIGNS && active) ? __ldg(p.signmask + (size_t)tid * (E / 32) + q) : 0u;
+    for (int q = 0; q < (E / 32 > 0 ? E / 32 : 1); ++q)
+      smask[q] = (p.has_signs && active) ? __ldg(p.signmask + (size_t)tid * (E / 32) + q) : 0u;
   }
-  float th[NTH];
-#pragma unroll
-  for (int k = 0; k < NTH; ++k) th[k] = p.thr[k];
+  // thresholds and decode tables stay in the parameter (constant) bank
 
+  if (OUT16 && BITS == 8)
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = p.lut8[i];
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * S; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
@@ -163,8 +217,10 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
   const int words_per_row = d * BITS / 32;
   const uint32_t row_bytes = (uint32_t)d * (uint32_t)sizeof(XT);
   const unsigned char* src = static_cast<const unsigned char*>(p.src);
+  // segmented warp reduction width: lanes of one slot share aligned segments
+  const int W = NT & -NT;
+  const int Wc = W < 32 ? W : 32;
 
-  // prologue: first row of this slot
   if (active && tid == 0) {
     const int64_t t0 = (int64_t)blockIdx.x * S + slot;
     if ((int64_t)blockIdx.x < groups && t0 < p.rows) {
@@ -178,7 +234,6 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
     const int64_t t = G * S + slot;
     const bool valid = active && t < p.rows;
     const int buf = it & 1;
-    // prefetch the next row of this slot into the other buffer
     bool issued = false;
     if (active && tid == 0) {
       const int64_t Gn = G + gridDim.x, tn = Gn * S + slot;
@@ -193,38 +248,33 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
     if (valid) ok = mbar_wait(&mbar[2 * slot + buf], (uint32_t)(it >> 1) & 1u, p.err);
 
     // ---------------- pass A: gather through pi, high-bit butterflies
-    const unsigned char* stage = stage0 + buf * p.stage_bytes;
+    const uint32_t stage_addr = stage0_addr + (uint32_t)(buf * p.stage_bytes);
     float v[E];
     float ss = 0.f;
 #pragma unroll
     for (int r = 0; r < E; ++r) {
       const uint32_t gi = (r & 1) ? (gidx[r >> 1] >> 16) : (gidx[r >> 1] & 0xFFFFu);
-      float x = valid ? load_x<XT>(stage, gi) : 0.f;
-      if constexpr (SIGNS) {
-        if ((smask[r >> 5] >> (r & 31)) & 1u) x = -x;
-      }
-      ss = fmaf(x, x, ss);
-      v[r] = x;
+      v[r] = valid ? load_x<XT>(stage_addr, gi) : 0.f;
     }
-    constexpr int LOGE = (E == 32) ? 5 : (E == 64 ? 6 : (E == 16 ? 4 : 0));
-    static_assert(LOGE > 0, "E must be 16, 32 or 64");
+    if (p.has_signs) {
+#pragma unroll
+      for (int r = 0; r < E; ++r)
+        if ((smask[r >> 5] >> (r & 31)) & 1u) v[r] = -v[r];
+    }
+#pragma unroll
+    for (int r = 0; r < E; ++r) ss = fmaf(v[r], v[r], ss);
     fwht_regs<E, 0, LOGE>(v);
 
-    if (PASSES == 2 && active) {
-      // scatter into the pass-B layout of block j (see file comment)
-      const int pad = HE < 32 ? HE : 0;
-      float* wb = work + j * (h + pad);
+    if constexpr (PASSES == 2) {
+      if (active) {
+        float* wb = work + j * (H + PAD);
+        const uint32_t cb4 = (uint32_t)(c >> 2) << 2, c3 = (uint32_t)(c & 3);
 #pragma unroll
-      for (int r = 0; r < E; ++r) {
-        const int pos = c + r * HE;
-        const int q = pos / E, w = pos - q * E;
-        wb[q * E + ((((w >> 2) + q) & (E / 4 - 1)) << 2) + (w & 3)] = v[r];
+        for (int r = 0; r < E; ++r) wb[(scatter_imm<E, HE>(r) ^ cb4) | c3] = v[r];
       }
     }
 
     // ---------------- norm: segmented warp reduction, then per slot
-    const int W = NT & -NT;                      // lanes per aligned segment
-    const int Wc = W < 32 ? W : 32;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1)
       if (off < Wc) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -232,7 +282,6 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
 
     const int failed = __syncthreads_or(!ok);
     if (failed) {
-      // let a copy still in flight land before the CTA leaves (bounded)
       if (issued) mbar_wait(&mbar[2 * slot + (buf ^ 1)], (uint32_t)((it + 1) >> 1) & 1u, p.err);
       break;
     }
@@ -247,53 +296,36 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
     // ---------------- pass B: low-bit butterflies, quantize, pack
     float z[E];
     if constexpr (PASSES == 2) {
-      const int pad = HE < 32 ? HE : 0;
-      const float* wb = work + j * (h + pad) + c * E;
+      const float* wb = work + j * (H + PAD) + c * E;
 #pragma unroll
       for (int q = 0; q < E / 4; ++q) {
-        const float4 f = *reinterpret_cast<const float4*>(wb + (((q + c) & (E / 4 - 1)) << 2));
+        const float4 f = *reinterpret_cast<const float4*>(wb + ((q ^ (c & (E / 4 - 1))) << 2));
         z[4 * q + 0] = f.x;
         z[4 * q + 1] = f.y;
         z[4 * q + 2] = f.z;
         z[4 * q + 3] = f.w;
       }
+      fwht_regs<E, 0, LOG_H - LOGE>(z);
     } else {
 #pragma unroll
       for (int r = 0; r < E; ++r) z[r] = v[r];
     }
 
-    if constexpr (PASSES == 2) {
-      // remaining bits [0, log_h - LOGE): at most LOGE of them
-      const int nb = p.log_h - LOGE;
-#pragma unroll
-      for (int b = 0; b < LOGE; ++b) {
-        if (b < nb) {
-          const int st = 1 << b;
-#pragma unroll
-          for (int r = 0; r < E; ++r) {
-            if ((r & st) == 0) {
-              const float a0 = z[r], b0 = z[r + st];
-              z[r] = a0 + b0;
-              z[r + st] = a0 - b0;
-            }
-          }
-        }
-      }
-    }
-
     if constexpr (BITS == 8) {
-      // this token's scaled thresholds (127 and +inf) in shared memory
+      // this token's scaled thresholds (127 and +inf) in shared memory; a
+      // zero token gets +inf everywhere (all coordinates 0 -> code L/2 - 1)
       if (valid)
-        for (int k = tid; k < 128; k += NT) thr8[slot * 128 + k] = p.thr[k] * s;
+        for (int k = tid; k < 128; k += NT) thr8[slot * 128 + k] = (s > 0.f) ? p.thr[k] * s : INFINITY;
       __syncthreads();
     }
 
     if (valid) {
+      // thresholds of this token; a zero token (s = 0) has every coordinate
+      // 0 and takes code L/2 - 1: +inf thresholds give exactly that
       float ts[NTH];
 #pragma unroll
-      for (int k = 0; k < NTH; ++k) ts[k] = th[k] * s;
-      const int pos0 = (PASSES == 2) ? (j * h + c * E) : (j * h);
-      uint32_t* crow = p.codes + (size_t)t * words_per_row;
+      for (int k = 0; k < NTH; ++k) ts[k] = (s > 0.f) ? p.thr[k] * s : INFINITY;
+      const int pos0 = (PASSES == 2) ? (j * H + c * E) : (j * H);
 #pragma unroll
       for (int gi = 0; gi < E / 32; ++gi) {
         // quantize 32 consecutive positions straight into BITS packed words
@@ -319,24 +351,36 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
               if (t8[lo + st - 1] < acmp) lo += st;
             cnt = lo;
           }
-          int cd = pos ? (N_HALF + cnt) : (N_HALF - 1 - cnt);
-          if (s == 0.f) cd = N_HALF - 1;
-          const uint32_t cv = (uint32_t)cd;
+          const uint32_t cv = (uint32_t)(pos ? (N_HALF + cnt) : (N_HALF - 1 - cnt));
           const int bit = i * BITS;
           w[bit >> 5] |= cv << (bit & 31);
           if ((bit & 31) + BITS > 32) w[(bit >> 5) + 1] |= cv >> (32 - (bit & 31));
         }
-        uint32_t* dst = crow + (size_t)((pos0 >> 5) + gi) * BITS;
-        if constexpr (BITS == 4) {
-          *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-        } else if constexpr (BITS == 2) {
-          *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-        } else if constexpr (BITS == 8) {
-          reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        } else {
+        if constexpr (OUT16) {
+          // the levels of these 32 codes as fp16: the contraction's A operand
+          uint4* dst = reinterpret_cast<uint4*>(p.out16 + (size_t)t * d + pos0 + gi * 32);
 #pragma unroll
-          for (int q = 0; q < BITS; ++q) dst[q] = w[q];
+          for (int q = 0; q < 4; ++q) {
+            uint4 o;
+            if constexpr (BITS == 4) o = dec4(w[q], p.dtab);
+            else if constexpr (BITS == 2) o = dec2((w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu, p.dtab);
+            else if constexpr (BITS == 3) o = decode_chunk<3>(make_uint4(w[0], w[1], w[2], 0u), q, p.dtab, lut8);
+            else o = dec8(w[2 * q], w[2 * q + 1], lut8);
+            dst[q] = o;
+          }
+        } else {
+          uint32_t* dst = p.codes + (size_t)t * words_per_row + (size_t)((pos0 >> 5) + gi) * BITS;
+          if constexpr (BITS == 4) {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+          } else if constexpr (BITS == 2) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+          } else if constexpr (BITS == 8) {
+            reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) dst[q] = w[q];
+          }
         }
       }
       if (tid == 0) p.norms[t] = s;
@@ -345,19 +389,22 @@ __global__ void __launch_bounds__(E == 64 ? 256 : 448) rq_kernel(const __grid_co
   }
 }
 
-template <int BITS, int E, int PASSES, typename XT, bool SIGNS>
-oq_status launch_t(const RQArgs& a, const RQKParams& kp_in, void* stream) {
+template <int BITS, int LOG_H, typename XT, bool OUT16>
+oq_status launch_t(const RQKParams& kp_in, void* stream) {
+  constexpr int H = 1 << LOG_H;
+  constexpr int E = elems_per_thread(H);
+  constexpr int MAXT = (E == 64) ? 256 : 448;
   RQKParams kp = kp_in;
-  auto kern = rq_kernel<BITS, E, PASSES, XT, SIGNS>;
+  auto kern = rq_kernel<BITS, LOG_H, XT, OUT16>;
   const int NT = kp.NT;
   int S = 1;
   while (S * NT < 128 && S < 64) S *= 2;
   const int threads = ((S * NT + 31) / 32) * 32;
-  if (threads > (E == 64 ? 256 : 448)) return OQ_ERR_UNSUPPORTED;
+  if (threads > MAXT) return OQ_ERR_UNSUPPORTED;
   kp.S = S;
-  kp.stage_bytes = (int)(((size_t)a.d * sizeof(XT) + 15) & ~(size_t)15);
+  kp.stage_bytes = (int)(((size_t)kp.d * sizeof(XT) + 15) & ~(size_t)15);
   const int slot_bytes = 2 * kp.stage_bytes + 4 * kp.work_words;
-  const size_t head = ((16 * S + 4 * threads + (BITS == 8 ? 512 * S : 0)) + 1023) & ~(size_t)1023;
+  const size_t head = ((16 * S + 4 * threads + (BITS == 8 ? 512 * S + 512 : 0)) + 1023) & ~(size_t)1023;
   const size_t smem = head + (size_t)S * slot_bytes;
   if (smem > 227 * 1024) return OQ_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -370,7 +417,7 @@ oq_status launch_t(const RQArgs& a, const RQKParams& kp_in, void* stream) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
   if (per_sm < 1) per_sm = 1;
-  const int64_t groups = (a.rows + S - 1) / S;
+  const int64_t groups = (kp.rows + S - 1) / S;
   const int64_t grid = std::min<int64_t>(groups, (int64_t)sms * per_sm);
   kern<<<(unsigned)grid, threads, smem, static_cast<cudaStream_t>(stream)>>>(kp);
   e = cudaGetLastError();
@@ -379,6 +426,33 @@ oq_status launch_t(const RQArgs& a, const RQKParams& kp_in, void* stream) {
     return OQ_ERR_CUDA;
   }
   return OQ_OK;
+}
+
+template <int BITS, typename XT, bool OUT16>
+oq_status launch_h(const RQKParams& kp, int log_h, void* stream) {
+  switch (log_h) {
+    case 5: return launch_t<BITS, 5, XT, OUT16>(kp, stream);
+    case 6: return launch_t<BITS, 6, XT, OUT16>(kp, stream);
+    case 7: return launch_t<BITS, 7, XT, OUT16>(kp, stream);
+    case 8: return launch_t<BITS, 8, XT, OUT16>(kp, stream);
+    case 9: return launch_t<BITS, 9, XT, OUT16>(kp, stream);
+    case 10: return launch_t<BITS, 10, XT, OUT16>(kp, stream);
+    case 11: return launch_t<BITS, 11, XT, OUT16>(kp, stream);
+    case 12: return launch_t<BITS, 12, XT, OUT16>(kp, stream);
+    default: return OQ_ERR_UNSUPPORTED;
+  }
+}
+
+template <int BITS>
+oq_status launch_bits(const RQKParams& kp, const RQArgs& a, void* stream) {
+  const bool bf = a.src_dtype == OQ_DTYPE_BF16;
+  if (a.out16) {
+    // fp16 operand output only for bf16 activations (the fused layer call)
+    if (!bf) return OQ_ERR_UNSUPPORTED;
+    return launch_h<BITS, __nv_bfloat16, true>(kp, a.log_h, stream);
+  }
+  if (bf) return launch_h<BITS, __nv_bfloat16, false>(kp, a.log_h, stream);
+  return launch_h<BITS, float, false>(kp, a.log_h, stream);
 }
 
 }  // namespace
@@ -390,50 +464,29 @@ oq_status rq_launch(const RQArgs& a, void* stream) {
   kp.src = a.src;
   kp.rows = a.rows;
   kp.d = a.d;
-  kp.h = a.h;
-  kp.log_h = a.log_h;
   const int E = rq_elems_per_thread(a.h);
-  kp.e = E;
   kp.NT = a.d / E;
   const int HE = a.h / E;
   kp.work_words = (a.h <= 64) ? 0 : (a.d / a.h) * (a.h + (HE < 32 ? HE : 0));
+  kp.has_signs = a.signmask != nullptr;
   kp.gather = a.gather;
   kp.signmask = a.signmask;
   kp.codes = a.codes;
+  kp.out16 = a.out16;
   kp.norms = a.norms;
   kp.err = a.err;
+  if (a.out16) {
+    for (int k = 0; k < 4; ++k) kp.dtab[k] = a.dtab[k];
+    kp.lut8 = a.lut8;
+  }
   std::memcpy(kp.thr, a.thr, sizeof(kp.thr));
-  const bool sg = a.signmask != nullptr;
-  const bool bf = a.src_dtype == OQ_DTYPE_BF16;
-
-#define OQ_RQ_CASE(BITS, EE, PP, XT, SG) \
-  return launch_t<BITS, EE, PP, XT, SG>(a, kp, stream);
-#define OQ_RQ_SHAPES(BITS, XT, SG)                                   \
-  switch (a.h) {                                                     \
-    case 32: OQ_RQ_CASE(BITS, 32, 1, XT, SG)                         \
-    case 64: OQ_RQ_CASE(BITS, 64, 1, XT, SG)                         \
-    case 128: case 256: case 512: case 1024: OQ_RQ_CASE(BITS, 32, 2, XT, SG) \
-    case 2048: case 4096: OQ_RQ_CASE(BITS, 64, 2, XT, SG)            \
-    default: return OQ_ERR_UNSUPPORTED;                              \
-  }
-#define OQ_RQ_DT(BITS)                                               \
-  if (bf) {                                                          \
-    if (sg) { OQ_RQ_SHAPES(BITS, __nv_bfloat16, true) }              \
-    else { OQ_RQ_SHAPES(BITS, __nv_bfloat16, false) }                \
-  } else {                                                           \
-    if (sg) { OQ_RQ_SHAPES(BITS, float, true) }                      \
-    else { OQ_RQ_SHAPES(BITS, float, false) }                        \
-  }
   switch (a.bits) {
-    case 2: OQ_RQ_DT(2)
-    case 3: OQ_RQ_DT(3)
-    case 4: OQ_RQ_DT(4)
-    case 8: OQ_RQ_DT(8)
+    case 2: return launch_bits<2>(kp, a, stream);
+    case 3: return launch_bits<3>(kp, a, stream);
+    case 4: return launch_bits<4>(kp, a, stream);
+    case 8: return launch_bits<8>(kp, a, stream);
     default: return OQ_ERR_UNSUPPORTED;
   }
-#undef OQ_RQ_DT
-#undef OQ_RQ_SHAPES
-#undef OQ_RQ_CASE
 }
 
 }  // namespace oq
