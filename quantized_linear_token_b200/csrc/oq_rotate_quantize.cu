@@ -397,8 +397,10 @@ oq_status launch_t(const RQKParams& kp_in, void* stream) {
   RQKParams kp = kp_in;
   auto kern = rq_kernel<BITS, LOG_H, XT, OUT16>;
   const int NT = kp.NT;
+  // one row per CTA once a row has 64 threads: small CTAs pack into the SM
+  // sub-partitions' register files better than 6-warp ones
   int S = 1;
-  while (S * NT < 128 && S < 64) S *= 2;
+  while (S * NT < 64 && S < 64) S *= 2;
   const int threads = ((S * NT + 31) / 32) * 32;
   if (threads > MAXT) return OQ_ERR_UNSUPPORTED;
   kp.S = S;
@@ -408,6 +410,8 @@ oq_status launch_t(const RQKParams& kp_in, void* stream) {
   const size_t smem = head + (size_t)S * slot_bytes;
   if (smem > 227 * 1024) return OQ_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) {
     set_error(std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
     return OQ_ERR_CUDA;
