@@ -180,9 +180,13 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
 /*
  * oq_linear_fused -- x -> y in one call: the rotate-quantize step produces
  * the A operand of the contraction (same results as oq_rotate_quantize
- * followed by oq_linear).  `workspace` is caller-owned device scratch of at
- * least oq_linear_fused_workspace_size(layer, T) bytes (the packed
- * activation codes and norms); it may be reused between calls on one stream.
+ * followed by oq_linear).  With bf16 x and d_out % 256 == 0 the rotate-quantize
+ * kernel writes the fp16 levels of the activation codes, which the contraction
+ * reads with TMA (only the weight codes are decoded in the contraction);
+ * otherwise the packed codes pass through the workspace.  `workspace` is
+ * caller-owned device scratch of at least
+ * oq_linear_fused_workspace_size(layer, T) bytes (the A operand and the
+ * norms), 256-byte aligned; it may be reused between calls on one stream.
  */
 size_t oq_linear_fused_workspace_size(const oq_layer* layer, int64_t T);
 oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
@@ -206,7 +210,7 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  *   Arguments as for oq_linear_fused.  Errors: OQ_ERR_INVALID_ARG when the
  *   batch needs more scratch than the array holds, i.e. when
  *   oq_linear_fused_workspace_size(layer, T) > OQ_STATIC_SCRATCH_BYTES
- *   (at d_in = 3072 and 4-bit activations about 10900 tokens).
+ *   (at d_in = 3072 with d_out % 256 == 0 about 2700 tokens).
  */
 #define OQ_STATIC_SCRATCH_BYTES (16u << 20)
 oq_status oq_linear_fused_static(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,

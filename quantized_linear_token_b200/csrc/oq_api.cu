@@ -3,6 +3,7 @@
 // and dispatch to the kernels.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -238,9 +239,11 @@ oq_status oq_weight_prepare(const oq_layer* L, const void* W, int32_t W_dtype, u
 }
 
 static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T,
-                             const uint32_t* Wcodes, const float* r, float* y, void* stream) {
-  GemmArgs g;
+                             const uint32_t* Wcodes, const float* r, float* y, void* stream,
+                             const uint16_t* a_f16 = nullptr) {
+  GemmArgs g{};
   g.a_codes = codes;
+  g.a_f16 = a_f16;
   g.b_codes = Wcodes;
   g.a_scale = s;
   g.b_scale = r;
@@ -270,10 +273,26 @@ oq_status oq_linear(const oq_layer* L, const uint32_t* codes, const float* s, in
   return linear_impl(L, codes, s, T, Wcodes, r, y, stream);
 }
 
+// The fused call has two routes.  With bf16 activations and d_out % 256 == 0
+// the rotate-quantize kernel writes the fp16 levels of the codes (the
+// contraction's A operand) and the CTA-pair kernel reads them with TMA, so
+// only the weight codes are decoded during the contraction.  Otherwise the
+// packed codes go through the workspace to the code-decoding contraction.
+static bool fused_f16_route(const oq_layer* L, int32_t x_dtype) {
+  return x_dtype == OQ_DTYPE_BF16 && L->d_out % 256 == 0;
+}
+
+static size_t fused_codes_bytes(const oq_layer* L, int64_t T) {
+  return (size_t)T * ((size_t)L->d_in * L->a_bits / 32) * 4;
+}
+
+static size_t fused_f16_bytes(const oq_layer* L, int64_t T) { return (size_t)T * (size_t)L->d_in * 2; }
+
 size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
   if (!L || T <= 0) return 0;
-  const size_t codes = (size_t)T * ((size_t)L->d_in * L->a_bits / 32) * 4;
-  return ((codes + 255) & ~(size_t)255) + (size_t)T * 4;
+  size_t a = fused_codes_bytes(L, T);
+  if (L->d_out % 256 == 0) a = std::max(a, fused_f16_bytes(L, T));
+  return ((a + 255) & ~(size_t)255) + (size_t)T * 4;
 }
 
 oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
@@ -288,9 +307,32 @@ oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int
     return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: misaligned pointer (workspace needs 256 bytes)");
   if (workspace_bytes < oq_linear_fused_workspace_size(L, T))
     return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
-  uint32_t* codes = static_cast<uint32_t*>(workspace);
-  const size_t cbytes = (size_t)T * ((size_t)L->d_in * L->a_bits / 32) * 4;
-  float* s = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + ((cbytes + 255) & ~(size_t)255));
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (fused_f16_route(L, x_dtype)) {
+    uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
+    float* s = reinterpret_cast<float*>(ws + ((fused_f16_bytes(L, T) + 255) & ~(size_t)255));
+    RQArgs a{};
+    a.src = x;
+    a.src_dtype = x_dtype;
+    a.rows = T;
+    a.d = L->d_in;
+    a.h = L->h;
+    a.log_h = L->log_h;
+    a.bits = L->a_bits;
+    a.gather = L->d_gather_a;
+    a.signmask = L->d_signmask;
+    a.thr = L->thr_a;
+    a.out16 = a16;
+    make_decode_tables(L->a_bits, L->lv_a, a.dtab);
+    a.lut8 = L->d_levels_a;
+    a.norms = s;
+    a.err = L->d_error;
+    st = rq_launch(a, stream);
+    if (st != OQ_OK) return st;
+    return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
+  }
+  uint32_t* codes = reinterpret_cast<uint32_t*>(ws);
+  float* s = reinterpret_cast<float*>(ws + ((fused_codes_bytes(L, T) + 255) & ~(size_t)255));
   st = rq(L, x, x_dtype, T, L->a_bits, L->thr_a, codes, s, stream);
   if (st != OQ_OK) return st;
   return linear_impl(L, codes, s, T, Wcodes, r, y, stream);

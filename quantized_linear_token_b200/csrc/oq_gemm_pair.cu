@@ -21,6 +21,8 @@
 // multicast by tcgen05.commit to both CTAs' `empty` / `acc_full` barriers;
 // epilogue warps of both CTAs arrive on the even CTA's `acc_empty`.  Every
 // wait is bounded (oq_ptx.cuh).
+#include <cuda.h>
+
 #include <algorithm>
 #include <cstring>
 
@@ -47,7 +49,11 @@ constexpr uint32_t TMEM_COLS = 2 * PN;
 constexpr uint32_t FULL_LOCAL = NDEC / 32;           // one arrival per decoder warp
 constexpr uint32_t ACC_EMPTY_COUNT = 2 * 4;           // one per epilogue warp, both CTAs
 
+constexpr int EPI_BYTES = 4 * 2 * 32 * 32 * 4;   // per epilogue warp: two 32 x 32 fp32 staging boxes
+
 struct PairParams {
+  CUtensorMap a_map;          // fp16 A operand [M, K] (A_TMA kernels), 128B-swizzled boxes of 128 x 64
+  CUtensorMap y_map;          // fp32 y [M, N], 128B-swizzled boxes of 32 x 32 (epilogue stores)
   const uint32_t* a_codes;
   const uint32_t* b_codes;
   const float* a_scale;
@@ -63,18 +69,24 @@ struct PairParams {
   int* err;
 };
 
-template <int A_BITS, int B_BITS>
+// A_TMA: the A operand is already fp16 levels in global memory (written by
+// the rotate-quantize kernel in the fused layer call); one thread per CTA
+// fetches each 128 x 64 A tile with a TMA load in the swizzled layout, and
+// the decoders expand only the weight codes.
+template <int A_BITS, int B_BITS, bool A_TMA>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     gemm_pair_kernel(const __grid_constant__ PairParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  constexpr int QA = Fmt<A_BITS>::QP, QB = Fmt<B_BITS>::QP;
+  constexpr int QA = A_TMA ? 0 : Fmt<A_BITS>::QP, QB = Fmt<B_BITS>::QP;
+  constexpr uint32_t FULL_CTA = FULL_LOCAL + (A_TMA ? 1 : 0);   // + the TMA's expect_tx arrival
   constexpr int ITEMS_A = RM * QA, ITEMS = RM * QA + RN * QB;
   constexpr int IPT = (ITEMS + NDEC - 1) / NDEC;
 
-  uint16_t* lut8 = reinterpret_cast<uint16_t*>(smem + OS * STAGE_BYTES);
-  uint64_t* op_full = reinterpret_cast<uint64_t*>(smem + OS * STAGE_BYTES + 512);
+  unsigned char* epi = smem + OS * STAGE_BYTES;      // epilogue staging (1024-aligned)
+  uint16_t* lut8 = reinterpret_cast<uint16_t*>(smem + OS * STAGE_BYTES + EPI_BYTES);
+  uint64_t* op_full = reinterpret_cast<uint64_t*>(smem + OS * STAGE_BYTES + EPI_BYTES + 512);
   uint64_t* op_empty = op_full + OS;
   uint64_t* acc_full = op_empty + OS;
   uint64_t* acc_empty = acc_full + 2;
@@ -91,7 +103,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < OS; ++s) {
       // the even CTA also counts the odd CTA's forwarded arrival
-      mbar_init(&op_full[s], rank == 0 ? FULL_LOCAL + 1 : FULL_LOCAL);
+      mbar_init(&op_full[s], rank == 0 ? FULL_CTA + 1 : FULL_CTA);
       mbar_init(&op_empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -126,9 +138,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     for (int it = 0; it < IPT; ++it) {
       const int id = threadIdx.x + NDEC * it;
       const bool is_a = id < ITEMS_A;
-      const int r = is_a ? id / QA : (id - ITEMS_A) / QB;
+      const int r = is_a ? id / (QA ? QA : 1) : (id - ITEMS_A) / QB;
       item_r[it] = r;
-      item_q[it] = is_a ? id % QA : (id - ITEMS_A) % QB;
+      item_q[it] = is_a ? id % (QA ? QA : 1) : (id - ITEMS_A) % QB;
       row_off[it] = (is_a ? 0u : (uint32_t)A_TILE) + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
       xs[it] = (uint32_t)(r & 7) << 4;
     }
@@ -213,13 +225,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
     int s = 0, d_kb = 0;
     uint32_t n = 0;
-    int64_t g = 0;
+    int64_t g = 0, d_tile = 0;
+    auto a_row0 = [&](int64_t tile_i) {
+      return (int32_t)(((pair + tile_i * npairs) / p.n_tiles) * (2 * RM) + rank * RM);
+    };
+    int32_t d_m0 = a_row0(0);
     auto step = [&](const uint4 (&cur)[IPT], uint4 (&fut)[IPT]) -> bool {
       if (g + 2 < total) {
         fetch(f_kb, fut);
         advance();
       }
       if (n > 0 && !mbar_wait(&op_empty[s], (n - 1) & 1u, p.err)) return false;
+      if (A_TMA && threadIdx.x == 0) {
+        // A tile of this K block: rows past M and columns past K arrive as zeros
+        mbar_arrive_expect_tx(&op_full[s], (uint32_t)A_TILE);
+        tma_load_2d(smem + s * STAGE_BYTES, &p.a_map, d_kb * BK, d_m0, &op_full[s]);
+      }
       if ((d_kb + 1) * BK > p.K) decode(cur, s, true, d_kb);
       else decode(cur, s, false, d_kb);
       // this warp's tiles -> visible to the async proxy, then one arrival
@@ -231,7 +252,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         s = 0;
         ++n;
       }
-      if (++d_kb == nkb) d_kb = 0;
+      if (++d_kb == nkb) {
+        d_kb = 0;
+        ++d_tile;
+        d_m0 = a_row0(d_tile);
+      }
       ++g;
       return true;
     };
@@ -242,14 +267,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     }
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
     // ------------------------------------------------ epilogue (both CTAs)
+    // Each warp drains its 32 TMEM lanes (rows) in chunks of 32 columns,
+    // scales them, stages the 32 x 32 box in shared memory (128B swizzle,
+    // conflict-free) and writes it with one TMA store: full-line writes and
+    // a handful of instructions per chunk.  Rows past M are clipped by TMA.
     const int q = warp & 3;
+    unsigned char* ebuf = epi + q * (2 * 32 * 32 * 4);
     for (int64_t i = 0; i < my_tiles; ++i) {
       const int a = (int)(i & 1);
       const uint32_t u = (uint32_t)(i >> 1);
       if (!mbar_wait(&acc_full[a], u & 1u, p.err)) break;
       tc_fence_after();
       const int64_t tt = pair + i * npairs;
-      const int64_t row = (tt / p.n_tiles) * (2 * RM) + rank * RM + q * 32 + lane;
+      const int64_t row0 = (tt / p.n_tiles) * (2 * RM) + rank * RM + q * 32;
+      const int64_t row = row0 + lane;
       const int n0 = (int)(tt % p.n_tiles) * PN;
       const float srow = (row < p.M) ? __ldg(p.a_scale + row) * p.out_scale : 0.f;
 #pragma unroll 1
@@ -261,23 +292,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * PN + cc * 32), v);
         tmem_wait_ld();
-        if (row < p.M) {
-          float* dst = p.y + row * p.N + nb;
+        unsigned char* buf = ebuf + (cc & 1) * (32 * 32 * 4);
+        // the store that last read this buffer (two chunks ago) must be done
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        const uint32_t rb = smem_u32(buf) + (uint32_t)lane * 128u;
 #pragma unroll
-          for (int k4 = 0; k4 < 8; ++k4) {
-            float4 o;
-            o.x = __uint_as_float(v[4 * k4 + 0]) * srow * rr[k4].x;
-            o.y = __uint_as_float(v[4 * k4 + 1]) * srow * rr[k4].y;
-            o.z = __uint_as_float(v[4 * k4 + 2]) * srow * rr[k4].z;
-            o.w = __uint_as_float(v[4 * k4 + 3]) * srow * rr[k4].w;
-            reinterpret_cast<float4*>(dst)[k4] = o;
-          }
+        for (int k4 = 0; k4 < 8; ++k4) {
+          uint4 o;
+          o.x = __float_as_uint(__uint_as_float(v[4 * k4 + 0]) * srow * rr[k4].x);
+          o.y = __float_as_uint(__uint_as_float(v[4 * k4 + 1]) * srow * rr[k4].y);
+          o.z = __float_as_uint(__uint_as_float(v[4 * k4 + 2]) * srow * rr[k4].z);
+          o.w = __float_as_uint(__uint_as_float(v[4 * k4 + 3]) * srow * rr[k4].w);
+          st_shared_v4(rb + ((uint32_t)(k4 ^ (lane & 7)) << 4), o);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&p.y_map, nb, (int32_t)row0, buf);
+          bulk_commit();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[a]), 0));
     }
+    // every store has finished reading shared memory and writing y
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
   } else if (warp == MMA_WARP && rank == 0) {
     // ------------------------------------------------ paired MMA issuer (even CTA)
     if (lane == 0) {
@@ -343,11 +385,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <int A_BITS, int B_BITS>
+template <int A_BITS, int B_BITS, bool A_TMA>
 oq_status launch_pair(const PairParams& kp_in, void* stream) {
   PairParams kp = kp_in;
-  auto kern = gemm_pair_kernel<A_BITS, B_BITS>;
-  const size_t smem = 1024 + (size_t)OS * STAGE_BYTES + 512 + 8 * (2 * OS + 4) + 16;
+  auto kern = gemm_pair_kernel<A_BITS, B_BITS, A_TMA>;
+  const size_t smem = 1024 + (size_t)OS * STAGE_BYTES + EPI_BYTES + 512 + 8 * (2 * OS + 4) + 16;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
     set_error(std::string("cudaFuncSetAttribute(gemm pair): ") + cudaGetErrorString(e));
@@ -369,14 +411,73 @@ oq_status launch_pair(const PairParams& kp_in, void* stream) {
   return OQ_OK;
 }
 
-template <int A_BITS>
+template <int A_BITS, bool A_TMA>
 oq_status launch_pair_b(const PairParams& kp, int b_bits, void* stream) {
   switch (b_bits) {
-    case 2: return launch_pair<A_BITS, 2>(kp, stream);
-    case 3: return launch_pair<A_BITS, 3>(kp, stream);
-    case 4: return launch_pair<A_BITS, 4>(kp, stream);
+    case 2: return launch_pair<A_BITS, 2, A_TMA>(kp, stream);
+    case 3: return launch_pair<A_BITS, 3, A_TMA>(kp, stream);
+    case 4: return launch_pair<A_BITS, 4, A_TMA>(kp, stream);
     default: return OQ_ERR_UNSUPPORTED;
   }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn g_encode = nullptr;
+
+static oq_status encode_fn(EncodeTiledFn* out) {
+  if (!g_encode) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) {
+      set_error("cuTensorMapEncodeTiled is not available from the driver");
+      return OQ_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  *out = g_encode;
+  return OQ_OK;
+}
+
+oq_status encode_y_map(CUtensorMap* map, float* y, int64_t M, int N) {
+  EncodeTiledFn fn = nullptr;
+  const oq_status st = encode_fn(&fn);
+  if (st != OQ_OK) return st;
+  const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed for y (code " + std::to_string((int)r) + ")");
+    return OQ_ERR_CUDA;
+  }
+  return OQ_OK;
+}
+
+oq_status encode_a_map(CUtensorMap* map, const uint16_t* a16, int64_t M, int K) {
+  EncodeTiledFn fn = nullptr;
+  const oq_status st = encode_fn(&fn);
+  if (st != OQ_OK) return st;
+  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
+  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)RM};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(a16), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error("cuTensorMapEncodeTiled failed for the fp16 A operand (code " + std::to_string((int)r) + ")");
+    return OQ_ERR_CUDA;
+  }
+  return OQ_OK;
 }
 
 }  // namespace
@@ -401,11 +502,23 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream) {
   make_decode_tables(g.b_bits, g.b_levels_host, kp.b_tab);
   kp.a_lut8 = g.a_levels;
   kp.err = g.err;
+  if (reinterpret_cast<uintptr_t>(g.y) & 15) return OQ_ERR_UNSUPPORTED;
+  {
+    const oq_status st = encode_y_map(&kp.y_map, g.y, g.M, g.N);
+    if (st != OQ_OK) return st;
+  }
+  if (g.a_f16) {
+    // fp16 A operand fetched by TMA: 16-byte aligned rows of K halves
+    if ((reinterpret_cast<uintptr_t>(g.a_f16) & 15) || (g.K % 8)) return OQ_ERR_UNSUPPORTED;
+    const oq_status st = encode_a_map(&kp.a_map, g.a_f16, g.M, g.K);
+    if (st != OQ_OK) return st;
+    return launch_pair_b<4, true>(kp, g.b_bits, stream);
+  }
   switch (g.a_bits) {
-    case 2: return launch_pair_b<2>(kp, g.b_bits, stream);
-    case 3: return launch_pair_b<3>(kp, g.b_bits, stream);
-    case 4: return launch_pair_b<4>(kp, g.b_bits, stream);
-    case 8: return launch_pair_b<8>(kp, g.b_bits, stream);
+    case 2: return launch_pair_b<2, false>(kp, g.b_bits, stream);
+    case 3: return launch_pair_b<3, false>(kp, g.b_bits, stream);
+    case 4: return launch_pair_b<4, false>(kp, g.b_bits, stream);
+    case 8: return launch_pair_b<8, false>(kp, g.b_bits, stream);
     default: return OQ_ERR_UNSUPPORTED;
   }
 }

@@ -67,6 +67,7 @@ oq_status rq_launch(const RQArgs& a, void* stream);
 // codebook contraction launch (oq_gemm.cu)
 struct GemmArgs {
   const uint32_t* a_codes;   // [M, K*a_bits/32]
+  const uint16_t* a_f16;     // or: fp16 levels of A [M, K] (fused call), null otherwise
   const uint32_t* b_codes;   // [N, K*b_bits/32]
   const float* a_scale;      // [M] per-row magnitude s
   const float* b_scale;      // [N] per-row magnitude r
