@@ -79,6 +79,78 @@ __device__ __forceinline__ uint4 dec8(uint32_t w0, uint32_t w1, const uint16_t* 
   return make_uint4(pr(w0, 0), pr(w0, 2), pr(w1, 0), pr(w1, 2));
 }
 
+// ---- the same decoders with their shifts and multiplies done as integer
+// multiply-adds: the multipliers come from kernel parameters, so they stay
+// opaque to the compiler and the work lands on the FMA pipe instead of the
+// integer ALU pipe (where the byte permutes already queue).  x >> s is the high
+// word of x * 2^(32-s); x << s is x * 2^s.
+struct DecK {
+  uint32_t hi16;   // 2^16: x >> 16 as a high multiply
+  uint32_t hi29;   // 2^29: x >> 3
+  uint32_t seven;  // 7
+  uint32_t m256;   // 2^8
+  uint32_t m16;    // 2^4
+  uint32_t m4;     // 2^2
+  uint32_t m2;     // 2^1
+};
+
+__host__ __forceinline__ DecK make_deck() { return DecK{1u << 16, 1u << 29, 7u, 256u, 16u, 4u, 2u}; }
+
+__device__ __forceinline__ uint4 dec4k(uint32_t w, const uint32_t (&t)[4], const DecK& k) {
+  const uint32_t n = (__umulhi(w, k.hi29) & 0x11111111u) ^ 0x11111111u;  // 1 per negative code (bit 3 clear)
+  const uint32_t m = (w & 0x77777777u) ^ (n * k.seven);                   // magnitude index
+  const uint32_t mh = __umulhi(m, k.hi16), nh = __umulhi(n, k.hi16);
+  const uint32_t lo_a = __byte_perm(t[0], t[1], m), hi_a = __byte_perm(t[2], t[3], m) | __byte_perm(0x8000u, 0u, n);
+  const uint32_t lo_b = __byte_perm(t[0], t[1], mh), hi_b = __byte_perm(t[2], t[3], mh) | __byte_perm(0x8000u, 0u, nh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+// x: 16 bits (eight 2-bit codes) in the low half
+__device__ __forceinline__ uint4 dec2k(uint32_t x, const uint32_t (&t)[4], const DecK& k) {
+  uint32_t y = (x | (x * k.m256)) & 0x00FF00FFu;
+  y = (y | (y * k.m16)) & 0x0F0F0F0Fu;
+  y = (y | (y * k.m4)) & 0x33333333u;
+  const uint32_t yh = __umulhi(y, k.hi16);
+  const uint32_t lo_a = __byte_perm(t[0], t[0], y), hi_a = __byte_perm(t[1], t[1], y);
+  const uint32_t lo_b = __byte_perm(t[0], t[0], yh), hi_b = __byte_perm(t[1], t[1], yh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+// x: 24 bits (eight 3-bit codes) in the low three bytes
+__device__ __forceinline__ uint4 dec3k(uint32_t x, const uint32_t (&t)[4], const DecK& k) {
+  uint32_t y = (x & 0xFFFu) + (x & 0xFFF000u) * k.m16;
+  y = (y & 0x003F003Fu) + (y & 0x0FC00FC0u) * k.m4;
+  y = (y & 0x07070707u) + (y & 0x38383838u) * k.m2;
+  const uint32_t yh = __umulhi(y, k.hi16);
+  const uint32_t lo_a = __byte_perm(t[0], t[1], y), hi_a = __byte_perm(t[2], t[3], y);
+  const uint32_t lo_b = __byte_perm(t[0], t[1], yh), hi_b = __byte_perm(t[2], t[3], yh);
+  return make_uint4(__byte_perm(lo_a, hi_a, 0x5140), __byte_perm(lo_a, hi_a, 0x7362),
+                    __byte_perm(lo_b, hi_b, 0x5140), __byte_perm(lo_b, hi_b, 0x7362));
+}
+
+template <int BITS>
+__device__ __forceinline__ uint4 decode_chunk_k(const uint4& v, int j, const uint32_t (&t)[4], const uint16_t* lut8,
+                                                const DecK& k) {
+  if constexpr (BITS == 4) {
+    const uint32_t w = j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+    return dec4k(w, t, k);
+  } else if constexpr (BITS == 2) {
+    const uint32_t w = (j < 2) ? v.x : (j < 4 ? v.y : (j < 6 ? v.z : v.w));
+    return dec2k((j & 1) ? __umulhi(w, k.hi16) : (w & 0xFFFFu), t, k);
+  } else if constexpr (BITS == 3) {
+    uint32_t x;
+    if (j == 0) x = v.x & 0xFFFFFFu;
+    else if (j == 1) x = ((v.x >> 24) | (v.y << 8)) & 0xFFFFFFu;
+    else if (j == 2) x = ((v.y >> 16) | (v.z << 16)) & 0xFFFFFFu;
+    else x = v.z >> 8;
+    return dec3k(x, t, k);
+  } else {
+    return j == 0 ? dec8(v.x, v.y, lut8) : dec8(v.z, v.w, lut8);
+  }
+}
+
 // chunk j of a part -> 8 fp16
 template <int BITS>
 __device__ __forceinline__ uint4 decode_chunk(const uint4& v, int j, const uint32_t (&t)[4], const uint16_t* lut8) {

@@ -14,8 +14,10 @@
 // so the epilogue of one tile overlaps the next tile's main loop.
 //
 // Warps: 0-15 decode (codes prefetched two K blocks ahead into registers),
-// 16-19 epilogue, 20 allocates tensor memory and (even CTA) issues the MMAs
-// (odd CTA: forwards the decoders' arrivals to the even CTA).
+// 16-19 epilogue, 20 allocates tensor memory and (even CTA) issues the MMAs,
+// 20 and 21 of the odd CTA forward the decoders' arrivals to the even CTA
+// (alternate K blocks), and in the fused call 22 fetches the fp16 A tiles by
+// TMA.
 // Synchronisation: decoders of both CTAs arrive (one thread per warp, release
 // at cluster scope) on the even CTA's `full` barrier; the MMA completion is
 // multicast by tcgen05.commit to both CTAs' `empty` / `acc_full` barriers;
@@ -39,14 +41,15 @@ constexpr int RN = 128;            // weight rows per CTA
 constexpr int BK = DEC_BK, UMMA_K = 16;
 constexpr int NDEC = 512;          // decoder threads (warps 0-15)
 constexpr int EPI_WARP0 = 16;      // epilogue warps 16-19 (TMEM lane quarters 0-3)
-constexpr int MMA_WARP = 20;
-constexpr int NTHREADS = 21 * 32;
+constexpr int MMA_WARP = 20;       // and the first forwarder (odd CTA)
+constexpr int FWD2_WARP = 21;      // second forwarder (odd CTA)
+constexpr int NTHREADS = 22 * 32;
+constexpr int TMA_WARP = 22;       // fused call only: A-tile TMA producer
 constexpr int OS = 6;              // operand stages
 constexpr int A_TILE = RM * BK * 2;
 constexpr int B_TILE = RN * BK * 2;
 constexpr int STAGE_BYTES = A_TILE + B_TILE;
 constexpr uint32_t TMEM_COLS = 2 * PN;
-constexpr uint32_t FULL_LOCAL = NDEC / 32;           // one arrival per decoder warp
 constexpr uint32_t ACC_EMPTY_COUNT = 2 * 4;           // one per epilogue warp, both CTAs
 
 constexpr int EPI_BYTES = 4 * 2 * 32 * 32 * 4;   // per epilogue warp: two 32 x 32 fp32 staging boxes
@@ -65,24 +68,34 @@ struct PairParams {
   int n_tiles, nkb;
   int64_t tiles;
   uint32_t a_tab[4], b_tab[4];
+  DecK kc;                    // decode multipliers (opaque to the compiler)
   const uint16_t* a_lut8;
   int* err;
 };
 
 // A_TMA: the A operand is already fp16 levels in global memory (written by
-// the rotate-quantize kernel in the fused layer call); one thread per CTA
-// fetches each 128 x 64 A tile with a TMA load in the swizzled layout, and
-// the decoders expand only the weight codes.
+// the rotate-quantize kernel in the fused layer call); a producer warp of its
+// own fetches each 128 x 64 A tile with a TMA load in the swizzled layout as
+// soon as the MMA has released the stage, and the decoders expand only the
+// weight codes.
 template <int A_BITS, int B_BITS, bool A_TMA>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
+// registers: six warps of one SM sub-partition share its 16K registers
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
     gemm_pair_kernel(const __grid_constant__ PairParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  static_assert(OS == 6, "the decoder loop is unrolled over six stages");
   constexpr int QA = A_TMA ? 0 : Fmt<A_BITS>::QP, QB = Fmt<B_BITS>::QP;
-  constexpr uint32_t FULL_CTA = FULL_LOCAL + (A_TMA ? 1 : 0);   // + the TMA's expect_tx arrival
   constexpr int ITEMS_A = RM * QA, ITEMS = RM * QA + RN * QB;
-  constexpr int IPT = (ITEMS + NDEC - 1) / NDEC;
+  // when the items fill at most half of the decoder threads (weights only, in
+  // the fused call) the decoders split into two groups that take alternate K
+  // blocks, so each warp has two MMA periods per stage it fills
+  constexpr int NG = (2 * ITEMS <= NDEC) ? 2 : 1;
+  constexpr int GT = NDEC / NG;                      // threads per group
+  constexpr int IPT = (ITEMS + GT - 1) / GT;
+  constexpr int DEC_WARPS = NDEC / 32;
+  constexpr uint32_t FULL_CTA = GT / 32 + (A_TMA ? 1 : 0);   // + the TMA's expect_tx arrival
 
   unsigned char* epi = smem + OS * STAGE_BYTES;      // epilogue staging (1024-aligned)
   uint16_t* lut8 = reinterpret_cast<uint16_t*>(smem + OS * STAGE_BYTES + EPI_BYTES);
@@ -96,7 +109,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int nkb = p.nkb;
-  const int64_t my_tiles = (p.tiles > pair) ? (p.tiles - 1 - pair) / npairs + 1 : 0;
+  const int my_tiles = (p.tiles > pair) ? (int)((p.tiles - 1 - pair) / npairs + 1) : 0;
 
   if (A_BITS == 8 && p.a_lut8)
     for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = p.a_lut8[i];
@@ -121,8 +134,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t smem_base = smem_u32(smem);
+  const int total = my_tiles * nkb;   // K blocks this CTA pair runs through
 
-  if (warp < NDEC / 32) {
+  if (warp < DEC_WARPS) {
     // ------------------------------------------------ decoders
     uint32_t ta[4], tb[4];
 #pragma unroll
@@ -130,141 +144,177 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
       ta[i] = p.a_tab[i];
       tb[i] = p.b_tab[i];
     }
-    // fixed per-thread items: operand row r, 16-byte code part q; the row's
-    // byte offset inside a stage and its swizzle pattern do not change
-    uint32_t row_off[IPT], xs[IPT];
+    const DecK kc = p.kc;
+    // fixed per-thread items: operand row r, 16-byte code part q; the shared
+    // address of each of its 16-byte chunks in stage 0 does not change
+    constexpr int CPA = Fmt<A_BITS>::CPP, CPB = Fmt<B_BITS>::CPP;
+    constexpr int CPM = CPA > CPB ? CPA : CPB;
+    uint32_t sts[IPT][CPM];
     int item_r[IPT], item_q[IPT];
+    bool item_a[IPT], item_on[IPT];
+    const int group = (int)threadIdx.x / GT, gtid = (int)threadIdx.x % GT;
 #pragma unroll
     for (int it = 0; it < IPT; ++it) {
-      const int id = threadIdx.x + NDEC * it;
+      const int id = gtid + GT * it;
       const bool is_a = id < ITEMS_A;
       const int r = is_a ? id / (QA ? QA : 1) : (id - ITEMS_A) / QB;
+      item_a[it] = is_a;
+      item_on[it] = id < ITEMS;
       item_r[it] = r;
       item_q[it] = is_a ? id % (QA ? QA : 1) : (id - ITEMS_A) % QB;
-      row_off[it] = (is_a ? 0u : (uint32_t)A_TILE) + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
-      xs[it] = (uint32_t)(r & 7) << 4;
+      const uint32_t row_base = smem_base + (is_a ? 0u : (uint32_t)A_TILE) + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+      const int cpp = is_a ? CPA : CPB;
+#pragma unroll
+      for (int j = 0; j < CPM; ++j)
+        sts[it][j] = row_base + ((((uint32_t)(item_q[it] * cpp + j)) << 4) ^ ((uint32_t)(r & 7) << 4));
     }
-    // code-row pointers of the tile the fetch cursor is in (null: the row is
-    // outside the matrix; its decoded values only reach discarded outputs)
+    // code-row pointers of the tile the fetch cursor is in; activation rows
+    // past M read row M - 1 instead (they only reach outputs the store clips)
     const uint32_t* frow[IPT];
-    auto origin = [&](int64_t tile_i) {
-      const int64_t tt = pair + tile_i * npairs;
+    auto origin = [&](int tile_i) {
+      const int64_t tt = pair + (int64_t)tile_i * npairs;
       const int64_t m0 = (tt / p.n_tiles) * (2 * RM) + rank * RM;
       const int n0 = (int)(tt % p.n_tiles) * PN + (int)rank * RN;
 #pragma unroll
       for (int it = 0; it < IPT; ++it) {
-        const int id = threadIdx.x + NDEC * it;
-        frow[it] = nullptr;
-        if (id < ITEMS_A) {
+        if (item_a[it]) {
           const int64_t row = m0 + item_r[it];
-          if (row < p.M) frow[it] = p.a_codes + row * p.a_wpr;
-        } else if (id < ITEMS) {
-          const int row = n0 + item_r[it];
-          if (row < p.N) frow[it] = p.b_codes + (int64_t)row * p.b_wpr;
+          frow[it] = p.a_codes + (row < p.M ? row : p.M - 1) * p.a_wpr;
+        } else {
+          frow[it] = p.b_codes + (int64_t)(n0 + item_r[it]) * p.b_wpr;
         }
       }
     };
     auto fetch = [&](int kb, uint4 (&dst)[IPT]) {
 #pragma unroll
       for (int it = 0; it < IPT; ++it) {
-        const int id = threadIdx.x + NDEC * it;
         dst[it] = make_uint4(0u, 0u, 0u, 0u);
-        if (frow[it] != nullptr) {
-          if (id < ITEMS_A) dst[it] = load_part<A_BITS>(frow[it], kb, item_q[it], p.K);
+        if (item_on[it]) {
+          if (item_a[it]) dst[it] = load_part<A_BITS>(frow[it], kb, item_q[it], p.K);
           else dst[it] = load_part<B_BITS>(frow[it], kb, item_q[it], p.K);
         }
       }
     };
-    // decode one K block into stage `st`; `tail`: the block runs past K and
-    // the A chunks beyond it must be zero
-    auto decode = [&](const uint4 (&cur)[IPT], int st, bool tail, int kb) {
-      const uint32_t st_base = smem_base + (uint32_t)(st * STAGE_BYTES);
+    // decode one K block into stage S; TAIL: the block runs past K and the A
+    // chunks beyond it must be zero
+    // (called with literal S and TAIL: after inlining the stage offset folds
+    // into the store's address)
+    auto decode = [&](int S, bool TAIL, const uint4 (&cur)[IPT], int kb) {
+      const uint32_t so = (uint32_t)(S * STAGE_BYTES);
 #pragma unroll
       for (int it = 0; it < IPT; ++it) {
-        const int id = threadIdx.x + NDEC * it;
-        const uint32_t rb = st_base + row_off[it];
-        if (id < ITEMS_A) {
+        if (item_a[it]) {
 #pragma unroll
-          for (int j = 0; j < Fmt<A_BITS>::CPP; ++j) {
-            const int cj = item_q[it] * Fmt<A_BITS>::CPP + j;
-            uint4 o = decode_chunk<A_BITS>(cur[it], j, ta, lut8);
-            if (tail && kb * BK + cj * 8 >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
-            st_shared_v4(rb | (((uint32_t)cj << 4) ^ xs[it]), o);
+          for (int j = 0; j < CPA; ++j) {
+            uint4 o = decode_chunk_k<A_BITS>(cur[it], j, ta, lut8, kc);
+            if (TAIL && kb * BK + (item_q[it] * CPA + j) * 8 >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
+            st_shared_v4(sts[it][j] + so, o);
           }
-        } else if (id < ITEMS) {
+        } else if (item_on[it]) {
 #pragma unroll
-          for (int j = 0; j < Fmt<B_BITS>::CPP; ++j) {
-            const int cj = item_q[it] * Fmt<B_BITS>::CPP + j;
-            st_shared_v4(rb | (((uint32_t)cj << 4) ^ xs[it]), decode_chunk<B_BITS>(cur[it], j, tb, lut8));
-          }
+          for (int j = 0; j < CPB; ++j)
+            st_shared_v4(sts[it][j] + so, decode_chunk_k<B_BITS>(cur[it], j, tb, lut8, kc));
         }
       }
     };
-    const int64_t total = my_tiles * nkb;
-    // the fetch cursor runs two K blocks ahead of the decode cursor; the three
-    // register buffers rotate by unrolling (no copies of registers whose loads
-    // are still in flight)
-    int64_t f_tile = 0;
-    int f_kb = 0;
-    origin(0);
+    // the fetch cursor runs two steps (2 NG K blocks) ahead of the decode
+    // cursor; the three register buffers and the stages rotate by unrolling
+    // (no copies of registers whose loads are still in flight, and every stage
+    // offset is an immediate)
+    int f_tile = group / nkb, f_kb = group % nkb;   // this group's first K block
+    origin(f_tile);
     auto advance = [&]() {
-      if (++f_kb == nkb) {
-        f_kb = 0;
+      f_kb += NG;
+      while (f_kb >= nkb) {   // (nkb may be 1 with two groups)
+        f_kb -= nkb;
         ++f_tile;
         origin(f_tile);
       }
     };
     uint4 c0[IPT], c1[IPT], c2[IPT];
-    if (total > 0) {
+    if (group < total) {
       fetch(f_kb, c0);
       advance();
     }
-    if (total > 1) {
+    if (group + NG < total) {
       fetch(f_kb, c1);
       advance();
     }
-    int s = 0, d_kb = 0;
-    uint32_t n = 0;
-    int64_t g = 0, d_tile = 0;
-    auto a_row0 = [&](int64_t tile_i) {
-      return (int32_t)(((pair + tile_i * npairs) / p.n_tiles) * (2 * RM) + rank * RM);
-    };
-    int32_t d_m0 = a_row0(0);
-    auto step = [&](const uint4 (&cur)[IPT], uint4 (&fut)[IPT]) -> bool {
-      if (g + 2 < total) {
+    const bool k_tail = p.K % BK != 0;
+    int g = group, d_kb = group % nkb;
+    bool dead = false;
+    auto step = [&](int S, const uint4 (&cur)[IPT], uint4 (&fut)[IPT]) -> void {
+      if (g + 2 * NG < total) {
         fetch(f_kb, fut);
         advance();
       }
-      if (n > 0 && !mbar_wait(&op_empty[s], (n - 1) & 1u, p.err)) return false;
-      if (A_TMA && threadIdx.x == 0) {
-        // A tile of this K block: rows past M and columns past K arrive as zeros
-        mbar_arrive_expect_tx(&op_full[s], (uint32_t)A_TILE);
-        tma_load_2d(smem + s * STAGE_BYTES, &p.a_map, d_kb * BK, d_m0, &op_full[s]);
-      }
-      if ((d_kb + 1) * BK > p.K) decode(cur, s, true, d_kb);
-      else decode(cur, s, false, d_kb);
+      // after a timed-out wait (error recorded) keep stepping without waiting
+      const uint32_t n = (uint32_t)(g / OS);
+      if (n > 0 && !dead && !mbar_wait(&op_empty[S], (n - 1) & 1u, p.err)) dead = true;
+      if (k_tail && d_kb == nkb - 1) decode(S, true, cur, d_kb);
+      else decode(S, false, cur, d_kb);
       // this warp's tiles -> visible to the async proxy, then one arrival
       // per warp on this CTA's `full` barrier (the odd CTA forwards it)
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&op_full[s]);
-      if (++s == OS) {
-        s = 0;
-        ++n;
-      }
-      if (++d_kb == nkb) {
-        d_kb = 0;
-        ++d_tile;
-        d_m0 = a_row0(d_tile);
-      }
-      ++g;
-      return true;
+      if (lane == 0) mbar_arrive(&op_full[S]);
+      d_kb += NG;
+      while (d_kb >= nkb) d_kb -= nkb;
+      g += NG;
     };
-    while (g < total) {
-      if (!step(c0, c2) || g >= total) break;
-      if (!step(c1, c0) || g >= total) break;
-      if (!step(c2, c1)) break;
+    if constexpr (NG == 1) {
+      while (g < total) {
+        step(0, c0, c2);
+        if (g >= total) break;
+        step(1, c1, c0);
+        if (g >= total) break;
+        step(2, c2, c1);
+        if (g >= total) break;
+        step(3, c0, c2);
+        if (g >= total) break;
+        step(4, c1, c0);
+        if (g >= total) break;
+        step(5, c2, c1);
+      }
+    } else {
+      // group 0 fills stages 0, 2, 4 and group 1 stages 1, 3, 5
+      auto run = [&](int s0) {
+        while (g < total) {
+          step(s0, c0, c2);
+          if (g >= total) break;
+          step(s0 + 2, c1, c0);
+          if (g >= total) break;
+          step(s0 + 4, c2, c1);
+        }
+      };
+      if (group == 0) run(0);
+      else run(1);
     }
+  } else if (A_TMA && warp == TMA_WARP) {
+    // ------------------------------------------------ A tiles by TMA (fused call)
+    if (lane == 0) {
+      int s = 0, kb = 0, tile = 0;
+      uint32_t n = 0;
+      auto a_row0 = [&](int tile_i) {
+        return (int32_t)(((pair + (int64_t)tile_i * npairs) / p.n_tiles) * (2 * RM) + rank * RM);
+      };
+      int32_t m0 = a_row0(0);
+      for (int g = 0; g < total; ++g) {
+        if (n > 0 && !mbar_wait(&op_empty[s], (n - 1) & 1u, p.err)) break;
+        // rows past M and columns past K arrive as zeros
+        mbar_arrive_expect_tx(&op_full[s], (uint32_t)A_TILE);
+        tma_load_2d(smem + s * STAGE_BYTES, &p.a_map, kb * BK, m0, &op_full[s]);
+        if (++s == OS) {
+          s = 0;
+          ++n;
+        }
+        if (++kb == nkb) {
+          kb = 0;
+          m0 = a_row0(++tile);
+        }
+      }
+    }
+    __syncwarp();
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
     // ------------------------------------------------ epilogue (both CTAs)
     // Each warp drains its 32 TMEM lanes (rows) in chunks of 32 columns,
@@ -286,9 +336,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 #pragma unroll 1
       for (int cc = 0; cc < PN / 32; ++cc) {
         const int nb = n0 + cc * 32;
-        float4 rr[8];
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) rr[k4] = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + k4);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * PN + cc * 32), v);
         tmem_wait_ld();
@@ -299,11 +346,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         const uint32_t rb = smem_u32(buf) + (uint32_t)lane * 128u;
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
+          const float4 rr = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + k4);
           uint4 o;
-          o.x = __float_as_uint(__uint_as_float(v[4 * k4 + 0]) * srow * rr[k4].x);
-          o.y = __float_as_uint(__uint_as_float(v[4 * k4 + 1]) * srow * rr[k4].y);
-          o.z = __float_as_uint(__uint_as_float(v[4 * k4 + 2]) * srow * rr[k4].z);
-          o.w = __float_as_uint(__uint_as_float(v[4 * k4 + 3]) * srow * rr[k4].w);
+          o.x = __float_as_uint(__uint_as_float(v[4 * k4 + 0]) * srow * rr.x);
+          o.y = __float_as_uint(__uint_as_float(v[4 * k4 + 1]) * srow * rr.y);
+          o.z = __float_as_uint(__uint_as_float(v[4 * k4 + 2]) * srow * rr.z);
+          o.w = __float_as_uint(__uint_as_float(v[4 * k4 + 3]) * srow * rr.w);
           st_shared_v4(rb + ((uint32_t)(k4 ^ (lane & 7)) << 4), o);
         }
         fence_proxy_async_smem();
@@ -356,20 +404,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     __syncwarp();
   }
 
-  if (warp == MMA_WARP && rank == 1) {
-    // ------------------------------------------------ forwarder (odd CTA)
-    // one cluster-scope release per stage instead of one per decoder warp
+  if ((warp == MMA_WARP || warp == FWD2_WARP) && rank == 1) {
+    // ------------------------------------------------ forwarders (odd CTA)
+    // one cluster-scope release per stage instead of one per decoder warp; a
+    // release at cluster scope takes longer than the MMAs of one K block, so
+    // two threads take alternate K blocks (even and odd stages)
     if (lane == 0) {
-      const int64_t total = my_tiles * nkb;
-      int s = 0;
-      uint32_t n = 0;
-      for (int64_t g = 0; g < total; ++g) {
-        if (!mbar_wait(&op_full[s], n & 1u, p.err)) break;
+      for (int g = (warp == MMA_WARP) ? 0 : 1; g < total; g += 2) {
+        const int s = g % OS;
+        if (!mbar_wait(&op_full[s], (uint32_t)(g / OS) & 1u, p.err)) break;
         mbar_arrive_cluster(mapa_shared(smem_u32(&op_full[s]), 0));
-        if (++s == OS) {
-          s = 0;
-          ++n;
-        }
       }
     }
     __syncwarp();
@@ -402,7 +446,9 @@ oq_status launch_pair(const PairParams& kp_in, void* stream) {
   kp.nkb = (kp.K + BK - 1) / BK;
   kp.tiles = ((kp.M + 2 * RM - 1) / (2 * RM)) * (int64_t)kp.n_tiles;
   const int64_t grid = std::min<int64_t>(2 * kp.tiles, (int64_t)(sms & ~1));
-  kern<<<(unsigned)grid, NTHREADS, smem, static_cast<cudaStream_t>(stream)>>>(kp);
+  // K-block counters are 32-bit
+  if (((kp.tiles + grid / 2 - 1) / (grid / 2)) * (int64_t)kp.nkb >= (int64_t)1 << 31) return OQ_ERR_UNSUPPORTED;
+  kern<<<(unsigned)grid, A_TMA ? NTHREADS + 32 : NTHREADS, smem, static_cast<cudaStream_t>(stream)>>>(kp);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("gemm pair launch: ") + cudaGetErrorString(e));
@@ -500,6 +546,7 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream) {
   kp.b_wpr = g.K * g.b_bits / 32;
   make_decode_tables(g.a_bits, g.a_levels_host, kp.a_tab);
   make_decode_tables(g.b_bits, g.b_levels_host, kp.b_tab);
+  kp.kc = make_deck();
   kp.a_lut8 = g.a_levels;
   kp.err = g.err;
   if (reinterpret_cast<uintptr_t>(g.y) & 15) return OQ_ERR_UNSUPPORTED;
