@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--workload", default="dit_image")
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's token count (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--route", choices=["levels", "codes"], default="levels",
+                    help="hot-path route of the timed step (the other one is reported beside it)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -209,45 +211,68 @@ def run_ours(args):
     flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        B.oq_rotate_quantize(layer, x, codes, s)
-        B.oq_linear(layer, codes, s, Wc, r, y)
+    a16 = torch.empty((T, d), dtype=torch.float16, device=dev)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize()
-    B.oq_poll_error(layer)
+    # the two routes of the hot path (both give the same y):
+    #   levels: oq_rotate_quantize_levels -> oq_linear_levels, the two stages of
+    #           oq_linear_fused (activation codes leave K1 as fp16 levels that
+    #           the contraction reads by TMA; only weight codes are decoded)
+    #   codes:  oq_rotate_quantize -> oq_linear (packed codes between them)
+    def stage1(route):
+        if route == "levels":
+            B.oq_rotate_quantize_levels(layer, x, a16, s)
+        else:
+            B.oq_rotate_quantize(layer, x, codes, s)
+
+    def stage2(route):
+        if route == "levels":
+            B.oq_linear_levels(layer, a16, s, Wc, r, y)
+        else:
+            B.oq_linear(layer, codes, s, Wc, r, y)
+
+    def timed(route, K, warmup, sample_clocks=False):
+        for _ in range(warmup):
+            flush.zero_()
+            stage1(route)
+            stage2(route)
+        torch.cuda.synchronize()
+        B.oq_poll_error(layer)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) \
+            if (rank == 0 and sample_clocks) else None
+        if clocks:
+            clocks.start()
+            time.sleep(0.3)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        for i in range(K):
+            flush.zero_()                              # L2 flushed, outside the events
+            ev[i][0].record(stream)
+            stage1(route)
+            ev[i][1].record(stream)
+            stage2(route)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        wall = time.perf_counter() - wall0
+        clk = clocks.stop() if clocks else None
+        t1 = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+        t2 = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+        B.oq_poll_error(layer)
+        return t1, t2, wall, clk
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    for i in range(K):
-        flush.zero_()                                  # L2 flushed, outside the events
-        ev[i][0].record(stream)
-        B.oq_rotate_quantize(layer, x, codes, s)
-        ev[i][1].record(stream)
-        B.oq_linear(layer, codes, s, Wc, r, y)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    wall = time.perf_counter() - wall0
-    clk = clocks.stop() if clocks else None
-    t_rq = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    t_mm = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    t_step = [a + b for a, b in zip(t_rq, t_mm)]
-    total_ms = max_over_ranks(sum(t_step), dev)
-    B.oq_poll_error(layer)
+    route = args.route
+    other = "codes" if route == "levels" else "levels"
+    t_rq, t_mm, wall, clk = timed(route, K, args.warmup, sample_clocks=True)
+    total_ms = max_over_ranks(sum(a + b for a, b in zip(t_rq, t_mm)), dev)
+    o_rq, o_mm, _, _ = timed(other, K, max(3, args.warmup // 2))
+    other_ms = max_over_ranks(sum(a + b for a, b in zip(o_rq, o_mm)), dev)
 
-    # fused call, same workload (one C call, both kernels)
+    # the fused call, same workload (one C call, both kernels)
     for _ in range(2):
         B.oq_linear_fused(layer, x, Wc, r, y, ws)
     evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
@@ -283,11 +308,29 @@ def run_ours(args):
 
     peaks = load_peaks()
     flops = 2.0 * T * d * dout
+
+    def rq_bytes_per_launch(rt):
+        # bf16 x read + A operand written (fp16 levels, or packed codes) + norms
+        return T * (2 * d + (2 * d if rt == "levels" else d * lay.a_bits / 8) + 4)
+
     mm_ms = statistics.mean(t_mm)
     rq_ms = statistics.mean(t_rq)
-    rq_bytes = T * (2 * d + d * lay.a_bits / 8 + 4)
+    rq_bytes = rq_bytes_per_launch(route)
     gemm_tf = flops / (mm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
+    kernels = {
+        "levels": ("codebook GEMM, fp16 A operand by TMA, weight codes decoded to fp16 in shared memory "
+                   "(tcgen05 CTA pair, fp32 TMEM accumulate)",
+                   "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes) writing the codes' fp16 levels"),
+        "codes": ("codebook GEMM, both operands' codes decoded to fp16 in shared memory "
+                  "(tcgen05 CTA pair, fp32 TMEM accumulate)",
+                  "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes, pack)"),
+    }
+    steps_desc = {
+        "levels": "oq_rotate_quantize_levels + oq_linear_levels (the two stages of oq_linear_fused; "
+                  "weights prepared once, offline)",
+        "codes": "oq_rotate_quantize + oq_linear (weights prepared once, offline)",
+    }
     out = {
         "metric": METRIC,
         "value": whole_job_rate(world, T, K, total_ms),
@@ -307,24 +350,30 @@ def run_ours(args):
             "h": d & -d, "x_dtype": "bf16", "y_dtype": "fp32",
             "parallelism": f"token-sharded x{world}, weights replicated",
             "l2": "flushed (256 MiB write) before every step, outside the timed events",
-            "step": "oq_rotate_quantize + oq_linear (weights prepared once, offline)",
+            "step": steps_desc[route],
         },
         "roofline": {
-            "kernel": "codebook GEMM (tcgen05, decode to fp16, fp32 TMEM accumulate)",
+            "kernel": kernels[route][0],
             "bound": "tensor", "achieved": gemm_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": gemm_tf / peaks["bf16_tflops"], "traffic": None,
             "peak_source": f"{peaks['source']} bf16 dense burst (fp16 has the same tensor rate)",
             "flops_per_launch": flops, "ms_per_launch": mm_ms,
         },
         "roofline_rotate_quantize": {
-            "kernel": "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes, pack)",
+            "kernel": kernels[route][1],
             "bound": "hbm", "achieved": rq_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": rq_gbs / peaks["hbm_gbs"], "traffic": None,
             "peak_source": f"{peaks['source']} HBM copy bandwidth",
             "bytes_per_launch": rq_bytes, "ms_per_launch": rq_ms,
         },
         "fused": {"value": T / (statistics.mean(t_fused) * 1e-3), "unit": UNIT,
-                  "ms_per_call": statistics.mean(t_fused)},
+                  "ms_per_call": statistics.mean(t_fused), "call": "oq_linear_fused"},
+        "other_route": {"route": other, "step": steps_desc[other],
+                        "value": whole_job_rate(world, T, K, other_ms), "unit": UNIT, "ms_per_step": other_ms / K,
+                        "gemm_tflops": flops / (statistics.mean(o_mm) * 1e-3) / 1e12,
+                        "gemm_ms": statistics.mean(o_mm),
+                        "rq_gbs": rq_bytes_per_launch(other) / (statistics.mean(o_rq) * 1e-3) / 1e9,
+                        "rq_ms": statistics.mean(o_rq)},
         "e2e": {"value": whole_job_rate(world, T, K, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()),

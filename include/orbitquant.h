@@ -194,6 +194,34 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The two stages of oq_linear_fused's fp16 route, as separate calls (for
+ * callers that schedule or time them separately; pith Figure 2 and gecl notes
+ * Method 2: the codes' levels are what the contraction multiplies):
+ *
+ * oq_rotate_quantize_levels -- oq_rotate_quantize, but instead of packed
+ * codes it writes each coordinate's codebook level as the fp16 A operand of
+ * the contraction:
+ *   a16[t, i] = fp16(a_scale * C_a[code_{t,i}])   (a_scale from
+ *               oq_layer_get_info: the per-codebook factor that makes the
+ *               levels close to exact in fp16)
+ *   x    device [T, d_in] bf16 (OQ_DTYPE_BF16 only, else OQ_ERR_UNSUPPORTED).
+ *   a16  device [T, d_in] uint16 (fp16 bits), 16-byte aligned.
+ *   s    device [T] fp32 token norms.
+ *
+ * oq_linear_levels -- oq_linear with the A operand given as those fp16
+ * levels (read by TMA; only the weight codes are decoded):
+ *   y[t, o] = s[t] r[o] / (a_scale w_scale) sum_i a16[t, i] fp16(w_scale C_w[Wcodes[o, i]])
+ *   Needs d_out % 256 == 0 (else OQ_ERR_UNSUPPORTED); y 16-byte aligned.
+ *
+ * oq_rotate_quantize_levels followed by oq_linear_levels gives exactly the y
+ * of oq_linear_fused (and of oq_rotate_quantize + oq_linear).
+ */
+oq_status oq_rotate_quantize_levels(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
+                                    uint16_t* a16, float* s, void* stream);
+oq_status oq_linear_levels(const oq_layer* layer, const uint16_t* a16, const float* s, int64_t T,
+                           const uint32_t* Wcodes, const float* r, float* y, void* stream);
+
+/*
  * oq_linear_fused_static -- the same computation as oq_linear_fused for
  * callers that cannot allocate device memory: code running inside a CUDA
  * graph capture, runtimes that give plug-ins no allocator, loops where an

@@ -26,7 +26,8 @@ OQ_FLAG_GAUSSIAN_MARGINAL = 2
 EXPORTS = (
     "oq_codebook_build", "oq_rotation_build", "oq_layer_create", "oq_layer_destroy", "oq_layer_get_info", "oq_layer_get_perm",
     "oq_rotate_quantize", "oq_weight_prepare", "oq_linear", "oq_linear_fused_workspace_size",
-    "oq_linear_fused", "oq_linear_fused_static", "oq_poll_error", "oq_last_error", "oq_status_string",
+    "oq_linear_fused", "oq_rotate_quantize_levels", "oq_linear_levels", "oq_linear_fused_static",
+    "oq_poll_error", "oq_last_error", "oq_status_string",
 )
 
 
@@ -79,6 +80,8 @@ def load_library(path: str = LIB_PATH):
         "oq_linear": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_linear_fused_workspace_size": (sz, [vp, i64]),
         "oq_linear_fused": (i32, [vp, vp, i32, i64, vp, vp, vp, vp, sz, vp]),
+        "oq_rotate_quantize_levels": (i32, [vp, vp, i32, i64, vp, vp, vp]),
+        "oq_linear_levels": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
         "oq_poll_error": (i32, [vp]),
         "oq_last_error": (ctypes.c_char_p, []),
@@ -243,6 +246,32 @@ def oq_linear_fused(layer: Layer, x, Wcodes, r, y=None, workspace=None):
                                           _dev(r, "r"), _dev(y, "y"), _dev(workspace, "workspace"),
                                           workspace.numel() * workspace.element_size(), _stream(x)),
            "oq_linear_fused")
+    return y
+
+
+def oq_rotate_quantize_levels(layer: Layer, x, a16=None, s=None):
+    """x [T, d_in] bf16 (CUDA) -> (a16 [T, d_in] fp16 levels of the codes, s [T] fp32):
+    the first stage of the fused call's fp16 route."""
+    torch = _torch()
+    T = x.shape[0]
+    if a16 is None:
+        a16 = torch.empty((T, layer.d_in), dtype=torch.float16, device=x.device)
+    if s is None:
+        s = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _check(load_library().oq_rotate_quantize_levels(layer.handle, _dev(x, "x"), _dtype_code(x), T, _dev(a16, "a16"),
+                                                    _dev(s, "s"), _stream(x)), "oq_rotate_quantize_levels")
+    return a16, s
+
+
+def oq_linear_levels(layer: Layer, a16, s, Wcodes, r, y=None):
+    """(a16 fp16 levels, s, Wcodes, r) -> y [T, d_out] fp32: the second stage of
+    the fused call's fp16 route."""
+    torch = _torch()
+    T = a16.shape[0]
+    if y is None:
+        y = torch.empty((T, layer.d_out), dtype=torch.float32, device=a16.device)
+    _check(load_library().oq_linear_levels(layer.handle, _dev(a16, "a16"), _dev(s, "s"), T, _dev(Wcodes, "Wcodes"),
+                                           _dev(r, "r"), _dev(y, "y"), _stream(a16)), "oq_linear_levels")
     return y
 
 

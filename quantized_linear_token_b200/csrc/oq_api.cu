@@ -295,6 +295,52 @@ size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
   return ((a + 255) & ~(size_t)255) + (size_t)T * 4;
 }
 
+static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint16_t* a16, float* s,
+                           void* stream) {
+  RQArgs a{};
+  a.src = x;
+  a.src_dtype = x_dtype;
+  a.rows = T;
+  a.d = L->d_in;
+  a.h = L->h;
+  a.log_h = L->log_h;
+  a.bits = L->a_bits;
+  a.gather = L->d_gather_a;
+  a.signmask = L->d_signmask;
+  a.thr = L->thr_a;
+  a.out16 = a16;
+  make_decode_tables(L->a_bits, L->lv_a, a.dtab);
+  a.lut8 = L->d_levels_a;
+  a.norms = s;
+  a.err = L->d_error;
+  return rq_launch(a, stream);
+}
+
+oq_status oq_rotate_quantize_levels(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint16_t* a16,
+                                    float* s, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize_levels: layer is null");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize_levels: T < 0");
+  if (T == 0) return OQ_OK;
+  oq_status st = check_rows_input(x, x_dtype, "oq_rotate_quantize_levels");
+  if (st != OQ_OK) return st;
+  if (x_dtype != OQ_DTYPE_BF16) return fail(OQ_ERR_UNSUPPORTED, "oq_rotate_quantize_levels: bf16 input only");
+  if (!a16 || !s || !aligned(a16, 16) || !aligned(s, 4))
+    return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize_levels: a16 (16-byte) / s (4-byte) pointers invalid");
+  return rq_levels(L, x, x_dtype, T, a16, s, stream);
+}
+
+oq_status oq_linear_levels(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint32_t* Wcodes,
+                           const float* r, float* y, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: layer is null");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: T < 0");
+  if (T == 0) return OQ_OK;
+  if (!a16 || !s || !Wcodes || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: null pointer");
+  if (!aligned(a16, 16) || !aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(s, 4) || !aligned(r, 16))
+    return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: misaligned pointer");
+  if (L->d_out % 256 != 0) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_levels: needs d_out % 256 == 0");
+  return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
+}
+
 oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
                           const float* r, float* y, void* workspace, size_t workspace_bytes, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: layer is null");
@@ -311,23 +357,7 @@ oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int
   if (fused_f16_route(L, x_dtype)) {
     uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
     float* s = reinterpret_cast<float*>(ws + ((fused_f16_bytes(L, T) + 255) & ~(size_t)255));
-    RQArgs a{};
-    a.src = x;
-    a.src_dtype = x_dtype;
-    a.rows = T;
-    a.d = L->d_in;
-    a.h = L->h;
-    a.log_h = L->log_h;
-    a.bits = L->a_bits;
-    a.gather = L->d_gather_a;
-    a.signmask = L->d_signmask;
-    a.thr = L->thr_a;
-    a.out16 = a16;
-    make_decode_tables(L->a_bits, L->lv_a, a.dtab);
-    a.lut8 = L->d_levels_a;
-    a.norms = s;
-    a.err = L->d_error;
-    st = rq_launch(a, stream);
+    st = rq_levels(L, x, x_dtype, T, a16, s, stream);
     if (st != OQ_OK) return st;
     return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
   }

@@ -64,7 +64,25 @@ def _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, flags=0, seed=0, w_ro
     lin = check_linear(y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, label + " y", rows=y_rows)
     # the fused call computes the same codes, so the same y
     np.testing.assert_array_equal(yf_np, y_np)
+    if x_np.dtype == np.uint16 and d_out % 256 == 0:
+        _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in)
     return st, lin
+
+
+def _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in):
+    """The fused call's fp16 route as two calls: the A operand holds exactly the
+    fp16 value of a_scale times the level of each code, the norms are the
+    same, and the contraction gives the same y."""
+    torch, B = env
+    a16, s2 = B.oq_rotate_quantize_levels(layer, x_t)
+    y2 = B.oq_linear_levels(layer, a16, s2, Wc, r)
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+    np.testing.assert_array_equal(s2.cpu().numpy(), s_np)
+    c = O.unpack_codes(codes_np, a_bits, d_in)
+    want = (layer.a_scale * np.asarray(cb_a.levels, dtype=np.float64))[c].astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(a16.cpu().numpy().view(np.uint16), want)
+    np.testing.assert_array_equal(y2.cpu().numpy(), y_np)
 
 
 CASES = [
