@@ -61,6 +61,27 @@ def load_peaks():
             "bf16_tflops_sustained": None, "source": "fallback"}
 
 
+def measured_traffic(key: str):
+    """Per-launch DRAM bytes (read + write) of a kernel from the ncu capture
+    recorded in profiles/traffic.json, or None when there is none or the
+    kernel's sources changed since it was taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)["kernels"].get(key)
+    if rec is None:
+        return None
+    m = hashlib.sha256()
+    for name in rec["sources"]:
+        with open(os.path.join(ROOT, "quantized_linear_token_b200", "csrc", name), "rb") as f:
+            m.update(f.read())
+    if m.hexdigest() != rec["sources_sha256"]:
+        return None
+    return rec["dram_read_bytes"] + rec["dram_write_bytes"]
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
@@ -355,15 +376,19 @@ def run_ours(args):
         "roofline": {
             "kernel": kernels[route][0],
             "bound": "tensor", "achieved": gemm_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-            "frac": gemm_tf / peaks["bf16_tflops"], "traffic": None,
+            "frac": gemm_tf / peaks["bf16_tflops"],
+            "traffic": measured_traffic("gemm_levels") if (route == "levels" and T == wl.tokens) else None,
             "peak_source": f"{peaks['source']} bf16 dense burst (fp16 has the same tensor rate)",
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, profiles/traffic.json",
             "flops_per_launch": flops, "ms_per_launch": mm_ms,
         },
         "roofline_rotate_quantize": {
             "kernel": kernels[route][1],
             "bound": "hbm", "achieved": rq_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": rq_gbs / peaks["hbm_gbs"], "traffic": None,
+            "frac": rq_gbs / peaks["hbm_gbs"],
+            "traffic": measured_traffic("rq_levels") if (route == "levels" and T == wl.tokens) else None,
             "peak_source": f"{peaks['source']} HBM copy bandwidth",
+            "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, profiles/traffic.json",
             "bytes_per_launch": rq_bytes, "ms_per_launch": rq_ms,
         },
         "fused": {"value": T / (statistics.mean(t_fused) * 1e-3), "unit": UNIT,
