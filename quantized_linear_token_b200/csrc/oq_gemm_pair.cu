@@ -195,11 +195,41 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
         }
       }
     };
-    // decode one K block into stage S; TAIL: the block runs past K and the A
-    // chunks beyond it must be zero
+    // decode one K block (TAIL: the block runs past K and the A chunks beyond
+    // it must be zero) into registers, and store decoded chunks into stage S
     // (called with literal S and TAIL: after inlining the stage offset folds
     // into the store's address)
-    auto decode = [&](int S, bool TAIL, const uint4 (&cur)[IPT], int kb) {
+    auto decode_regs = [&](bool TAIL, const uint4 (&cur)[IPT], int kb, uint4 (&dec)[IPT][CPM]) {
+#pragma unroll
+      for (int it = 0; it < IPT; ++it) {
+        if (item_a[it]) {
+#pragma unroll
+          for (int j = 0; j < CPA; ++j) {
+            uint4 o = decode_chunk_k<A_BITS>(cur[it], j, ta, lut8, kc);
+            if (TAIL && kb * BK + (item_q[it] * CPA + j) * 8 >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
+            dec[it][j] = o;
+          }
+        } else if (item_on[it]) {
+#pragma unroll
+          for (int j = 0; j < CPB; ++j) dec[it][j] = decode_chunk_k<B_BITS>(cur[it], j, tb, lut8, kc);
+        }
+      }
+    };
+    auto store = [&](int S, const uint4 (&dec)[IPT][CPM]) {
+      const uint32_t so = (uint32_t)(S * STAGE_BYTES);
+#pragma unroll
+      for (int it = 0; it < IPT; ++it) {
+        if (item_a[it]) {
+#pragma unroll
+          for (int j = 0; j < CPA; ++j) st_shared_v4(sts[it][j] + so, dec[it][j]);
+        } else if (item_on[it]) {
+#pragma unroll
+          for (int j = 0; j < CPB; ++j) st_shared_v4(sts[it][j] + so, dec[it][j]);
+        }
+      }
+    };
+    // decode and store chunk by chunk (few registers live)
+    auto decode_store = [&](int S, bool TAIL, const uint4 (&cur)[IPT], int kb) {
       const uint32_t so = (uint32_t)(S * STAGE_BYTES);
 #pragma unroll
       for (int it = 0; it < IPT; ++it) {
@@ -217,6 +247,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
         }
       }
     };
+    // with at most four decoded chunks per thread the decode runs before the
+    // wait for the stage to be free (off the MMA's critical path); larger
+    // per-thread loads decode after it (registers)
+    constexpr bool AHEAD = IPT * CPM <= 4;
     // the fetch cursor runs two steps (2 NG K blocks) ahead of the decode
     // cursor; the three register buffers and the stages rotate by unrolling
     // (no copies of registers whose loads are still in flight, and every stage
@@ -248,11 +282,20 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
         fetch(f_kb, fut);
         advance();
       }
-      // after a timed-out wait (error recorded) keep stepping without waiting
+      const bool tail = k_tail && d_kb == nkb - 1;
       const uint32_t n = (uint32_t)(g / OS);
-      if (n > 0 && !dead && !mbar_wait(&op_empty[S], (n - 1) & 1u, p.err)) dead = true;
-      if (k_tail && d_kb == nkb - 1) decode(S, true, cur, d_kb);
-      else decode(S, false, cur, d_kb);
+      // after a timed-out wait (error recorded) keep stepping without waiting
+      if constexpr (AHEAD) {
+        uint4 dec[IPT][CPM];
+        if (tail) decode_regs(true, cur, d_kb, dec);
+        else decode_regs(false, cur, d_kb, dec);
+        if (n > 0 && !dead && !mbar_wait(&op_empty[S], (n - 1) & 1u, p.err)) dead = true;
+        store(S, dec);
+      } else {
+        if (n > 0 && !dead && !mbar_wait(&op_empty[S], (n - 1) & 1u, p.err)) dead = true;
+        if (tail) decode_store(S, true, cur, d_kb);
+        else decode_store(S, false, cur, d_kb);
+      }
       // this warp's tiles -> visible to the async proxy, then one arrival
       // per warp on this CTA's `full` barrier (the odd CTA forwards it)
       fence_proxy_async_smem();
