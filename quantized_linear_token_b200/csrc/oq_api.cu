@@ -30,13 +30,6 @@ static oq_status cuda_check(cudaError_t e, const char* what) {
               std::string(what) + ": " + cudaGetErrorString(e));
 }
 
-static void scaled_thresholds(const oq_codebook& cb, int h, float* thr) {
-  const int n = 1 << (cb.bits - 1);
-  const double sh = std::sqrt((double)h);
-  for (int k = 0; k < 128; ++k) thr[k] = INFINITY;
-  // positive thresholds tau_1..tau_{n-1} = thresholds[n .. 2n-2]
-  for (int k = 1; k < n; ++k) thr[k - 1] = (float)(sh * cb.thresholds[n - 1 + k]);
-}
 
 }  // namespace oq
 
@@ -96,6 +89,10 @@ void oq_layer_destroy(oq_layer* L) {
   cudaFree(L->d_signmask);
   cudaFree(L->d_levels_a);
   cudaFree(L->d_levels_w);
+  cudaFree(L->bins_a.d_codes);
+  cudaFree(L->bins_a.d_levels);
+  cudaFree(L->bins_w.d_codes);
+  cudaFree(L->bins_w.d_levels);
   cudaFree(L->d_error);
   delete L;
 }
@@ -140,8 +137,14 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   for (int i = 0; i < (1 << w_bits); ++i) lv_w[i] = f64_to_f16_bits(L->w_scale * L->cb_w.levels[i]);
   std::memcpy(L->lv_a, lv_a, sizeof(lv_a));
   std::memcpy(L->lv_w, lv_w, sizeof(lv_w));
-  scaled_thresholds(L->cb_a, L->h, L->thr_a);
-  scaled_thresholds(L->cb_w, L->h, L->thr_w);
+  std::vector<uint32_t> ta_codes, ta_levels, tw_codes, tw_levels;
+  if ((st = build_bin_table(L->cb_a, d_in, L->h, lv_a, &L->bins_a.kscale, &L->bins_a.b0, &L->bins_a.nb, ta_codes,
+                            ta_levels)) != OQ_OK ||
+      (st = build_bin_table(L->cb_w, d_in, L->h, lv_w, &L->bins_w.kscale, &L->bins_w.b0, &L->bins_w.nb, tw_codes,
+                            tw_levels)) != OQ_OK) {
+    delete L;
+    return st;
+  }
 
   st = cuda_check(cudaMalloc(&L->d_gather_a, gather.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
   if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_gather_a, gather.data(), gather.size() * sizeof(uint16_t),
@@ -155,6 +158,15 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_levels_a, lv_a, sizeof(lv_a), cudaMemcpyHostToDevice), "upload levels");
   if (st == OQ_OK) st = cuda_check(cudaMalloc(&L->d_levels_w, sizeof(lv_w)), "cudaMalloc(levels)");
   if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_levels_w, lv_w, sizeof(lv_w), cudaMemcpyHostToDevice), "upload levels");
+  auto upload = [&](uint32_t** dst, const std::vector<uint32_t>& v) {
+    if (st == OQ_OK) st = cuda_check(cudaMalloc(dst, v.size() * 4), "cudaMalloc(threshold table)");
+    if (st == OQ_OK)
+      st = cuda_check(cudaMemcpy(*dst, v.data(), v.size() * 4, cudaMemcpyHostToDevice), "upload threshold table");
+  };
+  upload(&L->bins_a.d_codes, ta_codes);
+  upload(&L->bins_a.d_levels, ta_levels);
+  upload(&L->bins_w.d_codes, tw_codes);
+  upload(&L->bins_w.d_levels, tw_levels);
   if (st == OQ_OK) st = cuda_check(cudaMalloc(&L->d_error, sizeof(int)), "cudaMalloc(error word)");
   if (st == OQ_OK) st = cuda_check(cudaMemset(L->d_error, 0, sizeof(int)), "clear error word");
   if (st != OQ_OK) {
@@ -197,8 +209,8 @@ static oq_status check_rows_input(const void* x, int32_t dtype, const char* who)
   return OQ_OK;
 }
 
-static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t rows, int bits, const float* thr,
-                    uint32_t* codes, float* norms, void* stream) {
+static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t rows, int bits,
+                    const oq_bin_table& bins, uint32_t* codes, float* norms, void* stream) {
   RQArgs a{};
   a.src = x;
   a.src_dtype = dtype;
@@ -209,7 +221,10 @@ static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t row
   a.bits = bits;
   a.gather = L->d_gather_a;
   a.signmask = L->d_signmask;
-  a.thr = thr;
+  a.bins = bins.d_codes;
+  a.nb = bins.nb;
+  a.b0 = bins.b0;
+  a.kscale = bins.kscale;
   a.codes = codes;
   a.norms = norms;
   a.err = L->d_error;
@@ -225,7 +240,7 @@ oq_status oq_rotate_quantize(const oq_layer* L, const void* x, int32_t x_dtype, 
   if (st != OQ_OK) return st;
   if (!codes || !s || !aligned(codes, 16) || !aligned(s, 4))
     return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize: codes (16-byte) / s (4-byte) pointers invalid");
-  return rq(L, x, x_dtype, T, L->a_bits, L->thr_a, codes, s, stream);
+  return rq(L, x, x_dtype, T, L->a_bits, L->bins_a, codes, s, stream);
 }
 
 oq_status oq_weight_prepare(const oq_layer* L, const void* W, int32_t W_dtype, uint32_t* Wcodes, float* r,
@@ -235,7 +250,7 @@ oq_status oq_weight_prepare(const oq_layer* L, const void* W, int32_t W_dtype, u
   if (st != OQ_OK) return st;
   if (!Wcodes || !r || !aligned(Wcodes, 16) || !aligned(r, 4))
     return fail(OQ_ERR_INVALID_ARG, "oq_weight_prepare: Wcodes (16-byte) / r (4-byte) pointers invalid");
-  return rq(L, W, W_dtype, L->d_out, L->w_bits, L->thr_w, Wcodes, r, stream);
+  return rq(L, W, W_dtype, L->d_out, L->w_bits, L->bins_w, Wcodes, r, stream);
 }
 
 static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T,
@@ -307,10 +322,11 @@ static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, in
   a.bits = L->a_bits;
   a.gather = L->d_gather_a;
   a.signmask = L->d_signmask;
-  a.thr = L->thr_a;
+  a.bins = L->bins_a.d_levels;
+  a.nb = L->bins_a.nb;
+  a.b0 = L->bins_a.b0;
+  a.kscale = L->bins_a.kscale;
   a.out16 = a16;
-  make_decode_tables(L->a_bits, L->lv_a, a.dtab);
-  a.lut8 = L->d_levels_a;
   a.norms = s;
   a.err = L->d_error;
   return rq_launch(a, stream);
@@ -363,7 +379,7 @@ oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int
   }
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws);
   float* s = reinterpret_cast<float*>(ws + ((fused_codes_bytes(L, T) + 255) & ~(size_t)255));
-  st = rq(L, x, x_dtype, T, L->a_bits, L->thr_a, codes, s, stream);
+  st = rq(L, x, x_dtype, T, L->a_bits, L->bins_a, codes, s, stream);
   if (st != OQ_OK) return st;
   return linear_impl(L, codes, s, T, Wcodes, r, y, stream);
 }

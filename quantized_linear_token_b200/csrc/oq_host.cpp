@@ -343,4 +343,50 @@ double choose_fp16_scale(const oq_codebook& cb) {
   return best;
 }
 
+
+// Threshold search table (see oq_bin_table): the smallest power of two K for
+// which consecutive scaled thresholds (as fp32, the values the kernel compares
+// against) lie more than one bin apart, then per bin the number of thresholds
+// in earlier bins and the one threshold inside it (+inf if none).
+oq_status build_bin_table(const oq_codebook& cb, int d, int h, const uint16_t* lv16, float* kscale, int* b0, int* nb,
+                          std::vector<uint32_t>& codes, std::vector<uint32_t>& levels) {
+  const int L = 1 << cb.bits;
+  const double sd = std::sqrt((double)d);
+  auto bits_of = [](float f) {
+    uint32_t u;
+    std::memcpy(&u, &f, 4);
+    return u;
+  };
+  for (int lk = 0; lk <= 16; ++lk) {
+    const double K = std::ldexp(1.0, lk);
+    std::vector<float> tk(L - 1);
+    for (int j = 0; j < L - 1; ++j) tk[j] = (float)(K * sd * cb.thresholds[j]);
+    bool apart = true;
+    for (int j = 1; j < L - 1 && apart; ++j) apart = (double)tk[j] - (double)tk[j - 1] > 1.0;
+    if (!apart) continue;
+    const int lo = (int)std::nearbyint(tk[0]) - 1, hi = (int)std::nearbyint(tk[L - 2]) + 1;
+    const int n = hi - lo + 1;
+    if (n > OQ_MAX_BINS) break;
+    codes.assign(2 * (size_t)n, 0u);
+    levels.assign(2 * (size_t)n, 0u);
+    int j = 0;
+    for (int b = 0; b < n; ++b) {
+      const int m = lo + b;
+      while (j < L - 1 && (int)std::nearbyint(tk[j]) < m) ++j;
+      const bool has = j < L - 1 && (int)std::nearbyint(tk[j]) == m;
+      const uint32_t t = bits_of(has ? tk[j] : INFINITY);
+      codes[2 * b] = t;
+      codes[2 * b + 1] = (uint32_t)j;
+      levels[2 * b] = t;
+      levels[2 * b + 1] = (uint32_t)lv16[j] | ((uint32_t)lv16[has ? j + 1 : j] << 16);
+    }
+    *kscale = (float)(K * sd / std::sqrt((double)h));
+    *b0 = -lo;
+    *nb = n;
+    return OQ_OK;
+  }
+  set_error("threshold table: codebook thresholds too close for a bin table");
+  return OQ_ERR_UNSUPPORTED;
+}
+
 }  // namespace oq

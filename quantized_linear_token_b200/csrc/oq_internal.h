@@ -11,6 +11,18 @@
 #define OQ_DEVERR_TIMEOUT 1
 #define OQ_DEVERR_BOUNDS 2
 
+// Threshold search table of one codebook for the rotate-quantize kernel: with
+// g = K sqrt(d) u (u the unit-norm rotated coordinate, K a power of two bins
+// per unit) every bin [m - 1/2, m + 1/2] holds at most one threshold
+// TK_j = K sqrt(d) t_j, so code = base + (g > TK) with (TK, base) of the bin of
+// rint(g); bins past the outermost thresholds clamp to the two end bins.
+struct oq_bin_table {
+  float kscale;        // K sqrt(d / h): g = z * kscale / s for the unnormalised FWHT output z
+  int b0, nb;          // bin index = clamp(rint(g) + b0, 0, nb - 1)
+  uint32_t* d_codes;   // device [nb] x {TK bits, base code}
+  uint32_t* d_levels;  // device [nb] x {TK bits, fp16 level of base | fp16 level of base+1 << 16}
+};
+
 struct oq_layer {
   int d_in, d_out, h, k, log_h, a_bits, w_bits, flags;
   uint64_t seed;
@@ -26,8 +38,7 @@ struct oq_layer {
   uint16_t* d_levels_w;               // fp16 bits of w_scale * weight levels
   uint16_t lv_a[256], lv_w[256];      // host copies of the two level tables
   int* d_error;                       // device error word
-  float thr_a[128];                   // sqrt(h) * positive thresholds, +inf padded
-  float thr_w[128];
+  oq_bin_table bins_a, bins_w;       // threshold search tables (activation / weight codebook)
 };
 
 namespace oq {
@@ -41,6 +52,10 @@ oq_status get_codebook(int d, int bits, int flags, oq_codebook* out);
 uint16_t f64_to_f16_bits(double v);
 double f16_bits_to_f64(uint16_t h);
 double choose_fp16_scale(const oq_codebook& cb);
+// threshold search table of a codebook (host copies; words interleaved TK, payload)
+constexpr int OQ_MAX_BINS = 4096;
+oq_status build_bin_table(const oq_codebook& cb, int d, int h, const uint16_t* lv16, float* kscale, int* b0, int* nb,
+                          std::vector<uint32_t>& codes, std::vector<uint32_t>& levels);
 
 // rotate + quantize launch (oq_rotate_quantize.cu): rows of `src` -> packed codes + norms
 struct RQArgs {
@@ -50,11 +65,11 @@ struct RQArgs {
   int d, h, log_h, bits;
   const uint16_t* gather;    // per-thread gather offsets (kernel order)
   const uint32_t* signmask;  // or null
-  const float* thr;          // host array of 128 scaled thresholds
+  const uint32_t* bins;      // device threshold search table (codes, or levels for out16)
+  int nb, b0;
+  float kscale;
   uint32_t* codes;           // [rows, d*bits/32], or
   uint16_t* out16;           // fp16 levels [rows, d] (fused layer call); null otherwise
-  uint32_t dtab[4];          // prmt decode tables for out16
-  const uint16_t* lut8;      // device 8-bit level table for out16
   float* norms;              // [rows]
   int* err;
 };

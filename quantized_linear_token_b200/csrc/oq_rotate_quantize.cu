@@ -68,9 +68,9 @@ struct RQKParams {
   uint16_t* out16;     // fp16 levels [rows, d] (fused layer call)
   float* norms;
   int* err;
-  uint32_t dtab[4];    // prmt decode tables of the levels (out16)
-  const uint16_t* lut8;  // 8-bit levels (out16)
-  float thr[128];      // sqrt(h) * positive thresholds tau_1.., +inf padded
+  const uint2* bins;   // threshold search table {TK bits, base code | fp16 level pair}
+  int nb, b0;
+  float kscale;        // g = z * kscale / s in bin units
 };
 
 template <typename XT>
@@ -127,27 +127,6 @@ __host__ __device__ constexpr uint32_t scatter_imm(int r) {
   return (uint32_t)(E * ((r * HE) / E) + 4 * ((((r * HE) % E) / 4) ^ (((r * HE) / E) & (E / 4 - 1))));
 }
 
-// number of thresholds strictly below `a` among th[0..n-1] (sorted, last = +inf)
-template <int BITS>
-__device__ __forceinline__ int count_below(const float* th, float a) {
-  if constexpr (BITS == 2) {
-    return th[0] < a ? 1 : 0;
-  } else if constexpr (BITS == 3) {
-    const bool c1 = th[1] < a;
-    const float t2 = c1 ? th[2] : th[0];
-    const bool c2 = t2 < a;
-    return (c1 ? 2 : 0) + (c2 ? 1 : 0);
-  } else {
-    static_assert(BITS == 4, "register search for 2..4 bits");
-    const bool c1 = th[3] < a;
-    const float t2 = c1 ? th[5] : th[1];
-    const bool c2 = t2 < a;
-    const float t3 = c1 ? (c2 ? th[6] : th[4]) : (c2 ? th[2] : th[0]);
-    const bool c3 = t3 < a;
-    return (c1 ? 4 : 0) + (c2 ? 2 : 0) + (c3 ? 1 : 0);
-  }
-}
-
 __host__ __device__ constexpr int elems_per_thread(int h) { return h <= 64 ? h : (h <= 1024 ? 32 : 64); }
 __host__ __device__ constexpr int log2i(int x) { return x <= 1 ? 0 : 1 + log2i(x / 2); }
 
@@ -162,8 +141,6 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
   constexpr int HE = H / E;
   constexpr int PASSES = (H <= 64) ? 1 : 2;
   constexpr int PAD = (PASSES == 2 && HE < 32) ? HE : 0;   // words between blocks
-  constexpr int N_HALF = 1 << (BITS - 1);
-  constexpr int NTH = (BITS <= 4) ? N_HALF : 1;
   extern __shared__ __align__(1024) unsigned char smem[];
 
   const int S = p.S, NT = p.NT, d = p.d;
@@ -173,14 +150,12 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
   const int tid = active ? (int)threadIdx.x - slot * NT : 0;
   const int j = tid / HE, c = tid % HE;
 
-  // shared memory: mbarriers | reduction partials | 8-bit thresholds | 8-bit
-  // levels | slots (two row buffers + exchange area each)
+  // shared memory: mbarriers | reduction partials | threshold search table |
+  // slots (two row buffers + exchange area each)
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem);
   float* red = reinterpret_cast<float*>(smem + 16 * S);
-  float* thr8 = red + blockDim.x;
-  uint16_t* lut8 = reinterpret_cast<uint16_t*>(thr8 + (BITS == 8 ? 128 * S : 0));
-  unsigned char* slots =
-      smem + (((16 * S + 4 * blockDim.x + (BITS == 8 ? 512 * S + 512 : 0)) + 1023) & ~1023);
+  uint2* tbl = reinterpret_cast<uint2*>(smem + ((16 * S + 4 * blockDim.x + 7) & ~7));
+  unsigned char* slots = smem + (((((16 * S + 4 * blockDim.x + 7) & ~7) + 8 * p.nb) + 1023) & ~1023);
   const int slot_bytes = 2 * p.stage_bytes + 4 * p.work_words;
   unsigned char* stage0 = slots + (size_t)slot * slot_bytes;
   float* work = reinterpret_cast<float*>(stage0 + 2 * p.stage_bytes);
@@ -203,10 +178,8 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
     for (int q = 0; q < (E / 32 > 0 ? E / 32 : 1); ++q)
       smask[q] = (p.has_signs && active) ? __ldg(p.signmask + (size_t)tid * (E / 32) + q) : 0u;
   }
-  // thresholds and decode tables stay in the parameter (constant) bank
-
-  if (OUT16 && BITS == 8)
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = p.lut8[i];
+  for (int i = threadIdx.x; i < p.nb; i += blockDim.x) tbl[i] = __ldg(p.bins + i);
+  const int nb1 = p.nb - 1, boff = p.b0 - 0x4B400000;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * S; ++i) mbar_init(&mbar[i], 1);
     fence_mbar_init();
@@ -311,64 +284,59 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
       for (int r = 0; r < E; ++r) z[r] = v[r];
     }
 
-    if constexpr (BITS == 8) {
-      // this token's scaled thresholds (127 and +inf) in shared memory; a
-      // zero token gets +inf everywhere (all coordinates 0 -> code L/2 - 1)
-      if (valid)
-        for (int k = tid; k < 128; k += NT) thr8[slot * 128 + k] = (s > 0.f) ? p.thr[k] * s : INFINITY;
-      __syncthreads();
-    }
-
     if (valid) {
-      // thresholds of this token; a zero token (s = 0) has every coordinate
-      // 0 and takes code L/2 - 1: +inf thresholds give exactly that
-      float ts[NTH];
-#pragma unroll
-      for (int k = 0; k < NTH; ++k) ts[k] = (s > 0.f) ? p.thr[k] * s : INFINITY;
+      // g = sqrt(d) K u with u = z / (s sqrt(h)): bin rint(g) (by the fp32
+      // magic-number round), clamped to the table, then one compare against
+      // the bin's threshold: code = #{thresholds below g} exactly (a value on
+      // a threshold takes the lower code).  A zero token (s = 0) gets g = 0 and
+      // code L/2 - 1; non-finite values land in a clamped bin.
+      const float ks = (s > 0.f) ? p.kscale / s : 0.f;
       const int pos0 = (PASSES == 2) ? (j * H + c * E) : (j * H);
+      // the table offset is threaded through each group of eight lookups
+      // (an empty asm that "uses" the group's result): at most eight table
+      // loads are in flight per thread, which keeps the registers in budget
+      int boffv = boff;
 #pragma unroll
       for (int gi = 0; gi < E / 32; ++gi) {
-        // quantize 32 consecutive positions straight into BITS packed words
-        uint32_t w[BITS];
-#pragma unroll
-        for (int q = 0; q < BITS; ++q) w[q] = 0u;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float zz = z[gi * 32 + i];
-          const float a = fabsf(zz);
-          const bool pos = zz > 0.f;
-          // ties: a value exactly on a threshold takes the lower code, i.e.
-          // count t < a for positive values and t <= a for the others
-          const float acmp = pos ? a : __uint_as_float(__float_as_uint(a) + 1u);
-          int cnt;
-          if constexpr (BITS <= 4) {
-            cnt = count_below<BITS>(ts, acmp);
-          } else {
-            const float* t8 = thr8 + slot * 128;
-            int lo = 0;
-#pragma unroll
-            for (int st = 64; st >= 1; st >>= 1)
-              if (t8[lo + st - 1] < acmp) lo += st;
-            cnt = lo;
-          }
-          const uint32_t cv = (uint32_t)(pos ? (N_HALF + cnt) : (N_HALF - 1 - cnt));
-          const int bit = i * BITS;
-          w[bit >> 5] |= cv << (bit & 31);
-          if ((bit & 31) + BITS > 32) w[(bit >> 5) + 1] |= cv >> (32 - (bit & 31));
-        }
         if constexpr (OUT16) {
-          // the levels of these 32 codes as fp16: the contraction's A operand
+          // the codes' fp16 levels (the contraction's A operand), two per word
+          uint32_t o[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            uint32_t sel = 0u, pay[2];
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const float g = z[gi * 32 + i + e2] * ks;
+              int m = __float_as_int(g + 12582912.0f) + boffv;
+              m = min(max(m, 0), nb1);
+              const uint2 en = tbl[m];
+              pay[e2] = en.y;
+              const bool up = g > __uint_as_float(en.x);
+              sel |= (up ? 0x32u : 0x10u) << (8 * e2);
+            }
+            o[i >> 1] = __byte_perm(pay[0], pay[1], sel | 0x4400u);
+            if ((i & 7) == 6) asm volatile("" : "+r"(boffv) : "r"(o[i >> 1]));
+          }
           uint4* dst = reinterpret_cast<uint4*>(p.out16 + (size_t)t * d + pos0 + gi * 32);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 o;
-            if constexpr (BITS == 4) o = dec4(w[q], p.dtab);
-            else if constexpr (BITS == 2) o = dec2((w[q >> 1] >> (16 * (q & 1))) & 0xFFFFu, p.dtab);
-            else if constexpr (BITS == 3) o = decode_chunk<3>(make_uint4(w[0], w[1], w[2], 0u), q, p.dtab, lut8);
-            else o = dec8(w[2 * q], w[2 * q + 1], lut8);
-            dst[q] = o;
-          }
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         } else {
+          // 32 consecutive positions straight into BITS packed words
+          uint32_t w[BITS];
+#pragma unroll
+          for (int q = 0; q < BITS; ++q) w[q] = 0u;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float g = z[gi * 32 + i] * ks;
+            int m = __float_as_int(g + 12582912.0f) + boffv;
+            m = min(max(m, 0), nb1);
+            const uint2 en = tbl[m];
+            const uint32_t cv = en.y + (g > __uint_as_float(en.x) ? 1u : 0u);
+            const int bit = i * BITS;
+            w[bit >> 5] |= cv << (bit & 31);
+            if ((bit & 31) + BITS > 32) w[(bit >> 5) + 1] |= cv >> (32 - (bit & 31));
+            if ((i & 7) == 7) asm volatile("" : "+r"(boffv) : "r"(w[bit >> 5]));
+          }
           uint32_t* dst = p.codes + (size_t)t * words_per_row + (size_t)((pos0 >> 5) + gi) * BITS;
           if constexpr (BITS == 4) {
             *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -406,7 +374,7 @@ oq_status launch_t(const RQKParams& kp_in, void* stream) {
   kp.S = S;
   kp.stage_bytes = (int)(((size_t)kp.d * sizeof(XT) + 15) & ~(size_t)15);
   const int slot_bytes = 2 * kp.stage_bytes + 4 * kp.work_words;
-  const size_t head = ((16 * S + 4 * threads + (BITS == 8 ? 512 * S + 512 : 0)) + 1023) & ~(size_t)1023;
+  const size_t head = (((16 * S + 4 * threads + 7) & ~(size_t)7) + 8 * (size_t)kp.nb + 1023) & ~(size_t)1023;
   const size_t smem = head + (size_t)S * slot_bytes;
   if (smem > 227 * 1024) return OQ_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -479,11 +447,11 @@ oq_status rq_launch(const RQArgs& a, void* stream) {
   kp.out16 = a.out16;
   kp.norms = a.norms;
   kp.err = a.err;
-  if (a.out16) {
-    for (int k = 0; k < 4; ++k) kp.dtab[k] = a.dtab[k];
-    kp.lut8 = a.lut8;
-  }
-  std::memcpy(kp.thr, a.thr, sizeof(kp.thr));
+  kp.bins = reinterpret_cast<const uint2*>(a.bins);
+  kp.nb = a.nb;
+  kp.b0 = a.b0;
+  kp.kscale = a.kscale;
+  if (a.nb < 1 || a.nb > OQ_MAX_BINS) return OQ_ERR_UNSUPPORTED;
   switch (a.bits) {
     case 2: return launch_bits<2>(kp, a, stream);
     case 3: return launch_bits<3>(kp, a, stream);
