@@ -130,10 +130,10 @@ __host__ __device__ constexpr uint32_t scatter_imm(int r) {
 __host__ __device__ constexpr int elems_per_thread(int h) { return h <= 64 ? h : (h <= 1024 ? 32 : 64); }
 __host__ __device__ constexpr int log2i(int x) { return x <= 1 ? 0 : 1 + log2i(x / 2); }
 
-// register budget: 112 for 32 values per thread (3 CTAs of 192 per SM),
-// 168 for 64 values per thread
+// register budget: 96 for 32 values per thread (seven CTAs of 96 threads per
+// SM), 168 for 64 values per thread
 template <int BITS, int LOG_H, typename XT, bool OUT16>
-__global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
+__global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 96)
     rq_kernel(const __grid_constant__ RQKParams p) {
   constexpr int H = 1 << LOG_H;
   constexpr int E = elems_per_thread(H);
@@ -151,29 +151,29 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
   const int j = tid / HE, c = tid % HE;
 
   // shared memory: mbarriers | reduction partials | threshold search table |
-  // slots (two row buffers + exchange area each)
+  // gather offsets | slots (two row buffers + exchange area each)
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem);
   float* red = reinterpret_cast<float*>(smem + 16 * S);
-  uint2* tbl = reinterpret_cast<uint2*>(smem + ((16 * S + 4 * blockDim.x + 7) & ~7));
-  unsigned char* slots = smem + (((((16 * S + 4 * blockDim.x + 7) & ~7) + 8 * p.nb) + 1023) & ~1023);
+  const int tbl_off = (16 * S + 4 * blockDim.x + 15) & ~15;
+  uint2* tbl = reinterpret_cast<uint2*>(smem + tbl_off);
+  const int gtab_off = (tbl_off + 8 * p.nb + 15) & ~15;
+  uint4* gtab = reinterpret_cast<uint4*>(smem + gtab_off);   // [E/8][NT]: conflict-free per q
+  unsigned char* slots = smem + ((gtab_off + 2 * d + 1023) & ~1023);
   const int slot_bytes = 2 * p.stage_bytes + 4 * p.work_words;
   unsigned char* stage0 = slots + (size_t)slot * slot_bytes;
   float* work = reinterpret_cast<float*>(stage0 + 2 * p.stage_bytes);
   const uint32_t stage0_addr = smem_u32(stage0);
 
-  // this thread's gather offsets (pairs of 16-bit channel indices) and signs
-  uint32_t gidx[E / 2];
+  // the gather offsets (16-bit channel indices, kernel order) go to shared
+  // memory transposed so that a warp reads its threads' next eight offsets
+  // with one conflict-free 16-byte load each; this thread's sign bits stay in
+  // registers
+  for (int i = threadIdx.x; i < d / 8; i += blockDim.x) {
+    const int t = i % NT, q = i / NT;
+    gtab[i] = __ldg(reinterpret_cast<const uint4*>(p.gather) + (size_t)t * (E / 8) + q);
+  }
   uint32_t smask[E / 32 > 0 ? E / 32 : 1];
   {
-    const uint4* g4 = reinterpret_cast<const uint4*>(p.gather + (size_t)tid * E);
-#pragma unroll
-    for (int q = 0; q < E / 8; ++q) {
-      const uint4 v = active ? __ldg(g4 + q) : make_uint4(0, 0, 0, 0);
-      gidx[4 * q + 0] = v.x;
-      gidx[4 * q + 1] = v.y;
-      gidx[4 * q + 2] = v.z;
-      gidx[4 * q + 3] = v.w;
-    }
 #pragma unroll
     for (int q = 0; q < (E / 32 > 0 ? E / 32 : 1); ++q)
       smask[q] = (p.has_signs && active) ? __ldg(p.signmask + (size_t)tid * (E / 32) + q) : 0u;
@@ -225,9 +225,14 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
     float v[E];
     float ss = 0.f;
 #pragma unroll
-    for (int r = 0; r < E; ++r) {
-      const uint32_t gi = (r & 1) ? (gidx[r >> 1] >> 16) : (gidx[r >> 1] & 0xFFFFu);
-      v[r] = valid ? load_x<XT>(stage_addr, gi) : 0.f;
+    for (int q = 0; q < E / 8; ++q) {
+      const uint4 gq = gtab[q * NT + tid];
+      const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
+#pragma unroll
+      for (int e8 = 0; e8 < 8; ++e8) {
+        const uint32_t gi = (e8 & 1) ? (gw[e8 >> 1] >> 16) : (gw[e8 >> 1] & 0xFFFFu);
+        v[8 * q + e8] = valid ? load_x<XT>(stage_addr, gi) : 0.f;
+      }
     }
     if (p.has_signs) {
 #pragma unroll
@@ -292,10 +297,7 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
       // code L/2 - 1; non-finite values land in a clamped bin.
       const float ks = (s > 0.f) ? p.kscale / s : 0.f;
       const int pos0 = (PASSES == 2) ? (j * H + c * E) : (j * H);
-      // the table offset is threaded through each group of eight lookups
-      // (an empty asm that "uses" the group's result): at most eight table
-      // loads are in flight per thread, which keeps the registers in budget
-      int boffv = boff;
+      const int boffv = boff;
 #pragma unroll
       for (int gi = 0; gi < E / 32; ++gi) {
         if constexpr (OUT16) {
@@ -315,7 +317,6 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
               sel |= (up ? 0x32u : 0x10u) << (8 * e2);
             }
             o[i >> 1] = __byte_perm(pay[0], pay[1], sel | 0x4400u);
-            if ((i & 7) == 6) asm volatile("" : "+r"(boffv) : "r"(o[i >> 1]));
           }
           uint4* dst = reinterpret_cast<uint4*>(p.out16 + (size_t)t * d + pos0 + gi * 32);
 #pragma unroll
@@ -335,7 +336,6 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 112)
             const int bit = i * BITS;
             w[bit >> 5] |= cv << (bit & 31);
             if ((bit & 31) + BITS > 32) w[(bit >> 5) + 1] |= cv >> (32 - (bit & 31));
-            if ((i & 7) == 7) asm volatile("" : "+r"(boffv) : "r"(w[bit >> 5]));
           }
           uint32_t* dst = p.codes + (size_t)t * words_per_row + (size_t)((pos0 >> 5) + gi) * BITS;
           if constexpr (BITS == 4) {
@@ -374,7 +374,8 @@ oq_status launch_t(const RQKParams& kp_in, void* stream) {
   kp.S = S;
   kp.stage_bytes = (int)(((size_t)kp.d * sizeof(XT) + 15) & ~(size_t)15);
   const int slot_bytes = 2 * kp.stage_bytes + 4 * kp.work_words;
-  const size_t head = (((16 * S + 4 * threads + 7) & ~(size_t)7) + 8 * (size_t)kp.nb + 1023) & ~(size_t)1023;
+  const size_t head = ((((((16 * S + 4 * threads + 15) & ~(size_t)15) + 8 * (size_t)kp.nb + 15) & ~(size_t)15) +
+                        2 * (size_t)kp.d) + 1023) & ~(size_t)1023;
   const size_t smem = head + (size_t)S * slot_bytes;
   if (smem > 227 * 1024) return OQ_ERR_UNSUPPORTED;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
