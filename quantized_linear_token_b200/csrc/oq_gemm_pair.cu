@@ -417,7 +417,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
       constexpr uint32_t idesc = idesc_f16_f32(2 * RM, PN);
       int s = 0;
       uint32_t n = 0;
-      bool ok = true;
+      bool ok = true, rdy = false;
+      // the descriptors of all stages share their high word; the low word is
+      // the start address / 16 (plus the constant leading-offset field), so
+      // one descriptor per stage and K step is one 32-bit add (this thread
+      // shares its sub-partition with busy decoder warps: every instruction
+      // it saves is issue latency off the MMA's critical path)
+      const uint64_t desc0 = smem_desc_sw128(smem_base);
+      const uint32_t d_hi = (uint32_t)(desc0 >> 32), a_lo0 = (uint32_t)desc0;
       for (int64_t i = 0; i < my_tiles && ok; ++i) {
         const int a = (int)(i & 1);
         const uint32_t u = (uint32_t)(i >> 1);
@@ -425,21 +432,33 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(a * PN);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait_cluster(&op_full[s], n & 1u, p.err)) {
+          if (!rdy && !mbar_wait_cluster(&op_full[s], n & 1u, p.err)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_base + (uint32_t)(s * STAGE_BYTES), b_addr = a_addr + A_TILE;
-#pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma_f16_ss_pair(d_tmem, smem_desc_sw128(a_addr + kk * 32), smem_desc_sw128(b_addr + kk * 32), idesc,
-                               (kb > 0 || kk > 0) ? 1u : 0u);
-          tc_commit_pair_mc(&op_empty[s], (uint16_t)0x3);
-          if (++s == OS) {
-            s = 0;
-            ++n;
+          // probe the next stage before issuing this one's MMAs: a barrier
+          // check takes ~200 cycles even when the phase is long complete, and
+          // its answer is only needed after these MMAs are issued
+          int s1 = s + 1;
+          uint32_t n1 = n;
+          if (s1 == OS) {
+            s1 = 0;
+            ++n1;
           }
+          const bool more = kb + 1 < nkb || i + 1 < my_tiles;
+          const bool rdy1 = more && mbar_test_wait_cluster(&op_full[s1], n1 & 1u);
+          const uint32_t a_lo = a_lo0 + (uint32_t)s * (uint32_t)(STAGE_BYTES >> 4);
+          tc_mma_f16_ss_pair(d_tmem, ((uint64_t)d_hi << 32) | a_lo, ((uint64_t)d_hi << 32) | (a_lo + (A_TILE >> 4)),
+                             idesc, kb > 0 ? 1u : 0u);
+#pragma unroll
+          for (int kk = 1; kk < BK / UMMA_K; ++kk)
+            tc_mma_f16_ss_pair(d_tmem, ((uint64_t)d_hi << 32) | (a_lo + 2 * kk),
+                               ((uint64_t)d_hi << 32) | (a_lo + (A_TILE >> 4) + 2 * kk), idesc, 1u);
+          tc_commit_pair_mc(&op_empty[s], (uint16_t)0x3);
+          s = s1;
+          n = n1;
+          rdy = rdy1;
         }
         tc_commit_pair_mc(&acc_full[a], (uint16_t)0x3);
       }
