@@ -139,6 +139,7 @@ EDGE = [
     (128, 128, 8, 4, 5, 0),        # h = 128, 8-bit activations
     (640, 272, 4, 3, 257, 1),      # h = 128, k = 5, Rademacher signs
     (1024, 256, 4, 4, 130, 2),     # Gaussian-marginal codebook
+    (3072, 512, 4, 4, 96, 3),      # image-DiT width, signed RPBH and Gaussian marginal together
     (2048, 128, 4, 2, 70, 0),      # h = 2048 (64 per thread, two passes)
     (6144, 512, 3, 4, 33, 0),      # h = 2048, k = 3
 ]

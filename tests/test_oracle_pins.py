@@ -319,6 +319,46 @@ def test_rotated_coordinates_follow_the_marginal(key, d, T):
     assert stats.kstest(v, "norm").statistic <= 0.01
 
 
+def test_signed_rotation_keeps_the_marginal():
+    # pith Supplementary A adds Rademacher signs D before H; the rotated
+    # coordinates of the same outlier-heavy activations still follow the one
+    # fixed marginal (the signed RPBH variant of the scope's next steps)
+    wl = W.WORKLOADS["dit_image"]
+    d, T = 3072, 400
+    x = O.bf16_bits_to_f64(W.activations(wl, d, T))
+    _, _, u = O.rotate_quantize(x, O.rpbh_permutation(d, 0), O.hadamard_block_size(d), O.lloyd_max(d, 4),
+                                signs=O.rademacher_signs(d, 0))
+    assert stats.kstest((u * math.sqrt(d)).ravel(), "norm").statistic <= 0.01
+
+
+def test_signed_and_gaussian_variants_match_the_default():
+    # The two flag variants (signed RPBH; codebook on N(0, 1/d) instead of the
+    # exact sphere marginal) against the default on the image-DiT recipe at
+    # W4A4: at d = 3072 the two codebooks nearly coincide and the signs leave
+    # the marginal unchanged, so the layer error ||y_q - W x|| / ||W x|| of all
+    # four combinations agrees to within a few percent.
+    wl = W.WORKLOADS["dit_image"]
+    lay = wl.layers[0]
+    d, T, dout = 3072, 48, 256
+    x = O.bf16_bits_to_f64(W.activations(wl, d, T))
+    Wm = W.weights(wl, lay)[:dout].astype(np.float64)
+    h, perm = O.hadamard_block_size(d), O.rpbh_permutation(d, 0)
+    yx = O.linear_exact(x, Wm)
+    errs = {}
+    for signed in (False, True):
+        sg = O.rademacher_signs(d, 0) if signed else None
+        for gauss in (False, True):
+            cb = O.lloyd_max(d, 4, gauss)
+            xc, s, _ = O.rotate_quantize(x, perm, h, cb, signs=sg)
+            wc, r, _ = O.weight_prepare(Wm, perm, h, cb, signs=sg)
+            y, _ = O.linear_from_codes(xc, s, wc, r, cb.levels, cb.levels)
+            errs[(signed, gauss)] = np.linalg.norm(y - yx) / np.linalg.norm(yx)
+    base = errs[(False, False)]
+    assert 0.02 < base < 0.2
+    for v in errs.values():
+        assert abs(v / base - 1.0) < 0.05
+
+
 def test_permutation_balances_block_masses():
     # gecl notes Key Insight: without the permutation, outliers sitting in one
     # block leave that block with most of the mass; Pi spreads them out.
