@@ -179,8 +179,10 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
 
 /*
  * oq_linear_fused -- x -> y in one call: the rotate-quantize step produces
- * the A operand of the contraction (same results as oq_rotate_quantize
- * followed by oq_linear).  With bf16 x and d_out % 256 == 0 the rotate-quantize
+ * the A operand of the contraction (the same codes as oq_rotate_quantize
+ * followed by oq_linear, and the same y; for batches of at most 256 tokens the
+ * contraction runs a split-K kernel whose fp32 sums come in another order, so
+ * y agrees to rounding).  With bf16 x and d_out % 256 == 0 the rotate-quantize
  * kernel writes the fp16 levels of the activation codes, which the contraction
  * reads with TMA (only the weight codes are decoded in the contraction);
  * otherwise the packed codes pass through the workspace.  `workspace` is
@@ -214,7 +216,15 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  *   Needs d_out % 256 == 0 (else OQ_ERR_UNSUPPORTED); y 16-byte aligned.
  *
  * oq_rotate_quantize_levels followed by oq_linear_levels gives exactly the y
- * of oq_linear_fused (and of oq_rotate_quantize + oq_linear).
+ * of oq_linear_fused (and of oq_rotate_quantize + oq_linear, up to summation
+ * order for batches of at most 256 tokens).
+ *
+ * Small batches (T <= 256, d_out % 128 == 0) take a kernel whose M dimension
+ * is 128 weight rows and whose N is the padded batch, with the K range split
+ * across the SMs (the batch-1 / GEMV end of the workload sweep); the splits of
+ * a tile add into y in a fixed order through per-layer counters, so results
+ * repeat bit for bit, and calls on one layer must not overlap on the GPU
+ * (different streams or host threads).
  */
 oq_status oq_rotate_quantize_levels(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
                                     uint16_t* a16, float* s, void* stream);

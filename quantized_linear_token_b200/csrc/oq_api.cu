@@ -93,6 +93,7 @@ void oq_layer_destroy(oq_layer* L) {
   cudaFree(L->bins_a.d_levels);
   cudaFree(L->bins_w.d_codes);
   cudaFree(L->bins_w.d_levels);
+  cudaFree(L->d_counters);
   cudaFree(L->d_error);
   delete L;
 }
@@ -167,6 +168,11 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   upload(&L->bins_a.d_levels, ta_levels);
   upload(&L->bins_w.d_codes, tw_codes);
   upload(&L->bins_w.d_levels, tw_levels);
+  if (st == OQ_OK && d_out % 128 == 0) {
+    const size_t cb = (size_t)(d_out / 32) * sizeof(int);
+    st = cuda_check(cudaMalloc(&L->d_counters, cb), "cudaMalloc(split counters)");
+    if (st == OQ_OK) st = cuda_check(cudaMemset(L->d_counters, 0, cb), "clear split counters");
+  }
   if (st == OQ_OK) st = cuda_check(cudaMalloc(&L->d_error, sizeof(int)), "cudaMalloc(error word)");
   if (st == OQ_OK) st = cuda_check(cudaMemset(L->d_error, 0, sizeof(int)), "clear error word");
   if (st != OQ_OK) {
@@ -274,6 +280,9 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
   g.a_bits = L->a_bits;
   g.b_bits = L->w_bits;
   g.err = L->d_error;
+  // a few hundred tokens or fewer: the small-batch kernel (weight rows as the
+  // MMA's M, split K); larger batches: the CTA-pair kernel
+  if (a_f16 && T <= SKINNY_MAX_T && L->d_counters) return gemm_skinny_launch(g, L->d_counters, stream);
   return gemm_launch(g, stream);
 }
 
@@ -392,6 +401,8 @@ oq_status oq_poll_error(const oq_layer* L) {
   st = cuda_check(cudaMemcpy(&word, L->d_error, sizeof(int), cudaMemcpyDeviceToHost), "oq_poll_error: read");
   if (st != OQ_OK) return st;
   if (word) cudaMemset(L->d_error, 0, sizeof(int));
+  // a timed-out small-batch call can leave split counters mid-way
+  if ((word & OQ_DEVERR_TIMEOUT) && L->d_counters) cudaMemset(L->d_counters, 0, (size_t)(L->d_out / 32) * sizeof(int));
   if (word & OQ_DEVERR_TIMEOUT) return fail(OQ_ERR_TIMEOUT, "a kernel's bounded wait ran out");
   if (word & OQ_DEVERR_BOUNDS) return fail(OQ_ERR_DEVICE, "a kernel's bounds check fired");
   return OQ_OK;

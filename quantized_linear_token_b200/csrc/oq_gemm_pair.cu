@@ -31,6 +31,7 @@
 #include "oq_decode.cuh"
 #include "oq_internal.h"
 #include "oq_ptx.cuh"
+#include "oq_tmap.cuh"
 
 namespace oq {
 namespace {
@@ -437,9 +438,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
             break;
           }
           tc_fence_after();
-          // probe the next stage before issuing this one's MMAs: a barrier
-          // check takes ~200 cycles even when the phase is long complete, and
-          // its answer is only needed after these MMAs are issued
+          // probe the next stage while this one's MMAs issue (a barrier check
+          // costs ~200 cycles even when the phase is long complete)
           int s1 = s + 1;
           uint32_t n1 = n;
           if (s1 == OS) {
@@ -447,15 +447,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
             ++n1;
           }
           const bool more = kb + 1 < nkb || i + 1 < my_tiles;
-          const bool rdy1 = more && mbar_test_wait_cluster(&op_full[s1], n1 & 1u);
           const uint32_t a_lo = a_lo0 + (uint32_t)s * (uint32_t)(STAGE_BYTES >> 4);
-          tc_mma_f16_ss_pair(d_tmem, ((uint64_t)d_hi << 32) | a_lo, ((uint64_t)d_hi << 32) | (a_lo + (A_TILE >> 4)),
-                             idesc, kb > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 1; kk < BK / UMMA_K; ++kk)
-            tc_mma_f16_ss_pair(d_tmem, ((uint64_t)d_hi << 32) | (a_lo + 2 * kk),
-                               ((uint64_t)d_hi << 32) | (a_lo + (A_TILE >> 4) + 2 * kk), idesc, 1u);
-          tc_commit_pair_mc(&op_empty[s], (uint16_t)0x3);
+          const bool rdy1 = tc_kblock64_f16<2>(d_tmem, a_lo, a_lo + (A_TILE >> 4), d_hi, idesc, kb > 0 ? 1u : 0u,
+                                               &op_empty[s], (uint16_t)0x3, &op_full[s1], n1 & 1u, more ? 1u : 0u);
           s = s1;
           n = n1;
           rdy = rdy1;
@@ -529,32 +523,9 @@ oq_status launch_pair_b(const PairParams& kp, int b_bits, void* stream) {
   }
 }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
-// against the driver library)
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn g_encode = nullptr;
-
-static oq_status encode_fn(EncodeTiledFn* out) {
-  if (!g_encode) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
-    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) {
-      set_error("cuTensorMapEncodeTiled is not available from the driver");
-      return OQ_ERR_CUDA;
-    }
-    g_encode = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  *out = g_encode;
-  return OQ_OK;
-}
-
 oq_status encode_y_map(CUtensorMap* map, float* y, int64_t M, int N) {
   EncodeTiledFn fn = nullptr;
-  const oq_status st = encode_fn(&fn);
+  const oq_status st = tmap_encode_fn(&fn);
   if (st != OQ_OK) return st;
   const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
   const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
@@ -565,24 +536,6 @@ oq_status encode_y_map(CUtensorMap* map, float* y, int64_t M, int N) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_error("cuTensorMapEncodeTiled failed for y (code " + std::to_string((int)r) + ")");
-    return OQ_ERR_CUDA;
-  }
-  return OQ_OK;
-}
-
-oq_status encode_a_map(CUtensorMap* map, const uint16_t* a16, int64_t M, int K) {
-  EncodeTiledFn fn = nullptr;
-  const oq_status st = encode_fn(&fn);
-  if (st != OQ_OK) return st;
-  const cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)RM};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t*>(a16), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    set_error("cuTensorMapEncodeTiled failed for the fp16 A operand (code " + std::to_string((int)r) + ")");
     return OQ_ERR_CUDA;
   }
   return OQ_OK;
@@ -619,7 +572,8 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream) {
   if (g.a_f16) {
     // fp16 A operand fetched by TMA: 16-byte aligned rows of K halves
     if ((reinterpret_cast<uintptr_t>(g.a_f16) & 15) || (g.K % 8)) return OQ_ERR_UNSUPPORTED;
-    const oq_status st = encode_a_map(&kp.a_map, g.a_f16, g.M, g.K);
+    const oq_status st = encode_operand_map(&kp.a_map, g.a_f16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.M, g.K, RM,
+                                            "the fp16 A operand");
     if (st != OQ_OK) return st;
     return launch_pair_b<4, true>(kp, g.b_bits, stream);
   }

@@ -39,6 +39,7 @@ struct oq_layer {
   uint16_t lv_a[256], lv_w[256];      // host copies of the two level tables
   int* d_error;                       // device error word
   oq_bin_table bins_a, bins_w;       // threshold search tables (activation / weight codebook)
+  int* d_counters;                    // split-K hand-off counters of the small-batch contraction (zero at rest)
 };
 
 namespace oq {
@@ -99,6 +100,10 @@ struct GemmArgs {
 oq_status gemm_launch(const GemmArgs& g, void* stream);
 // paired-CTA contraction (oq_gemm_pair.cu); OQ_ERR_UNSUPPORTED unless N % 256 == 0
 oq_status gemm_pair_launch(const GemmArgs& g, void* stream);
+// small-batch contraction (oq_gemm_skinny.cu): fp16 A operand, T <= SKINNY_MAX_T,
+// N % 128 == 0; `counters` holds N / 32 zeroed ints
+constexpr int SKINNY_MAX_T = 256;
+oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream);
 // prmt decode tables of a codebook's fp16 levels (oq_gemm.cu)
 void make_decode_tables(int bits, const uint16_t* levels, uint32_t* t);
 

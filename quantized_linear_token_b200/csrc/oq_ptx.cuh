@@ -262,6 +262,62 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
                : "memory");
 }
 
+// One K block of 64 (four kind::f16 MMAs of K 16; the smem descriptors
+// {lo, hi} advance by 2 in their low word per K step), the commit of its
+// completion to `bar`, and -- when `probe` is set -- a non-blocking check of
+// phase `next_parity` of `next_bar` (.acquire.cluster).  The probe is issued
+// before the MMAs and its answer is only read after them, so the ~200-cycle
+// latency of a barrier check overlaps the MMA issue.  `accumulate` applies to
+// the first MMA; the other three always accumulate.
+template <int CG>
+__device__ __forceinline__ bool tc_kblock64_f16(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t d_hi,
+                                                uint32_t idesc, uint32_t accumulate, uint64_t* bar, uint16_t mask,
+                                                uint64_t* next_bar, uint32_t next_parity, uint32_t probe) {
+  uint32_t ready;
+  if constexpr (CG == 2) {
+    asm volatile(
+        "{\n\t.reg .pred pa, pt, pp, pn;\n\t.reg .b64 da, db;\n\t.reg .b32 al, bl;\n\t"
+        "setp.ne.b32 pa, %5, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\tsetp.ne.b32 pp, %10, 0;\n\t"
+        "setp.ne.b32 pn, 0, 0;\n\t"
+        "@pp mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 pn, [%8], %9;\n\t"
+        "mov.b64 da, {%2, %4};\n\tmov.b64 db, {%3, %4};\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], da, db, %6, pa;\n\t"
+        "add.u32 al, %2, 2;\n\tadd.u32 bl, %3, 2;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], da, db, %6, pt;\n\t"
+        "add.u32 al, %2, 4;\n\tadd.u32 bl, %3, 4;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], da, db, %6, pt;\n\t"
+        "add.u32 al, %2, 6;\n\tadd.u32 bl, %3, 6;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], da, db, %6, pt;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%7], %11;\n\t"
+        "selp.u32 %0, 1, 0, pn;\n\t}"
+        : "=r"(ready)
+        : "r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(accumulate), "r"(idesc), "r"(smem_u32(bar)),
+          "r"(smem_u32(next_bar)), "r"(next_parity), "r"(probe), "h"(mask)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred pa, pt, pp, pn;\n\t.reg .b64 da, db;\n\t.reg .b32 al, bl;\n\t"
+        "setp.ne.b32 pa, %5, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\tsetp.ne.b32 pp, %10, 0;\n\t"
+        "setp.ne.b32 pn, 0, 0;\n\t"
+        "@pp mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 pn, [%8], %9;\n\t"
+        "mov.b64 da, {%2, %4};\n\tmov.b64 db, {%3, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%1], da, db, %6, pa;\n\t"
+        "add.u32 al, %2, 2;\n\tadd.u32 bl, %3, 2;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%1], da, db, %6, pt;\n\t"
+        "add.u32 al, %2, 4;\n\tadd.u32 bl, %3, 4;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%1], da, db, %6, pt;\n\t"
+        "add.u32 al, %2, 6;\n\tadd.u32 bl, %3, 6;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%1], da, db, %6, pt;\n\t"
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
+        "selp.u32 %0, 1, 0, pn;\n\t}"
+        : "=r"(ready)
+        : "r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(accumulate), "r"(idesc), "r"(smem_u32(bar)),
+          "r"(smem_u32(next_bar)), "r"(next_parity), "r"(probe), "h"(mask)
+        : "memory");
+  }
+  return ready != 0;
+}
+
 // ---------------------------------------------------------------- tcgen05, CTA pair
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),

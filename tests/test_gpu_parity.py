@@ -62,14 +62,39 @@ def _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, flags=0, seed=0, w_ro
     # contraction on the GPU's own codes
     y_np, yf_np = y.cpu().numpy(), yf.cpu().numpy()
     lin = check_linear(y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, label + " y", rows=y_rows)
-    # the fused call computes the same codes, so the same y
-    np.testing.assert_array_equal(yf_np, y_np)
+    # the fused call computes the same codes, so the same y: bit for bit when
+    # both run the CTA-pair kernel; for small batches the fused route runs the
+    # split-K small-batch kernel (another summation order), which is checked
+    # against the oracle itself and against the codes route to fp32 rounding
+    _same_y(yf_np, y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, T_small=_small_batch(x_np, d_out),
+            label=label + " fused", rows=y_rows)
     if x_np.dtype == np.uint16 and d_out % 256 == 0:
-        _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in)
+        _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in,
+                            Wc_np, r_np, cb_w, y_rows, label)
     return st, lin
 
 
-def _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in):
+SKINNY_MAX_T = 256   # batches up to this size take the small-batch kernel on the fp16-level route
+
+
+def _small_batch(x_np, d_out):
+    return x_np.dtype == np.uint16 and x_np.shape[0] <= SKINNY_MAX_T and d_out % 128 == 0
+
+
+def _same_y(y_new, y_ref, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, T_small, label, rows=None):
+    if not T_small:
+        np.testing.assert_array_equal(y_new, y_ref)
+        return
+    check_linear(y_new, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, label, rows=rows)
+    _, bound = O.linear_from_codes(O.unpack_codes(codes_np, cb_a.bits, d_in), s_np.astype(np.float64),
+                                   O.unpack_codes(Wc_np, cb_w.bits, d_in), r_np.astype(np.float64),
+                                   cb_a.levels, cb_w.levels)
+    diff = np.abs(y_new.astype(np.float64) - y_ref.astype(np.float64))
+    assert float((diff / np.where(bound > 0, bound, 1.0)).max()) <= 1e-5, label
+
+
+def _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in, Wc_np, r_np, cb_w,
+                        y_rows, label):
     """The fused call's fp16 route as two calls: the A operand holds exactly the
     fp16 value of a_scale times the level of each code, the norms are the
     same, and the contraction gives the same y."""
@@ -82,7 +107,14 @@ def _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bi
     c = O.unpack_codes(codes_np, a_bits, d_in)
     want = (layer.a_scale * np.asarray(cb_a.levels, dtype=np.float64))[c].astype(np.float16).view(np.uint16)
     np.testing.assert_array_equal(a16.cpu().numpy().view(np.uint16), want)
-    np.testing.assert_array_equal(y2.cpu().numpy(), y_np)
+    # the split-K small-batch path adds its splits in a fixed order: repeat
+    # calls give the same bits
+    y3 = B.oq_linear_levels(layer, a16, s2, Wc, r)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(y3.cpu().numpy(), y2.cpu().numpy())
+    _same_y(y2.cpu().numpy(), y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in,
+            T_small=codes_np.shape[0] <= SKINNY_MAX_T and Wc_np.shape[0] % 128 == 0, label=label + " levels",
+            rows=y_rows)
 
 
 CASES = [
@@ -150,6 +182,16 @@ def test_edge_shapes(env, d_in, d_out, a_bits, w_bits, T, flags):
     x_np = W.custom_activations(T, d_in, seed=d_in + T, outliers=min(4, d_in // 8))
     Wm = W.custom_weights(d_out, d_in, seed=d_out)
     _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, flags=flags, seed=3, label=f"edge{d_in}x{d_out}")
+
+
+@pytest.mark.parametrize("T", [1, 16, 64, 200, 256, 257])
+def test_small_batch_sweep(env, T):
+    # the small-T end of the workload sweep (d 13824 -> 5120, W4A4): batches of
+    # up to 256 tokens take the split-K small-batch kernel, 257 the CTA pair
+    x_np, Wm = _inputs("stress_w4a4", 13824, 5120, T)
+    rng = np.random.default_rng(11)
+    w_rows = np.unique(np.concatenate([np.arange(32), rng.choice(5120, 64, replace=False)]))
+    _run_layer(env, 13824, 5120, 4, 4, x_np, Wm, w_rows=w_rows, label=f"small{T}")
 
 
 def test_degenerate_tokens(env):
