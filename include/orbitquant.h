@@ -66,9 +66,13 @@ enum {
   OQ_FLAG_SIGNS = 1,              /* Rademacher signs D_j before each block
                                      Hadamard (pith Supplementary A);
                                      off by default                          */
-  OQ_FLAG_GAUSSIAN_MARGINAL = 2   /* design the codebook on N(0, 1/d) (pith
+  OQ_FLAG_GAUSSIAN_MARGINAL = 2,  /* design the codebook on N(0, 1/d) (pith
                                      Figure 2) instead of the exact sphere
                                      marginal f_d                            */
+  OQ_FLAG_WEIGHT_ONLY_INT4 = 4    /* the AdaLN exception path (gecl notes
+                                     Method 5: INT4 weight-only RTN, no
+                                     rotation, 16-bit activations); see
+                                     oq_layer_create                         */
 };
 
 /*
@@ -119,6 +123,17 @@ oq_status oq_rotation_build(int32_t d, uint64_t seed, int32_t flags, uint32_t* p
  * `*out` is library-owned; release it with oq_layer_destroy.
  * Errors: OQ_ERR_INVALID_ARG (null out), OQ_ERR_UNSUPPORTED (shape/bits),
  * OQ_ERR_NOMEM / OQ_ERR_CUDA (allocation or upload failed).
+ *
+ * With OQ_FLAG_WEIGHT_ONLY_INT4 (alone in `flags`) the layer is the AdaLN
+ * modulation projection that the pages keep at INT4 weight-only round-to-
+ * nearest because a static rotation cannot fold into it (gecl notes Method 5):
+ *   a_bits must be 16 and w_bits 4, d_in % 32 == 0, d_out % 128 == 0;
+ *   oq_weight_prepare stores per row r_o = max_i |w_oi| / 7 and codes of
+ *     q = round-half-even(w / r_o) in [-7, 7] (fp32, IEEE division), in the
+ *     4-bit code format (q >= 0 -> q + 8, q < 0 -> q + 7);
+ *   oq_linear_fused with bf16 x gives y = x (q r)^T in fp32 (bf16 operands on
+ *     the tensor cores, fp32 accumulation); its workspace size is 0;
+ *   the rotation and activation-code calls return OQ_ERR_UNSUPPORTED.
  */
 typedef struct oq_layer oq_layer;
 

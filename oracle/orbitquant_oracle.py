@@ -60,12 +60,17 @@ __all__ = [
     "linear_exact",
     "OQ_SIGNS",
     "OQ_GAUSSIAN_MARGINAL",
+    "OQ_WEIGHT_ONLY_INT4",
+    "int4_rtn_weight_prepare",
+    "int4_level",
+    "int4_rtn_linear",
 ]
 
 # Option flags; the same numeric values as the C-ABI flags (a documented
 # interface, not shared code).
 OQ_SIGNS = 1              # Rademacher signs D_j before each block Hadamard
 OQ_GAUSSIAN_MARGINAL = 2  # design the codebook on N(0,1/d) instead of exact f_d
+OQ_WEIGHT_ONLY_INT4 = 4   # AdaLN exception path: INT4 round-to-nearest weights, 16-bit activations
 
 _MASK64 = (1 << 64) - 1
 
@@ -451,3 +456,42 @@ def linear_from_codes(codes_a: np.ndarray, s: np.ndarray, codes_w: np.ndarray,
 def linear_exact(x: np.ndarray, W: np.ndarray) -> np.ndarray:
     """The unquantised layer y = W x for every token (llmdb summary)."""
     return np.asarray(x, dtype=np.float64) @ np.asarray(W, dtype=np.float64).T
+
+
+# ------------------------------------------------------------ AdaLN exception
+# gecl notes Method 5: the dynamic AdaLN modulation projection cannot absorb a
+# static rotation, so it is kept at INT4 weight-only round-to-nearest (the
+# podcast page says the same: INT4, not the 2-bit of the rest).  The pages do
+# not say how the scale is chosen; reading D18: symmetric, one scale per
+# output row, s_o = max_i |w_oi| / 7, q = round-half-even(w / s_o) in
+# [-7, 7], no rotation and no activation quantization.  The decision of each
+# integer is taken in fp32 (the precision the kernel takes it in: the pages
+# fix none), with IEEE division and round-half-even, so the codes are exact.
+# Codes use the 4-bit format of the Lloyd-Max codes: c >= 8 is the level
+# c - 8, c < 8 the level c - 7 (q >= 0 -> q + 8, q < 0 -> q + 7).
+
+def int4_rtn_weight_prepare(W: np.ndarray):
+    """INT4 RTN of each weight row (reading D18).  Returns (codes [d_out, d_in]
+    int in 0..15 -- 7 never occurs --, scale [d_out] float32)."""
+    W32 = np.asarray(W, dtype=np.float32)
+    amax = np.max(np.abs(W32), axis=1)
+    scale = (amax / np.float32(7.0)).astype(np.float32)        # IEEE fp32 division
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = np.rint((W32 / safe[:, None]).astype(np.float32))       # fp32 quotient, ties to even
+    q = np.where(scale[:, None] > 0, np.clip(q, -7, 7), 0).astype(np.int64)
+    codes = np.where(q >= 0, q + 8, q + 7)
+    return codes, scale
+
+
+def int4_level(codes: np.ndarray) -> np.ndarray:
+    """The integer level of an INT4 code (c >= 8: c - 8; c < 8: c - 7)."""
+    codes = np.asarray(codes, dtype=np.int64)
+    return np.where(codes >= 8, codes - 8, codes - 7)
+
+
+def int4_rtn_linear(x: np.ndarray, codes: np.ndarray, scale: np.ndarray):
+    """y = x W^T with the RTN weights (level * scale) in fp64, and the bound
+    sum_i |x_i| |w^_oi| used for the bound-relative tolerance."""
+    Wq = int4_level(codes).astype(np.float64) * np.asarray(scale, dtype=np.float64)[:, None]
+    x = np.asarray(x, dtype=np.float64)
+    return x @ Wq.T, np.abs(x) @ np.abs(Wq).T

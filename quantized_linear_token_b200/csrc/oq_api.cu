@@ -98,10 +98,59 @@ void oq_layer_destroy(oq_layer* L) {
   delete L;
 }
 
+// The AdaLN exception layer (gecl notes Method 5): INT4 weight-only RTN, no
+// rotation, no codebooks; bf16 decode tables of the integer levels -7..7.
+static oq_status create_int4_layer(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_bits, int32_t w_bits,
+                                   int32_t flags, oq_layer** out) {
+  if (flags != OQ_FLAG_WEIGHT_ONLY_INT4)
+    return fail(OQ_ERR_INVALID_ARG, "OQ_FLAG_WEIGHT_ONLY_INT4 takes no other flag");
+  if (a_bits != 16 || w_bits != 4)
+    return fail(OQ_ERR_UNSUPPORTED, "the INT4 weight-only layer takes a_bits = 16, w_bits = 4");
+  if (d_in <= 0 || d_out <= 0) return fail(OQ_ERR_INVALID_ARG, "dimensions must be positive");
+  if (d_in % 32 || d_out % 128)
+    return fail(OQ_ERR_UNSUPPORTED, "the INT4 weight-only layer needs d_in % 32 == 0 and d_out % 128 == 0");
+  oq_layer* L = new (std::nothrow) oq_layer();
+  if (!L) return fail(OQ_ERR_NOMEM, "host allocation failed");
+  L->int4_only = true;
+  L->d_in = d_in;
+  L->d_out = d_out;
+  L->h = d_in & -d_in;
+  L->k = d_in / L->h;
+  L->a_bits = a_bits;
+  L->w_bits = w_bits;
+  L->flags = flags;
+  L->seed = seed;
+  L->a_scale = L->w_scale = 1.0;
+  cudaGetDevice(&L->device);
+  // bf16 bits of the level of each code (c >= 8: c - 8; c < 8: c - 7)
+  for (int c = 0; c < 16; ++c) {
+    const float v = (float)(c >= 8 ? c - 8 : c - 7);
+    uint32_t u;
+    std::memcpy(&u, &v, 4);
+    L->lv_w[c] = (uint16_t)(u >> 16);   // exact: small integers
+  }
+  const size_t cb = (size_t)(d_out / 32) * sizeof(int);
+  oq_status st = cuda_check(cudaMalloc(&L->d_counters, cb), "cudaMalloc(split counters)");
+  if (st == OQ_OK) st = cuda_check(cudaMemset(L->d_counters, 0, cb), "clear split counters");
+  if (st == OQ_OK) st = cuda_check(cudaMalloc(&L->d_error, sizeof(int)), "cudaMalloc(error word)");
+  if (st == OQ_OK) st = cuda_check(cudaMemset(L->d_error, 0, sizeof(int)), "clear error word");
+  if (st != OQ_OK) {
+    oq_layer_destroy(L);
+    return st;
+  }
+  *out = L;
+  return OQ_OK;
+}
+
+static oq_status not_for_int4(const oq_layer* L, const char* who) {
+  return fail(OQ_ERR_UNSUPPORTED, std::string(who) + ": not available on an INT4 weight-only layer");
+}
+
 oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_bits, int32_t w_bits,
                           int32_t flags, oq_layer** out) {
   if (!out) return fail(OQ_ERR_INVALID_ARG, "oq_layer_create: out is null");
   *out = nullptr;
+  if (flags & OQ_FLAG_WEIGHT_ONLY_INT4) return create_int4_layer(d_in, d_out, seed, a_bits, w_bits, flags, out);
   oq_status st = check_shape(d_in, d_out, a_bits, w_bits);
   if (st != OQ_OK) return st;
   if (flags & ~(OQ_FLAG_SIGNS | OQ_FLAG_GAUSSIAN_MARGINAL)) return fail(OQ_ERR_INVALID_ARG, "unknown flag bits");
@@ -203,6 +252,7 @@ oq_status oq_layer_get_info(const oq_layer* L, oq_layer_info* out) {
 
 oq_status oq_layer_get_perm(const oq_layer* L, uint32_t* perm) {
   if (!L || !perm) return fail(OQ_ERR_INVALID_ARG, "oq_layer_get_perm: null argument");
+  if (L->int4_only) return not_for_int4(L, "oq_layer_get_perm");
   std::memcpy(perm, L->perm_host.data(), L->perm_host.size() * sizeof(uint32_t));
   return OQ_OK;
 }
@@ -240,6 +290,7 @@ static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t row
 oq_status oq_rotate_quantize(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint32_t* codes,
                              float* s, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize: layer is null");
+  if (L->int4_only) return not_for_int4(L, "oq_rotate_quantize");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize: T < 0");
   if (T == 0) return OQ_OK;
   oq_status st = check_rows_input(x, x_dtype, "oq_rotate_quantize");
@@ -256,6 +307,7 @@ oq_status oq_weight_prepare(const oq_layer* L, const void* W, int32_t W_dtype, u
   if (st != OQ_OK) return st;
   if (!Wcodes || !r || !aligned(Wcodes, 16) || !aligned(r, 4))
     return fail(OQ_ERR_INVALID_ARG, "oq_weight_prepare: Wcodes (16-byte) / r (4-byte) pointers invalid");
+  if (L->int4_only) return rtn4_prepare_launch(W, W_dtype, L->d_out, L->d_in, Wcodes, r, stream);
   return rq(L, W, W_dtype, L->d_out, L->w_bits, L->bins_w, Wcodes, r, stream);
 }
 
@@ -289,6 +341,7 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
 oq_status oq_linear(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T, const uint32_t* Wcodes,
                     const float* r, float* y, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear: layer is null");
+  if (L->int4_only) return not_for_int4(L, "oq_linear");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear: T < 0");
   if (T == 0) return OQ_OK;
   if (!codes || !s || !Wcodes || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear: null pointer");
@@ -313,7 +366,7 @@ static size_t fused_codes_bytes(const oq_layer* L, int64_t T) {
 static size_t fused_f16_bytes(const oq_layer* L, int64_t T) { return (size_t)T * (size_t)L->d_in * 2; }
 
 size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
-  if (!L || T <= 0) return 0;
+  if (!L || T <= 0 || L->int4_only) return 0;
   size_t a = fused_codes_bytes(L, T);
   if (L->d_out % 256 == 0) a = std::max(a, fused_f16_bytes(L, T));
   return ((a + 255) & ~(size_t)255) + (size_t)T * 4;
@@ -344,6 +397,7 @@ static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, in
 oq_status oq_rotate_quantize_levels(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint16_t* a16,
                                     float* s, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize_levels: layer is null");
+  if (L->int4_only) return not_for_int4(L, "oq_rotate_quantize_levels");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize_levels: T < 0");
   if (T == 0) return OQ_OK;
   oq_status st = check_rows_input(x, x_dtype, "oq_rotate_quantize_levels");
@@ -357,6 +411,7 @@ oq_status oq_rotate_quantize_levels(const oq_layer* L, const void* x, int32_t x_
 oq_status oq_linear_levels(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint32_t* Wcodes,
                            const float* r, float* y, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: layer is null");
+  if (L->int4_only) return not_for_int4(L, "oq_linear_levels");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: T < 0");
   if (T == 0) return OQ_OK;
   if (!a16 || !s || !Wcodes || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: null pointer");
@@ -366,6 +421,37 @@ oq_status oq_linear_levels(const oq_layer* L, const uint16_t* a16, const float* 
   return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
 }
 
+// y = x (q r)^T for the INT4 weight-only layer: bf16 x straight into the
+// small-batch kernel as its token operand, in launches of up to 256 tokens
+static oq_status int4_linear(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                             const float* r, float* y, void* stream) {
+  if (x_dtype != OQ_DTYPE_BF16) return fail(OQ_ERR_UNSUPPORTED, "INT4 weight-only layer: bf16 activations only");
+  if (!Wcodes || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: null pointer");
+  if (!aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(r, 4))
+    return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: misaligned pointer");
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  for (int64_t t0 = 0; t0 < T; t0 += SKINNY_MAX_T) {
+    GemmArgs g{};
+    g.a_f16 = xb + t0 * L->d_in;
+    g.a_bf16 = true;
+    g.b_codes = Wcodes;
+    g.a_scale = nullptr;
+    g.b_scale = r;
+    g.b_levels_host = L->lv_w;
+    g.out_scale = 1.f;
+    g.y = y + t0 * L->d_out;
+    g.M = std::min<int64_t>(SKINNY_MAX_T, T - t0);
+    g.N = L->d_out;
+    g.K = L->d_in;
+    g.a_bits = 16;
+    g.b_bits = 4;
+    g.err = L->d_error;
+    const oq_status st = gemm_skinny_launch(g, L->d_counters, stream);
+    if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "INT4 weight-only layer: unsupported shape") : st;
+  }
+  return OQ_OK;
+}
+
 oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
                           const float* r, float* y, void* workspace, size_t workspace_bytes, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: layer is null");
@@ -373,6 +459,7 @@ oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int
   if (T == 0) return OQ_OK;
   oq_status st = check_rows_input(x, x_dtype, "oq_linear_fused");
   if (st != OQ_OK) return st;
+  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, y, stream);
   if (!Wcodes || !r || !y || !workspace) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: null pointer");
   if (!aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(r, 16) || !aligned(workspace, 256))
     return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: misaligned pointer (workspace needs 256 bytes)");

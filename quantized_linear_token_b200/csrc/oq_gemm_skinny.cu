@@ -94,7 +94,9 @@ __device__ __forceinline__ Item item_of(const SkinnyParams& p, int w) {
   return it;
 }
 
-template <int B_BITS>
+// TOK_BF16: the token operand is bf16 (the INT4 weight-only layer's x), and
+// the weight levels are decoded as bf16 too (one operand type per MMA)
+template <int B_BITS, bool TOK_BF16>
 __global__ void __launch_bounds__(NTHREADS, 1) gemm_skinny_kernel(const __grid_constant__ SkinnyParams p) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_skinny_kernel(const __grid_c
   } else if (warp == MMA_WARP) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_f16_f32(WR, p.NT);
+      const uint32_t idesc = TOK_BF16 ? idesc_bf16_f32(WR, p.NT) : idesc_f16_f32(WR, p.NT);
       const uint64_t desc0 = smem_desc_sw128(smem_base);
       const uint32_t d_hi = (uint32_t)(desc0 >> 32), w_lo0 = (uint32_t)desc0;
       int s = 0;
@@ -330,18 +332,24 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_skinny_kernel(const __grid_c
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(qd * 32) << 16) + (uint32_t)a * acc_cols + (uint32_t)c0, v);
         tmem_wait_ld();
-        // the previous splits' sums of these 32 tokens: all loads first (no
+        // the previous splits' sums, 16 tokens at a time: all loads first (no
         // load waits behind a store), then the stores
-        float old[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = c0 + j;
-          old[j] = (it.split > 0 && t < p.T) ? __ldcg(p.y + (int64_t)t * p.N + o) : 0.f;
-        }
+        for (int h = 0; h < 32; h += 16) {
+          float old[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = c0 + j;
-          if (t < p.T) p.y[(int64_t)t * p.N + o] = __uint_as_float(v[j]) * ro * __ldg(p.a_scale + t) + old[j];
+          for (int j = 0; j < 16; ++j) {
+            const int t = c0 + h + j;
+            old[j] = (it.split > 0 && t < p.T) ? __ldcg(p.y + (int64_t)t * p.N + o) : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = c0 + h + j;
+            if (t < p.T) {
+              const float st = p.a_scale ? __ldg(p.a_scale + t) : 1.f;
+              p.y[(int64_t)t * p.N + o] = __uint_as_float(v[h + j]) * ro * st + old[j];
+            }
+          }
         }
       }
       tc_fence_before();
@@ -363,10 +371,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_skinny_kernel(const __grid_c
   }
 }
 
-template <int B_BITS>
+template <int B_BITS, bool TOK_BF16>
 oq_status launch_skinny(const SkinnyParams& kp_in, void* stream) {
   SkinnyParams kp = kp_in;
-  auto kern = gemm_skinny_kernel<B_BITS>;
+  auto kern = gemm_skinny_kernel<B_BITS, TOK_BF16>;
   kp.stage_bytes = W_TILE + kp.NT * BK * 2;
   constexpr int ring_bytes = NCS * WR * (2 * BK * B_BITS / 8);
   kp.stages = std::min(MAX_STAGES, (208 * 1024 - ring_bytes) / kp.stage_bytes);
@@ -420,8 +428,9 @@ oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream) {
   kp.nkb = (g.K + BK - 1) / BK;
   make_decode_tables(g.b_bits, g.b_levels_host, kp.b_tab);
   kp.kc = make_deck();
-  oq_status st = encode_operand_map(&kp.x_map, g.a_f16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.M, g.K, kp.NT,
-                                    "the fp16 token operand");
+  oq_status st = encode_operand_map(&kp.x_map, g.a_f16,
+                                    g.a_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.M,
+                                    g.K, kp.NT, "the token operand");
   if (st != OQ_OK) return st;
   {
     // weight codes as a byte matrix [N, K bits / 8]; rows must be 16-byte multiples
@@ -442,10 +451,11 @@ oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream) {
       return OQ_ERR_CUDA;
     }
   }
+  if (g.a_bf16) return g.b_bits == 4 ? launch_skinny<4, true>(kp, stream) : OQ_ERR_UNSUPPORTED;
   switch (g.b_bits) {
-    case 2: return launch_skinny<2>(kp, stream);
-    case 3: return launch_skinny<3>(kp, stream);
-    case 4: return launch_skinny<4>(kp, stream);
+    case 2: return launch_skinny<2, false>(kp, stream);
+    case 3: return launch_skinny<3, false>(kp, stream);
+    case 4: return launch_skinny<4, false>(kp, stream);
     default: return OQ_ERR_UNSUPPORTED;
   }
 }

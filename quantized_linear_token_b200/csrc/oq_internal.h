@@ -25,6 +25,7 @@ struct oq_bin_table {
 
 struct oq_layer {
   int d_in, d_out, h, k, log_h, a_bits, w_bits, flags;
+  bool int4_only;                     // OQ_FLAG_WEIGHT_ONLY_INT4: AdaLN path (no rotation or codebooks)
   uint64_t seed;
   int device;
   oq_codebook cb_a, cb_w;
@@ -84,8 +85,9 @@ oq_status rq_launch(const RQArgs& a, void* stream);
 struct GemmArgs {
   const uint32_t* a_codes;   // [M, K*a_bits/32]
   const uint16_t* a_f16;     // or: fp16 levels of A [M, K] (fused call), null otherwise
+  bool a_bf16;               // a_f16 holds bf16 values (INT4 weight-only layer; b levels are bf16 too)
   const uint32_t* b_codes;   // [N, K*b_bits/32]
-  const float* a_scale;      // [M] per-row magnitude s
+  const float* a_scale;      // [M] per-row magnitude s (null: 1)
   const float* b_scale;      // [N] per-row magnitude r
   const uint16_t* a_levels;       // device fp16 bits, 2^a_bits (8-bit table)
   const uint16_t* b_levels;       // device fp16 bits, 2^b_bits
@@ -104,6 +106,10 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream);
 // N % 128 == 0; `counters` holds N / 32 zeroed ints
 constexpr int SKINNY_MAX_T = 256;
 oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream);
+// INT4 weight-only round-to-nearest of weight rows (oq_int4.cu): per-row
+// scale max|w| / 7 and 4-bit codes of q in [-7, 7] (q >= 0 -> q + 8, else q + 7)
+oq_status rtn4_prepare_launch(const void* W, int w_dtype, int rows, int d, uint32_t* codes, float* scale,
+                              void* stream);
 // prmt decode tables of a codebook's fp16 levels (oq_gemm.cu)
 void make_decode_tables(int bits, const uint16_t* levels, uint32_t* t);
 

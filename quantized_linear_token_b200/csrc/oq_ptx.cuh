@@ -181,12 +181,17 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_addr) {
 }
 
 // Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 D, M x N.
+// the same with bf16 A and B (both operands of a kind::f16 MMA share a type)
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N);
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4)                                   // D format f32
          | (0u << 7) | (0u << 10)                    // A, B format f16
          | (0u << 15) | (0u << 16)                   // A, B K-major
          | ((uint32_t)(N >> 3) << 17)                // N / 8
          | ((uint32_t)(M >> 4) << 24);               // M / 16
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return idesc_f16_f32(M, N) | (1u << 7) | (1u << 10);   // A, B format bf16
 }
 
 // ---------------------------------------------------------------- clusters

@@ -194,6 +194,38 @@ def test_small_batch_sweep(env, T):
     _run_layer(env, 13824, 5120, 4, 4, x_np, Wm, w_rows=w_rows, label=f"small{T}")
 
 
+@pytest.mark.parametrize("T,d_in,d_out,w_bf16", [(2, 3072, 18432, False), (7, 1024, 256, True),
+                                                   (300, 512, 384, False)])
+def test_int4_weight_only_layer(env, T, d_in, d_out, w_bf16):
+    # the AdaLN exception path (INT4 weight-only RTN; modulation width 6 x 3072
+    # at batch 2, a bf16-weight case, and more than 256 tokens): codes and
+    # scales bit-exact against the oracle (both decide in fp32), y against the
+    # oracle's fp64 contraction of the same codes
+    torch, B = env
+    layer = B.oq_layer_create(d_in, d_out, 0, 16, 4, B.OQ_FLAG_WEIGHT_ONLY_INT4)
+    Wm = W.custom_weights(d_out, d_in, seed=d_out + 1)
+    if w_bf16:
+        Wm = W.bf16_bits_to_f32(W.f32_to_bf16_bits(Wm))
+        W_t = torch.from_numpy(Wm).cuda().to(torch.bfloat16)
+    else:
+        W_t = torch.from_numpy(Wm).cuda()
+    Wc, r = B.oq_weight_prepare(layer, W_t)
+    x_np = W.custom_activations(T, d_in, seed=T + 3)
+    x_t, x64 = _x_tensor(torch, x_np)
+    y = B.oq_linear_fused(layer, x_t, Wc, r)
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+    codes_or, scale_or = O.int4_rtn_weight_prepare(Wm)
+    np.testing.assert_array_equal(r.cpu().numpy().view(np.uint32), scale_or.view(np.uint32))
+    np.testing.assert_array_equal(O.unpack_codes(to_numpy_u32(Wc), 4, d_in), codes_or)
+    y_or, bound = O.int4_rtn_linear(x64, codes_or, scale_or)
+    rel = np.abs(y.cpu().numpy().astype(np.float64) - y_or) / np.where(bound > 0, bound, 1.0)
+    assert float(rel.max()) <= 1e-3
+    for call in (lambda: B.oq_rotate_quantize(layer, x_t), lambda: B.oq_linear(layer, Wc, r, Wc, r)):
+        with pytest.raises(B.OrbitQuantError):
+            call()
+
+
 def test_degenerate_tokens(env):
     # a zero token (s = 0, every code L/2 - 1, y = 0) and tokens with very
     # small and very large norms

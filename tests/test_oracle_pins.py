@@ -414,3 +414,45 @@ def test_linear_exact_when_codebooks_are_fine():
     cw = u.size + np.arange(v.size).reshape(v.shape)
     y, _ = O.linear_from_codes(ca, np.linalg.norm(x, axis=1), cw, np.linalg.norm(Wm, axis=1), levels, levels)
     np.testing.assert_allclose(y, O.linear_exact(x, Wm), rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- INT4 RTN (AdaLN)
+def test_int4_rtn_hand_example():
+    # one row, max |w| = 3.5 -> scale 0.5: w / s = [7, -2, 1.5, 0.5, -0.5, 0]
+    # round half to even -> [7, -2, 2, 0, -0, 0]; codes q+8 / q+7
+    codes, scale = O.int4_rtn_weight_prepare(np.array([[3.5, -1.0, 0.75, 0.25, -0.25, 0.0]]))
+    assert scale.tolist() == [np.float32(0.5)]
+    assert O.int4_level(codes).tolist() == [[7, -2, 2, 0, 0, 0]]
+    assert codes.tolist() == [[15, 5, 10, 8, 8, 8]]
+
+
+def test_int4_rtn_is_nearest_level_brute_force():
+    rng = np.random.default_rng(3)
+    W = (rng.standard_normal((40, 96)) * rng.uniform(0.01, 3.0, (40, 1))).astype(np.float32)
+    codes, scale = O.int4_rtn_weight_prepare(W)
+    assert set(np.unique(codes).tolist()) <= set(range(16)) - {7}
+    lv = O.int4_level(codes)
+    assert np.all(np.abs(lv).max(axis=1) == 7)                 # the largest |w| maps to +-7
+    cand = np.arange(-7, 8)
+    for o in range(W.shape[0]):
+        t = W[o].astype(np.float64) / float(scale[o])
+        best = cand[np.argmin(np.abs(t[:, None] - cand[None, :]), axis=1)]
+        # away from exact ties the fp32 decision is the nearest integer level
+        far = np.abs(np.abs(t - np.floor(t)) - 0.5) > 1e-5
+        assert np.array_equal(lv[o][far], best[far])
+    err = np.abs(W - lv * scale[:, None])
+    assert np.all(err <= 0.5 * scale[:, None] * (1 + 1e-6))
+
+
+def test_int4_rtn_zero_row_and_lossless_row():
+    codes, scale = O.int4_rtn_weight_prepare(np.zeros((1, 8)))
+    assert scale[0] == 0 and np.all(O.int4_level(codes) == 0)
+    # a row already on the grid (integer multiples of max / 7) is reproduced exactly
+    lv = np.array([[7, -7, 3, -2, 0, 1, -5, 6]], dtype=np.float64)
+    W = lv * 0.25
+    codes, scale = O.int4_rtn_weight_prepare(W)
+    np.testing.assert_array_equal(O.int4_level(codes), lv)
+    x = np.random.default_rng(5).standard_normal((3, 8))
+    y, bound = O.int4_rtn_linear(x, codes, scale)
+    np.testing.assert_allclose(y, x @ W.T, rtol=0, atol=1e-12)
+    assert np.all(np.abs(y) <= bound + 1e-12)
