@@ -69,10 +69,17 @@ enum {
   OQ_FLAG_GAUSSIAN_MARGINAL = 2,  /* design the codebook on N(0, 1/d) (pith
                                      Figure 2) instead of the exact sphere
                                      marginal f_d                            */
-  OQ_FLAG_WEIGHT_ONLY_INT4 = 4    /* the AdaLN exception path (gecl notes
+  OQ_FLAG_WEIGHT_ONLY_INT4 = 4,   /* the AdaLN exception path (gecl notes
                                      Method 5: INT4 weight-only RTN, no
                                      rotation, 16-bit activations); see
                                      oq_layer_create                         */
+  OQ_FLAG_FP8_CONTRACTION = 8     /* lower-precision contraction mode: both
+                                     operands' 4-bit codes decode to e4m3 and
+                                     multiply on kind::f8f6f4 tensor cores
+                                     (twice the fp16 rate).  Same codes, but y
+                                     carries the e4m3 rounding of the levels
+                                     and does not meet the 1e-3 bound of the
+                                     default mode; see oq_layer_create       */
 };
 
 /*
@@ -134,6 +141,13 @@ oq_status oq_rotation_build(int32_t d, uint64_t seed, int32_t flags, uint32_t* p
  *   oq_linear_fused with bf16 x gives y = x (q r)^T in fp32 (bf16 operands on
  *     the tensor cores, fp32 accumulation); its workspace size is 0;
  *   the rotation and activation-code calls return OQ_ERR_UNSUPPORTED.
+ *
+ * With OQ_FLAG_FP8_CONTRACTION (combinable with the two codebook/rotation
+ * flags) a_bits and w_bits must be 4 and d_out % 256 == 0: the codes and
+ * norms are those of the default mode, while oq_linear and oq_linear_fused
+ * decode both operands' levels to e4m3 (each codebook scaled so its levels
+ * land closest to e4m3 values) and accumulate in fp32.  The fp16-level calls
+ * (oq_rotate_quantize_levels, oq_linear_levels) return OQ_ERR_UNSUPPORTED.
  */
 typedef struct oq_layer oq_layer;
 

@@ -22,6 +22,7 @@ OQ_DTYPE_BF16 = 1
 OQ_FLAG_SIGNS = 1
 OQ_FLAG_GAUSSIAN_MARGINAL = 2
 OQ_FLAG_WEIGHT_ONLY_INT4 = 4
+OQ_FLAG_FP8_CONTRACTION = 8
 
 # every symbol include/orbitquant.h declares
 EXPORTS = (

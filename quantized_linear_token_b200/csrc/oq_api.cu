@@ -153,7 +153,10 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   if (flags & OQ_FLAG_WEIGHT_ONLY_INT4) return create_int4_layer(d_in, d_out, seed, a_bits, w_bits, flags, out);
   oq_status st = check_shape(d_in, d_out, a_bits, w_bits);
   if (st != OQ_OK) return st;
-  if (flags & ~(OQ_FLAG_SIGNS | OQ_FLAG_GAUSSIAN_MARGINAL)) return fail(OQ_ERR_INVALID_ARG, "unknown flag bits");
+  if (flags & ~(OQ_FLAG_SIGNS | OQ_FLAG_GAUSSIAN_MARGINAL | OQ_FLAG_FP8_CONTRACTION))
+    return fail(OQ_ERR_INVALID_ARG, "unknown flag bits");
+  if ((flags & OQ_FLAG_FP8_CONTRACTION) && (a_bits != 4 || w_bits != 4 || d_out % 256))
+    return fail(OQ_ERR_UNSUPPORTED, "the FP8 contraction mode needs a_bits = w_bits = 4 and d_out % 256 == 0");
 
   oq_layer* L = new (std::nothrow) oq_layer();
   if (!L) return fail(OQ_ERR_NOMEM, "host allocation failed");
@@ -187,6 +190,15 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   for (int i = 0; i < (1 << w_bits); ++i) lv_w[i] = f64_to_f16_bits(L->w_scale * L->cb_w.levels[i]);
   std::memcpy(L->lv_a, lv_a, sizeof(lv_a));
   std::memcpy(L->lv_w, lv_w, sizeof(lv_w));
+  if (flags & OQ_FLAG_FP8_CONTRACTION) {
+    L->fp8 = true;
+    L->a8_scale = choose_fp8_scale(L->cb_a, &L->a8_err);
+    L->w8_scale = choose_fp8_scale(L->cb_w, &L->w8_err);
+    for (int i = 0; i < 16; ++i) {
+      L->lv8_a[i] = f64_to_e4m3_bits(L->a8_scale * L->cb_a.levels[i]);
+      L->lv8_w[i] = f64_to_e4m3_bits(L->w8_scale * L->cb_w.levels[i]);
+    }
+  }
   std::vector<uint32_t> ta_codes, ta_levels, tw_codes, tw_levels;
   if ((st = build_bin_table(L->cb_a, d_in, L->h, lv_a, &L->bins_a.kscale, &L->bins_a.b0, &L->bins_a.nb, ta_codes,
                             ta_levels)) != OQ_OK ||
@@ -325,6 +337,12 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
   g.a_levels_host = L->lv_a;
   g.b_levels_host = L->lv_w;
   g.out_scale = (float)(1.0 / (L->a_scale * L->w_scale));
+  if (L->fp8) {
+    g.fp8 = true;
+    g.a_levels8 = L->lv8_a;
+    g.b_levels8 = L->lv8_w;
+    g.out_scale = (float)(1.0 / (L->a8_scale * L->w8_scale));
+  }
   g.y = y;
   g.M = T;
   g.N = L->d_out;
@@ -356,7 +374,7 @@ oq_status oq_linear(const oq_layer* L, const uint32_t* codes, const float* s, in
 // only the weight codes are decoded during the contraction.  Otherwise the
 // packed codes go through the workspace to the code-decoding contraction.
 static bool fused_f16_route(const oq_layer* L, int32_t x_dtype) {
-  return x_dtype == OQ_DTYPE_BF16 && L->d_out % 256 == 0;
+  return x_dtype == OQ_DTYPE_BF16 && L->d_out % 256 == 0 && !L->fp8;
 }
 
 static size_t fused_codes_bytes(const oq_layer* L, int64_t T) {
@@ -398,6 +416,7 @@ oq_status oq_rotate_quantize_levels(const oq_layer* L, const void* x, int32_t x_
                                     float* s, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize_levels: layer is null");
   if (L->int4_only) return not_for_int4(L, "oq_rotate_quantize_levels");
+  if (L->fp8) return fail(OQ_ERR_UNSUPPORTED, "oq_rotate_quantize_levels: the fp16-level route is not used in the FP8 mode");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_rotate_quantize_levels: T < 0");
   if (T == 0) return OQ_OK;
   oq_status st = check_rows_input(x, x_dtype, "oq_rotate_quantize_levels");
@@ -412,6 +431,7 @@ oq_status oq_linear_levels(const oq_layer* L, const uint16_t* a16, const float* 
                            const float* r, float* y, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: layer is null");
   if (L->int4_only) return not_for_int4(L, "oq_linear_levels");
+  if (L->fp8) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_levels: the fp16-level route is not used in the FP8 mode");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: T < 0");
   if (T == 0) return OQ_OK;
   if (!a16 || !s || !Wcodes || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: null pointer");

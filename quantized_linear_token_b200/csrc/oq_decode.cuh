@@ -151,6 +151,31 @@ __device__ __forceinline__ uint4 decode_chunk_k(const uint4& v, int j, const uin
   }
 }
 
+// ---- FP8 (e4m3) decode of 4-bit codes, for the lower-precision contraction
+// mode: one byte per value, so a byte permute yields four values at once.
+// t[0], t[1]: e4m3 bytes of the eight positive levels (magnitude index 0-7).
+constexpr int DEC_BK_F8 = 128;   // K elements per operand block (128 bytes of e4m3)
+
+__device__ __forceinline__ uint2 dec4_e4m3k(uint32_t w, const uint32_t (&t)[4], const DecK& k) {
+  const uint32_t n = (__umulhi(w, k.hi29) & 0x11111111u) ^ 0x11111111u;  // 1 per negative code (bit 3 clear)
+  const uint32_t m = (w & 0x77777777u) ^ (n * k.seven);                   // magnitude index
+  const uint32_t mh = __umulhi(m, k.hi16), nh = __umulhi(n, k.hi16);
+  return make_uint2(__byte_perm(t[0], t[1], m) | __byte_perm(0x8000u, 0u, n),
+                    __byte_perm(t[0], t[1], mh) | __byte_perm(0x8000u, 0u, nh));
+}
+
+// the codes of part q (32 codes, 16 bytes) of FP8 K block kb of a 4-bit row (zeros past K)
+__device__ __forceinline__ uint4 load_part_f8(const uint32_t* row, int kb, int q, int K) {
+  if (kb * DEC_BK_F8 + q * 32 >= K) return make_uint4(0u, 0u, 0u, 0u);
+  return __ldg(reinterpret_cast<const uint4*>(row) + kb * 4 + q);
+}
+
+// chunk j (16 codes -> 16 e4m3 bytes) of an FP8 part
+__device__ __forceinline__ uint4 decode_chunk_f8(const uint4& v, int j, const uint32_t (&t)[4], const DecK& k) {
+  const uint2 a = dec4_e4m3k(j == 0 ? v.x : v.z, t, k), b = dec4_e4m3k(j == 0 ? v.y : v.w, t, k);
+  return make_uint4(a.x, a.y, b.x, b.y);
+}
+
 // chunk j of a part -> 8 fp16
 template <int BITS>
 __device__ __forceinline__ uint4 decode_chunk(const uint4& v, int j, const uint32_t (&t)[4], const uint16_t* lut8) {

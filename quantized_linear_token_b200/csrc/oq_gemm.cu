@@ -343,6 +343,7 @@ void make_decode_tables(int bits, const uint16_t* lv, uint32_t* t) {
 
 oq_status gemm_launch(const GemmArgs& g, void* stream) {
   if (g.M == 0) return OQ_OK;
+  if (g.fp8) return gemm_pair_launch(g, stream);   // the FP8 mode exists only on CTA pairs
   // CTA-pair tiles (256 x 256) whenever the output width allows them
   if (g.N % 256 == 0) {
     const oq_status st = gemm_pair_launch(g, stream);

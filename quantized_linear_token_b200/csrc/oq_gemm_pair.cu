@@ -79,7 +79,9 @@ struct PairParams {
 // own fetches each 128 x 64 A tile with a TMA load in the swizzled layout as
 // soon as the MMA has released the stage, and the decoders expand only the
 // weight codes.
-template <int A_BITS, int B_BITS, bool A_TMA>
+// F8: the lower-precision contraction mode (4-bit codes of both operands
+// decoded to e4m3, K blocks of 128, kind::f8f6f4 MMAs with K 32).
+template <int A_BITS, int B_BITS, bool A_TMA, bool F8>
 // registers: six warps of one SM sub-partition share its 16K registers
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
     gemm_pair_kernel(const __grid_constant__ PairParams p) {
@@ -87,7 +89,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   static_assert(OS == 6, "the decoder loop is unrolled over six stages");
-  constexpr int QA = A_TMA ? 0 : Fmt<A_BITS>::QP, QB = Fmt<B_BITS>::QP;
+  static_assert(!F8 || (A_BITS == 4 && B_BITS == 4 && !A_TMA), "the FP8 mode takes 4-bit codes of both operands");
+  constexpr int BKE = F8 ? DEC_BK_F8 : BK;                 // K elements per stage
+  constexpr int CHUNK_E = F8 ? 16 : 8;                     // K elements per 16-byte operand chunk
+  constexpr int QA = A_TMA ? 0 : (F8 ? 4 : Fmt<A_BITS>::QP), QB = F8 ? 4 : Fmt<B_BITS>::QP;
   constexpr int ITEMS_A = RM * QA, ITEMS = RM * QA + RN * QB;
   // when the items fill at most half of the decoder threads (weights only, in
   // the fused call) the decoders split into two groups that take alternate K
@@ -148,7 +153,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
     const DecK kc = p.kc;
     // fixed per-thread items: operand row r, 16-byte code part q; the shared
     // address of each of its 16-byte chunks in stage 0 does not change
-    constexpr int CPA = Fmt<A_BITS>::CPP, CPB = Fmt<B_BITS>::CPP;
+    constexpr int CPA = F8 ? 2 : Fmt<A_BITS>::CPP, CPB = F8 ? 2 : Fmt<B_BITS>::CPP;
     constexpr int CPM = CPA > CPB ? CPA : CPB;
     uint32_t sts[IPT][CPM];
     int item_r[IPT], item_q[IPT];
@@ -191,10 +196,19 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
       for (int it = 0; it < IPT; ++it) {
         dst[it] = make_uint4(0u, 0u, 0u, 0u);
         if (item_on[it]) {
-          if (item_a[it]) dst[it] = load_part<A_BITS>(frow[it], kb, item_q[it], p.K);
+          if constexpr (F8) dst[it] = load_part_f8(frow[it], kb, item_q[it], p.K);
+          else if (item_a[it]) dst[it] = load_part<A_BITS>(frow[it], kb, item_q[it], p.K);
           else dst[it] = load_part<B_BITS>(frow[it], kb, item_q[it], p.K);
         }
       }
+    };
+    auto dec_a = [&](const uint4& v, int j) -> uint4 {
+      if constexpr (F8) return decode_chunk_f8(v, j, ta, kc);
+      else return decode_chunk_k<A_BITS>(v, j, ta, lut8, kc);
+    };
+    auto dec_b = [&](const uint4& v, int j) -> uint4 {
+      if constexpr (F8) return decode_chunk_f8(v, j, tb, kc);
+      else return decode_chunk_k<B_BITS>(v, j, tb, lut8, kc);
     };
     // decode one K block (TAIL: the block runs past K and the A chunks beyond
     // it must be zero) into registers, and store decoded chunks into stage S
@@ -206,13 +220,13 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
         if (item_a[it]) {
 #pragma unroll
           for (int j = 0; j < CPA; ++j) {
-            uint4 o = decode_chunk_k<A_BITS>(cur[it], j, ta, lut8, kc);
-            if (TAIL && kb * BK + (item_q[it] * CPA + j) * 8 >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
+            uint4 o = dec_a(cur[it], j);
+            if (TAIL && kb * BKE + (item_q[it] * CPA + j) * CHUNK_E >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
             dec[it][j] = o;
           }
         } else if (item_on[it]) {
 #pragma unroll
-          for (int j = 0; j < CPB; ++j) dec[it][j] = decode_chunk_k<B_BITS>(cur[it], j, tb, lut8, kc);
+          for (int j = 0; j < CPB; ++j) dec[it][j] = dec_b(cur[it], j);
         }
       }
     };
@@ -237,14 +251,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
         if (item_a[it]) {
 #pragma unroll
           for (int j = 0; j < CPA; ++j) {
-            uint4 o = decode_chunk_k<A_BITS>(cur[it], j, ta, lut8, kc);
-            if (TAIL && kb * BK + (item_q[it] * CPA + j) * 8 >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
+            uint4 o = dec_a(cur[it], j);
+            if (TAIL && kb * BKE + (item_q[it] * CPA + j) * CHUNK_E >= p.K) o = make_uint4(0u, 0u, 0u, 0u);
             st_shared_v4(sts[it][j] + so, o);
           }
         } else if (item_on[it]) {
 #pragma unroll
           for (int j = 0; j < CPB; ++j)
-            st_shared_v4(sts[it][j] + so, decode_chunk_k<B_BITS>(cur[it], j, tb, lut8, kc));
+            st_shared_v4(sts[it][j] + so, dec_b(cur[it], j));
         }
       }
     };
@@ -448,8 +462,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
           }
           const bool more = kb + 1 < nkb || i + 1 < my_tiles;
           const uint32_t a_lo = a_lo0 + (uint32_t)s * (uint32_t)(STAGE_BYTES >> 4);
-          const bool rdy1 = tc_kblock64_f16<2>(d_tmem, a_lo, a_lo + (A_TILE >> 4), d_hi, idesc, kb > 0 ? 1u : 0u,
-                                               &op_empty[s], (uint16_t)0x3, &op_full[s1], n1 & 1u, more ? 1u : 0u);
+          const bool rdy1 = tc_kblock_4mma<2, F8>(d_tmem, a_lo, a_lo + (A_TILE >> 4), d_hi, idesc, kb > 0 ? 1u : 0u,
+                                                  &op_empty[s], (uint16_t)0x3, &op_full[s1], n1 & 1u, more ? 1u : 0u);
           s = s1;
           n = n1;
           rdy = rdy1;
@@ -485,10 +499,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(80)
   }
 }
 
-template <int A_BITS, int B_BITS, bool A_TMA>
+template <int A_BITS, int B_BITS, bool A_TMA, bool F8 = false>
 oq_status launch_pair(const PairParams& kp_in, void* stream) {
   PairParams kp = kp_in;
-  auto kern = gemm_pair_kernel<A_BITS, B_BITS, A_TMA>;
+  auto kern = gemm_pair_kernel<A_BITS, B_BITS, A_TMA, F8>;
   const size_t smem = 1024 + (size_t)OS * STAGE_BYTES + EPI_BYTES + 512 + 8 * (2 * OS + 4) + 16;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) {
@@ -499,7 +513,7 @@ oq_status launch_pair(const PairParams& kp_in, void* stream) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   kp.n_tiles = kp.N / PN;
-  kp.nkb = (kp.K + BK - 1) / BK;
+  kp.nkb = (kp.K + (F8 ? DEC_BK_F8 : BK) - 1) / (F8 ? DEC_BK_F8 : BK);
   kp.tiles = ((kp.M + 2 * RM - 1) / (2 * RM)) * (int64_t)kp.n_tiles;
   const int64_t grid = std::min<int64_t>(2 * kp.tiles, (int64_t)(sms & ~1));
   // K-block counters are 32-bit
@@ -559,8 +573,19 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream) {
   kp.K = g.K;
   kp.a_wpr = g.K * g.a_bits / 32;
   kp.b_wpr = g.K * g.b_bits / 32;
-  make_decode_tables(g.a_bits, g.a_levels_host, kp.a_tab);
-  make_decode_tables(g.b_bits, g.b_levels_host, kp.b_tab);
+  if (g.fp8) {
+    // e4m3 bytes of the eight positive levels (codes 8..15) in two words
+    for (int w = 0; w < 2; ++w) {
+      kp.a_tab[w] = kp.b_tab[w] = 0u;
+      for (int b = 0; b < 4; ++b) {
+        kp.a_tab[w] |= (uint32_t)g.a_levels8[8 + 4 * w + b] << (8 * b);
+        kp.b_tab[w] |= (uint32_t)g.b_levels8[8 + 4 * w + b] << (8 * b);
+      }
+    }
+  } else {
+    make_decode_tables(g.a_bits, g.a_levels_host, kp.a_tab);
+    make_decode_tables(g.b_bits, g.b_levels_host, kp.b_tab);
+  }
   kp.kc = make_deck();
   kp.a_lut8 = g.a_levels;
   kp.err = g.err;
@@ -568,6 +593,10 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream) {
   {
     const oq_status st = encode_y_map(&kp.y_map, g.y, g.M, g.N);
     if (st != OQ_OK) return st;
+  }
+  if (g.fp8) {
+    if (g.a_f16 || g.a_bits != 4 || g.b_bits != 4) return OQ_ERR_UNSUPPORTED;
+    return launch_pair<4, 4, false, true>(kp, stream);
   }
   if (g.a_f16) {
     // fp16 A operand fetched by TMA: 16-byte aligned rows of K halves

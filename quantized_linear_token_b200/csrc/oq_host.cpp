@@ -324,6 +324,54 @@ double f16_bits_to_f64(uint16_t h) {
   return (h & 0x8000) ? -v : v;
 }
 
+// e4m3 (4 exponent bits, bias 7, 3 mantissa bits, largest finite 448) for
+// the lower-precision contraction mode: round to nearest, ties to even,
+// normal range only (levels are scaled into [2^-6, 448)).
+uint8_t f64_to_e4m3_bits(double v) {
+  const uint8_t sign = v < 0 ? 0x80 : 0;
+  const double a = std::fabs(v);
+  if (a == 0.0) return sign;
+  int e;
+  const double m = std::frexp(a, &e);    // a = m * 2^e, m in [0.5, 1)
+  int E = e - 1 + 7;
+  double r = std::nearbyint(m * 16.0);   // 4 significant bits, in [8, 16]
+  if (r >= 16.0) {
+    r = 8.0;
+    ++E;
+  }
+  if (E <= 0 || E > 15 || (E == 15 && r == 15.0)) return sign;   // not produced for our levels
+  return (uint8_t)(sign | (E << 3) | ((int)r - 8));
+}
+
+double e4m3_bits_to_f64(uint8_t b) {
+  const int E = (b >> 3) & 15, f = b & 7;
+  const double v = (E == 0) ? f / 8.0 * std::ldexp(1.0, -6) : (1.0 + f / 8.0) * std::ldexp(1.0, E - 7);
+  return (b & 0x80) ? -v : v;
+}
+
+// the scale that brings the positive levels closest to e4m3 values (largest
+// relative error over the levels), searched in [8, 16) / max level so that the
+// largest level lands in [8, 16)
+double choose_fp8_scale(const oq_codebook& cb, double* worst) {
+  const int L = 1 << cb.bits;
+  const double base = 8.0 / cb.levels[L - 1];
+  double best = base, best_err = 1e30;
+  for (int j = 0; j < 4096; ++j) {
+    const double alpha = base * (1.0 + j / 4096.0);
+    double err = 0.0;
+    for (int i = L / 2; i < L; ++i) {
+      const double v = alpha * cb.levels[i];
+      err = std::max(err, std::fabs(e4m3_bits_to_f64(f64_to_e4m3_bits(v)) - v) / v);
+    }
+    if (err < best_err) {
+      best_err = err;
+      best = alpha;
+    }
+  }
+  if (worst) *worst = best_err;
+  return best;
+}
+
 double choose_fp16_scale(const oq_codebook& cb) {
   const int L = 1 << cb.bits;
   const double base = std::sqrt((double)cb.d);

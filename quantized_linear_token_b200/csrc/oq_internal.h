@@ -26,6 +26,10 @@ struct oq_bin_table {
 struct oq_layer {
   int d_in, d_out, h, k, log_h, a_bits, w_bits, flags;
   bool int4_only;                     // OQ_FLAG_WEIGHT_ONLY_INT4: AdaLN path (no rotation or codebooks)
+  bool fp8;                           // OQ_FLAG_FP8_CONTRACTION: levels decoded to e4m3, kind::f8f6f4 MMAs
+  double a8_scale, w8_scale;          // e4m3 decode scale per codebook (fp8 mode)
+  double a8_err, w8_err;              // their worst relative level rounding
+  uint8_t lv8_a[16], lv8_w[16];       // e4m3 bytes of the scaled levels (fp8 mode, 4-bit)
   uint64_t seed;
   int device;
   oq_codebook cb_a, cb_w;
@@ -54,6 +58,9 @@ oq_status get_codebook(int d, int bits, int flags, oq_codebook* out);
 uint16_t f64_to_f16_bits(double v);
 double f16_bits_to_f64(uint16_t h);
 double choose_fp16_scale(const oq_codebook& cb);
+uint8_t f64_to_e4m3_bits(double v);
+double e4m3_bits_to_f64(uint8_t b);
+double choose_fp8_scale(const oq_codebook& cb, double* worst);
 // threshold search table of a codebook (host copies; words interleaved TK, payload)
 constexpr int OQ_MAX_BINS = 4096;
 oq_status build_bin_table(const oq_codebook& cb, int d, int h, const uint16_t* lv16, float* kscale, int* b0, int* nb,
@@ -86,6 +93,9 @@ struct GemmArgs {
   const uint32_t* a_codes;   // [M, K*a_bits/32]
   const uint16_t* a_f16;     // or: fp16 levels of A [M, K] (fused call), null otherwise
   bool a_bf16;               // a_f16 holds bf16 values (INT4 weight-only layer; b levels are bf16 too)
+  bool fp8;                  // decode both operands to e4m3 and contract with kind::f8f6f4 (4-bit codes)
+  const uint8_t* a_levels8;  // host e4m3 level bytes (fp8 mode)
+  const uint8_t* b_levels8;
   const uint32_t* b_codes;   // [N, K*b_bits/32]
   const float* a_scale;      // [M] per-row magnitude s (null: 1)
   const float* b_scale;      // [N] per-row magnitude r

@@ -274,6 +274,52 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint4& v) {
 // before the MMAs and its answer is only read after them, so the ~200-cycle
 // latency of a barrier check overlaps the MMA issue.  `accumulate` applies to
 // the first MMA; the other three always accumulate.
+// F8: the same with kind::f8f6f4 MMAs (K 32 e4m3 per MMA: 128 K per call;
+// the descriptors advance by the same 32 bytes per MMA).
+#define OQ_KBLOCK_ASM(CGS, KIND, WAITSCOPE, COMMIT)                                                             \
+  "{\n\t.reg .pred pa, pt, pp, pn;\n\t.reg .b64 da, db;\n\t.reg .b32 al, bl;\n\t"                                \
+  "setp.ne.b32 pa, %5, 0;\n\tsetp.eq.b32 pt, 0, 0;\n\tsetp.ne.b32 pp, %10, 0;\n\t"                                  \
+  "setp.ne.b32 pn, 0, 0;\n\t"                                                                                    \
+  "@pp mbarrier.test_wait.parity.acquire." WAITSCOPE ".shared::cta.b64 pn, [%8], %9;\n\t"                         \
+  "mov.b64 da, {%2, %4};\n\tmov.b64 db, {%3, %4};\n\t"                                                          \
+  "tcgen05.mma.cta_group::" CGS ".kind::" KIND " [%1], da, db, %6, pa;\n\t"                                      \
+  "add.u32 al, %2, 2;\n\tadd.u32 bl, %3, 2;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"              \
+  "tcgen05.mma.cta_group::" CGS ".kind::" KIND " [%1], da, db, %6, pt;\n\t"                                      \
+  "add.u32 al, %2, 4;\n\tadd.u32 bl, %3, 4;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"              \
+  "tcgen05.mma.cta_group::" CGS ".kind::" KIND " [%1], da, db, %6, pt;\n\t"                                      \
+  "add.u32 al, %2, 6;\n\tadd.u32 bl, %3, 6;\n\tmov.b64 da, {al, %4};\n\tmov.b64 db, {bl, %4};\n\t"              \
+  "tcgen05.mma.cta_group::" CGS ".kind::" KIND " [%1], da, db, %6, pt;\n\t" COMMIT                              \
+  "selp.u32 %0, 1, 0, pn;\n\t}"
+
+template <int CG, bool F8>
+__device__ __forceinline__ bool tc_kblock_4mma(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t d_hi,
+                                               uint32_t idesc, uint32_t accumulate, uint64_t* bar, uint16_t mask,
+                                               uint64_t* next_bar, uint32_t next_parity, uint32_t probe) {
+  uint32_t ready;
+#define OQ_KBLOCK_ARGS                                                                                        \
+  : "=r"(ready)                                                                                               \
+  : "r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(accumulate), "r"(idesc), "r"(smem_u32(bar)),              \
+    "r"(smem_u32(next_bar)), "r"(next_parity), "r"(probe), "h"(mask)                                            \
+  : "memory"
+  if constexpr (CG == 2 && F8) {
+    asm volatile(OQ_KBLOCK_ASM("2", "f8f6f4", "cluster",
+                               "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::"
+                               "cluster.b64 [%7], %11;\n\t") OQ_KBLOCK_ARGS);
+  } else if constexpr (CG == 2) {
+    asm volatile(OQ_KBLOCK_ASM("2", "f16", "cluster",
+                               "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::"
+                               "cluster.b64 [%7], %11;\n\t") OQ_KBLOCK_ARGS);
+  } else {
+    static_assert(!F8, "one-CTA FP8 K blocks are not used");
+    asm volatile(OQ_KBLOCK_ASM("1", "f16", "cta",
+                               "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t")
+                     OQ_KBLOCK_ARGS);
+  }
+#undef OQ_KBLOCK_ARGS
+  return ready != 0;
+}
+#undef OQ_KBLOCK_ASM
+
 template <int CG>
 __device__ __forceinline__ bool tc_kblock64_f16(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t d_hi,
                                                 uint32_t idesc, uint32_t accumulate, uint64_t* bar, uint16_t mask,

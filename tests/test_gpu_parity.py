@@ -226,6 +226,43 @@ def test_int4_weight_only_layer(env, T, d_in, d_out, w_bf16):
             call()
 
 
+def test_fp8_contraction_mode(env):
+    # the lower-precision contraction variant (a separate mode): the same codes
+    # and norms as the default mode, y from e4m3 levels on kind::f8f6f4 MMAs;
+    # its error against the oracle's exact-level contraction is measured in
+    # the bound-relative metric of the default mode and must stay within the
+    # e4m3 rounding of the levels (a few 1e-2), far from the default 1e-3 bound
+    torch, B = env
+    d_in, d_out, T = 3072, 512, 300
+    x_np, Wm = _inputs("dit_image", d_in, d_out, T)
+    Wm = np.ascontiguousarray(Wm[:d_out])
+    x_t, x64 = _x_tensor(torch, x_np)
+    W_t = torch.from_numpy(Wm).cuda()
+    ref = B.oq_layer_create(d_in, d_out, 0, 4, 4)
+    f8 = B.oq_layer_create(d_in, d_out, 0, 4, 4, B.OQ_FLAG_FP8_CONTRACTION)
+    Wc, r = B.oq_weight_prepare(ref, W_t)
+    Wc8, r8 = B.oq_weight_prepare(f8, W_t)
+    codes, s = B.oq_rotate_quantize(ref, x_t)
+    codes8, s8 = B.oq_rotate_quantize(f8, x_t)
+    y8 = B.oq_linear(f8, codes8, s8, Wc8, r8)
+    y8f = B.oq_linear_fused(f8, x_t, Wc8, r8)
+    torch.cuda.synchronize()
+    B.oq_poll_error(f8)
+    np.testing.assert_array_equal(to_numpy_u32(codes8), to_numpy_u32(codes))
+    np.testing.assert_array_equal(to_numpy_u32(Wc8), to_numpy_u32(Wc))
+    np.testing.assert_array_equal(y8f.cpu().numpy(), y8.cpu().numpy())
+    cb = O.lloyd_max(d_in, 4)
+    y_or, bound = O.linear_from_codes(O.unpack_codes(to_numpy_u32(codes), 4, d_in), s.cpu().numpy().astype(np.float64),
+                                      O.unpack_codes(to_numpy_u32(Wc), 4, d_in), r.cpu().numpy().astype(np.float64),
+                                      cb.levels, cb.levels)
+    rel = np.abs(y8.cpu().numpy().astype(np.float64) - y_or) / np.where(bound > 0, bound, 1.0)
+    yn = np.linalg.norm(y8.cpu().numpy() - y_or) / np.linalg.norm(y_or)
+    print(f"fp8 mode: max bound-relative error {rel.max():.4f}, relative l2 error {yn:.4f}")
+    assert float(rel.max()) < 0.05 and yn < 0.05
+    with pytest.raises(B.OrbitQuantError):
+        B.oq_rotate_quantize_levels(f8, x_t)
+
+
 def test_degenerate_tokens(env):
     # a zero token (s = 0, every code L/2 - 1, y = 0) and tokens with very
     # small and very large norms
