@@ -215,9 +215,16 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
  * kernel writes the fp16 levels of the activation codes, which the contraction
  * reads with TMA (only the weight codes are decoded in the contraction);
  * otherwise the packed codes pass through the workspace.  `workspace` is
- * caller-owned device scratch of at least
- * oq_linear_fused_workspace_size(layer, T) bytes (the A operand and the
- * norms), 256-byte aligned; it may be reused between calls on one stream.
+ * caller-owned device scratch, 256-byte aligned, that may be reused between
+ * calls on one stream.  oq_linear_fused_workspace_size(layer, T) gives the
+ * bytes of the fastest route: the A operand and the norms, and from 1024
+ * tokens on (bf16 x, d_out % 256 == 0) also 2 d_out d_in bytes for the
+ * weights' fp16 levels, which are then decoded once per call
+ * (oq_weight_levels) and contracted with oq_linear_decoded's kernel.  A
+ * smaller workspace that still holds the A operand and the norms is accepted
+ * and decodes the weights inside the contraction instead; the y values are
+ * the same up to fp32 summation order.  Errors: OQ_ERR_INVALID_ARG when the
+ * workspace is below that least size.
  */
 size_t oq_linear_fused_workspace_size(const oq_layer* layer, int64_t T);
 oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
@@ -244,9 +251,25 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  *   y[t, o] = s[t] r[o] / (a_scale w_scale) sum_i a16[t, i] fp16(w_scale C_w[Wcodes[o, i]])
  *   Needs d_out % 256 == 0 (else OQ_ERR_UNSUPPORTED); y 16-byte aligned.
  *
+ * oq_weight_levels -- the weights' operand as fp16 levels, decoded once
+ * (gecl notes Limitation 3: the centroid lookup of every code):
+ *   w16[o, i] = fp16(w_scale * C_w[Wcodes[o, i]])
+ *   Wcodes  device [d_out, d_in*w_bits/32] from oq_weight_prepare, 16-byte aligned.
+ *   w16     device [d_out, d_in] uint16 (fp16 bits), 16-byte aligned, caller-owned.
+ *   Reads the codes once and writes 2 d_out d_in bytes.
+ *
+ * oq_linear_decoded -- the contraction of the two fp16 level operands, both
+ * read by TMA (no decoding in the contraction; the route oq_linear_fused takes
+ * for large batches):
+ *   y[t, o] = s[t] r[o] / (a_scale w_scale) sum_i a16[t, i] w16[o, i]
+ *   a16, s from oq_rotate_quantize_levels; w16 from oq_weight_levels; r from
+ *   oq_weight_prepare (16-byte aligned); y device [T, d_out] fp32, 16-byte
+ *   aligned.  Needs d_out % 256 == 0 (else OQ_ERR_UNSUPPORTED).
+ *
  * oq_rotate_quantize_levels followed by oq_linear_levels gives exactly the y
- * of oq_linear_fused (and of oq_rotate_quantize + oq_linear, up to summation
- * order for batches of at most 256 tokens).
+ * of oq_linear_fused for T < 1024, and followed by oq_weight_levels +
+ * oq_linear_decoded exactly its y for T >= 1024 with the full workspace (and
+ * the y of oq_rotate_quantize + oq_linear up to fp32 summation order).
  *
  * Small batches (T <= 256, d_out % 128 == 0) take a kernel whose M dimension
  * is 128 weight rows and whose N is the padded batch, with the K range split
@@ -259,6 +282,9 @@ oq_status oq_rotate_quantize_levels(const oq_layer* layer, const void* x, int32_
                                     uint16_t* a16, float* s, void* stream);
 oq_status oq_linear_levels(const oq_layer* layer, const uint16_t* a16, const float* s, int64_t T,
                            const uint32_t* Wcodes, const float* r, float* y, void* stream);
+oq_status oq_weight_levels(const oq_layer* layer, const uint32_t* Wcodes, uint16_t* w16, void* stream);
+oq_status oq_linear_decoded(const oq_layer* layer, const uint16_t* a16, const float* s, int64_t T,
+                            const uint16_t* w16, const float* r, float* y, void* stream);
 
 /*
  * oq_linear_fused_static -- the same computation as oq_linear_fused for
@@ -274,10 +300,11 @@ oq_status oq_linear_levels(const oq_layer* layer, const uint16_t* a16, const flo
  *   that device current); make that first call before any stream capture.
  *   Every call shares the array: calls that overlap on the GPU (different
  *   streams or host threads) race and give wrong results.
- *   Arguments as for oq_linear_fused.  Errors: OQ_ERR_INVALID_ARG when the
- *   batch needs more scratch than the array holds, i.e. when
- *   oq_linear_fused_workspace_size(layer, T) > OQ_STATIC_SCRATCH_BYTES
- *   (at d_in = 3072 with d_out % 256 == 0 about 2700 tokens).
+ *   Arguments as for oq_linear_fused; the array serves as its least
+ *   workspace (A operand and norms), so weights are decoded inside the
+ *   contraction.  Errors: OQ_ERR_INVALID_ARG when the batch needs more
+ *   scratch than the array holds (at d_in = 3072 with d_out % 256 == 0 about
+ *   2700 tokens).
  */
 #define OQ_STATIC_SCRATCH_BYTES (16u << 20)
 oq_status oq_linear_fused_static(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,

@@ -28,7 +28,8 @@ OQ_FLAG_FP8_CONTRACTION = 8
 EXPORTS = (
     "oq_codebook_build", "oq_rotation_build", "oq_layer_create", "oq_layer_destroy", "oq_layer_get_info", "oq_layer_get_perm",
     "oq_rotate_quantize", "oq_weight_prepare", "oq_linear", "oq_linear_fused_workspace_size",
-    "oq_linear_fused", "oq_rotate_quantize_levels", "oq_linear_levels", "oq_linear_fused_static",
+    "oq_linear_fused", "oq_rotate_quantize_levels", "oq_linear_levels", "oq_weight_levels", "oq_linear_decoded",
+    "oq_linear_fused_static",
     "oq_poll_error", "oq_last_error", "oq_status_string",
 )
 
@@ -84,6 +85,8 @@ def load_library(path: str = LIB_PATH):
         "oq_linear_fused": (i32, [vp, vp, i32, i64, vp, vp, vp, vp, sz, vp]),
         "oq_rotate_quantize_levels": (i32, [vp, vp, i32, i64, vp, vp, vp]),
         "oq_linear_levels": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
+        "oq_weight_levels": (i32, [vp, vp, vp, vp]),
+        "oq_linear_decoded": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
         "oq_poll_error": (i32, [vp]),
         "oq_last_error": (ctypes.c_char_p, []),
@@ -274,6 +277,29 @@ def oq_linear_levels(layer: Layer, a16, s, Wcodes, r, y=None):
         y = torch.empty((T, layer.d_out), dtype=torch.float32, device=a16.device)
     _check(load_library().oq_linear_levels(layer.handle, _dev(a16, "a16"), _dev(s, "s"), T, _dev(Wcodes, "Wcodes"),
                                            _dev(r, "r"), _dev(y, "y"), _stream(a16)), "oq_linear_levels")
+    return y
+
+
+def oq_weight_levels(layer: Layer, Wcodes, w16=None):
+    """Wcodes [d_out, d_in*w_bits/32] -> w16 [d_out, d_in] fp16 levels of the
+    weight codes (decoded once; the large-batch route's B operand)."""
+    torch = _torch()
+    if w16 is None:
+        w16 = torch.empty((layer.d_out, layer.d_in), dtype=torch.float16, device=Wcodes.device)
+    _check(load_library().oq_weight_levels(layer.handle, _dev(Wcodes, "Wcodes"), _dev(w16, "w16"), _stream(Wcodes)),
+           "oq_weight_levels")
+    return w16
+
+
+def oq_linear_decoded(layer: Layer, a16, s, w16, r, y=None):
+    """(a16, s, w16, r) -> y [T, d_out] fp32: the contraction of two fp16 level
+    operands, both read by TMA."""
+    torch = _torch()
+    T = a16.shape[0]
+    if y is None:
+        y = torch.empty((T, layer.d_out), dtype=torch.float32, device=a16.device)
+    _check(load_library().oq_linear_decoded(layer.handle, _dev(a16, "a16"), _dev(s, "s"), T, _dev(w16, "w16"),
+                                            _dev(r, "r"), _dev(y, "y"), _stream(a16)), "oq_linear_decoded")
     return y
 
 

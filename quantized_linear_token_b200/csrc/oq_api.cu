@@ -383,11 +383,29 @@ static size_t fused_codes_bytes(const oq_layer* L, int64_t T) {
 
 static size_t fused_f16_bytes(const oq_layer* L, int64_t T) { return (size_t)T * (size_t)L->d_in * 2; }
 
-size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
+static size_t round256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+// Large batches on the fp16-level route decode the weight codes once per call
+// into fp16 levels held in the workspace, and both contraction operands come
+// by TMA (oq_gemm_w16.cu); this needs 2 d_out d_in more bytes.
+static bool fused_w16_route(const oq_layer* L, int32_t x_dtype, int64_t T) {
+  return fused_f16_route(L, x_dtype) && T >= W16_MIN_T;
+}
+
+static size_t fused_w16_bytes(const oq_layer* L) { return round256((size_t)L->d_out * (size_t)L->d_in * 2); }
+
+// the least workspace oq_linear_fused accepts (without the decoded weights)
+static size_t min_workspace(const oq_layer* L, int64_t T) {
   if (!L || T <= 0 || L->int4_only) return 0;
   size_t a = fused_codes_bytes(L, T);
   if (L->d_out % 256 == 0) a = std::max(a, fused_f16_bytes(L, T));
-  return ((a + 255) & ~(size_t)255) + (size_t)T * 4;
+  return round256(a) + (size_t)T * 4;
+}
+
+size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
+  const size_t base = min_workspace(L, T);
+  if (base && fused_w16_route(L, OQ_DTYPE_BF16, T)) return round256(base) + fused_w16_bytes(L);
+  return base;
 }
 
 static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint16_t* a16, float* s,
@@ -441,6 +459,49 @@ oq_status oq_linear_levels(const oq_layer* L, const uint16_t* a16, const float* 
   return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
 }
 
+oq_status oq_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* w16, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_weight_levels: layer is null");
+  if (L->int4_only) return not_for_int4(L, "oq_weight_levels");
+  if (L->fp8) return fail(OQ_ERR_UNSUPPORTED, "oq_weight_levels: the fp16-level route is not used in the FP8 mode");
+  if (!Wcodes || !w16 || !aligned(Wcodes, 16) || !aligned(w16, 16))
+    return fail(OQ_ERR_INVALID_ARG, "oq_weight_levels: Wcodes / w16 must be 16-byte aligned device pointers");
+  const oq_status st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
+  return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_weight_levels: unsupported shape") : st;
+}
+
+static oq_status linear_w16(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
+                            const float* r, float* y, void* stream) {
+  GemmArgs g{};
+  g.a_f16 = a16;
+  g.b_f16 = w16;
+  g.a_scale = s;
+  g.b_scale = r;
+  g.out_scale = (float)(1.0 / (L->a_scale * L->w_scale));
+  g.y = y;
+  g.M = T;
+  g.N = L->d_out;
+  g.K = L->d_in;
+  g.a_bits = L->a_bits;
+  g.b_bits = L->w_bits;
+  g.err = L->d_error;
+  const oq_status st = gemm_w16_launch(g, stream);
+  return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_decoded: unsupported shape") : st;
+}
+
+oq_status oq_linear_decoded(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
+                            const float* r, float* y, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_decoded: layer is null");
+  if (L->int4_only) return not_for_int4(L, "oq_linear_decoded");
+  if (L->fp8) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_decoded: the fp16-level route is not used in the FP8 mode");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_decoded: T < 0");
+  if (T == 0) return OQ_OK;
+  if (!a16 || !s || !w16 || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear_decoded: null pointer");
+  if (!aligned(a16, 16) || !aligned(w16, 16) || !aligned(y, 16) || !aligned(s, 4) || !aligned(r, 16))
+    return fail(OQ_ERR_INVALID_ARG, "oq_linear_decoded: misaligned pointer");
+  if (L->d_out % 256 != 0) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_decoded: needs d_out % 256 == 0");
+  return linear_w16(L, a16, s, T, w16, r, y, stream);
+}
+
 // y = x (q r)^T for the INT4 weight-only layer: bf16 x straight into the
 // small-batch kernel as its token operand, in launches of up to 256 tokens
 static oq_status int4_linear(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
@@ -483,14 +544,22 @@ oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int
   if (!Wcodes || !r || !y || !workspace) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: null pointer");
   if (!aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(r, 16) || !aligned(workspace, 256))
     return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: misaligned pointer (workspace needs 256 bytes)");
-  if (workspace_bytes < oq_linear_fused_workspace_size(L, T))
-    return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
+  const size_t need = min_workspace(L, T);
+  if (workspace_bytes < need) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   if (fused_f16_route(L, x_dtype)) {
     uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
-    float* s = reinterpret_cast<float*>(ws + ((fused_f16_bytes(L, T) + 255) & ~(size_t)255));
+    float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
     st = rq_levels(L, x, x_dtype, T, a16, s, stream);
     if (st != OQ_OK) return st;
+    // large batches with room for the decoded weights: decode them once, then
+    // contract two fp16 operands; otherwise decode weights inside the contraction
+    if (fused_w16_route(L, x_dtype, T) && workspace_bytes >= round256(need) + fused_w16_bytes(L)) {
+      uint16_t* w16 = reinterpret_cast<uint16_t*>(ws + round256(need));
+      st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
+      if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_fused: unsupported shape") : st;
+      return linear_w16(L, a16, s, T, w16, r, y, stream);
+    }
     return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
   }
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws);
@@ -516,3 +585,7 @@ oq_status oq_poll_error(const oq_layer* L) {
 }
 
 }  // extern "C"
+
+namespace oq {
+size_t fused_min_workspace(const oq_layer* L, int64_t T) { return min_workspace(L, T); }
+}  // namespace oq

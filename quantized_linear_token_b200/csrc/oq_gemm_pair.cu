@@ -537,24 +537,6 @@ oq_status launch_pair_b(const PairParams& kp, int b_bits, void* stream) {
   }
 }
 
-oq_status encode_y_map(CUtensorMap* map, float* y, int64_t M, int N) {
-  EncodeTiledFn fn = nullptr;
-  const oq_status st = tmap_encode_fn(&fn);
-  if (st != OQ_OK) return st;
-  const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
-  const cuuint32_t box[2] = {32, 32};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    set_error("cuTensorMapEncodeTiled failed for y (code " + std::to_string((int)r) + ")");
-    return OQ_ERR_CUDA;
-  }
-  return OQ_OK;
-}
-
 }  // namespace
 
 oq_status gemm_pair_launch(const GemmArgs& g, void* stream) {

@@ -97,6 +97,7 @@ struct GemmArgs {
   const uint8_t* a_levels8;  // host e4m3 level bytes (fp8 mode)
   const uint8_t* b_levels8;
   const uint32_t* b_codes;   // [N, K*b_bits/32]
+  const uint16_t* b_f16;     // or: fp16 levels of B [N, K] (decode-then-contract route), null otherwise
   const float* a_scale;      // [M] per-row magnitude s (null: 1)
   const float* b_scale;      // [N] per-row magnitude r
   const uint16_t* a_levels;       // device fp16 bits, 2^a_bits (8-bit table)
@@ -120,6 +121,16 @@ oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream);
 // scale max|w| / 7 and 4-bit codes of q in [-7, 7] (q >= 0 -> q + 8, else q + 7)
 oq_status rtn4_prepare_launch(const void* W, int w_dtype, int rows, int d, uint32_t* codes, float* scale,
                               void* stream);
+// decode-then-contract route (oq_gemm_w16.cu): packed code rows [rows, K] ->
+// fp16 levels [rows, K] (K % 32 == 0), and the CTA-pair contraction of two
+// fp16 level operands (g.a_f16, g.b_f16; N % 256 == 0, K % 8 == 0)
+oq_status levels_launch(const uint32_t* codes, int64_t rows, int K, int bits, const uint16_t* levels_host,
+                        const uint16_t* levels_dev, uint16_t* out, void* stream);
+oq_status gemm_w16_launch(const GemmArgs& g, void* stream);
+// the fused call decodes the weights once per call from this many tokens on
+constexpr int64_t W16_MIN_T = 1024;
+// the least workspace oq_linear_fused accepts (oq_api.cu)
+size_t fused_min_workspace(const oq_layer* L, int64_t T);
 // prmt decode tables of a codebook's fp16 levels (oq_gemm.cu)
 void make_decode_tables(int bits, const uint16_t* levels, uint32_t* t);
 

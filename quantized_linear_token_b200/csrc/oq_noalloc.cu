@@ -74,7 +74,9 @@ extern "C" oq_status oq_linear_fused_static(const oq_layer* layer, const void* x
     return OQ_ERR_INVALID_ARG;
   }
   if (T == 0) return OQ_OK;
-  const size_t need = oq_linear_fused_workspace_size(layer, T);
+  // the static array holds the fused call's least workspace (large batches
+  // then decode weights inside the contraction)
+  const size_t need = oq::fused_min_workspace(layer, T);
   if (need > (size_t)OQ_STATIC_SCRATCH_BYTES) {
     oq::set_error("oq_linear_fused_static: " + std::to_string(T) + " tokens need " + std::to_string(need) +
                   " bytes of scratch, more than the " + std::to_string((size_t)OQ_STATIC_SCRATCH_BYTES) +

@@ -93,6 +93,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst_smem, const void* tmap, in
       : "memory");
 }
 
+// The same load issued by either CTA of a pair whose MMAs run with
+// cta_group::2: the box lands in the issuing CTA's shared memory and its bytes
+// are counted on the barrier at `bar_cluster`, a shared::cluster address that
+// may lie in the peer CTA (no multicast)
+__device__ __forceinline__ void tma_load_2d_pair(void* dst_smem, const void* tmap, int32_t x, int32_t y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst_smem)),
+      "l"(tmap), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
 // 2-D tiled TMA store of a shared-memory box to (x, y) of a tensor map; boxes
 // reaching past the tensor's bounds are clipped.  Tracked as a bulk group.
 __device__ __forceinline__ void tma_store_2d(const void* tmap, int32_t x, int32_t y, const void* src_smem) {

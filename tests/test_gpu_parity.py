@@ -115,6 +115,24 @@ def _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bi
     _same_y(y2.cpu().numpy(), y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in,
             T_small=codes_np.shape[0] <= SKINNY_MAX_T and Wc_np.shape[0] % 128 == 0, label=label + " levels",
             rows=y_rows)
+    _check_decoded(env, layer, a16, s2, Wc, r, codes_np, s_np, y_np, d_in, Wc_np, r_np, cb_a, cb_w, y_rows, label)
+
+
+def _check_decoded(env, layer, a16, s, Wc, r, codes_np, s_np, y_np, d_in, Wc_np, r_np, cb_a, cb_w, y_rows, label):
+    """The decode-then-contract route: the weights' fp16 levels hold exactly
+    fp16(w_scale C_w[code]), and the contraction of the two fp16 operands gives
+    the codes route's y (the same MMAs in the same order on CTA pairs; to fp32
+    summation order against the small-batch kernel)."""
+    torch, B = env
+    w16 = B.oq_weight_levels(layer, Wc)
+    y4 = B.oq_linear_decoded(layer, a16, s, w16, r)
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+    c = O.unpack_codes(Wc_np, cb_w.bits, d_in)
+    want = (layer.w_scale * np.asarray(cb_w.levels, dtype=np.float64))[c].astype(np.float16).view(np.uint16)
+    np.testing.assert_array_equal(w16.cpu().numpy().view(np.uint16), want)
+    _same_y(y4.cpu().numpy(), y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in,
+            T_small=codes_np.shape[0] <= SKINNY_MAX_T, label=label + " decoded", rows=y_rows)
 
 
 CASES = [
@@ -261,6 +279,50 @@ def test_fp8_contraction_mode(env):
     assert float(rel.max()) < 0.05 and yn < 0.05
     with pytest.raises(B.OrbitQuantError):
         B.oq_rotate_quantize_levels(f8, x_t)
+
+
+DECODED = [
+    # d_in, d_out, a, w, T: ragged M and K tails, every weight width, T past
+    # the fused call's switch to the decoded-weight route
+    (96, 256, 4, 2, 1100),       # K = 96: a half K block of 64
+    (640, 512, 3, 3, 1024),
+    (3072, 768, 4, 4, 1300),
+    (13824, 256, 8, 4, 1030),
+]
+
+
+@pytest.mark.parametrize("d_in,d_out,a_bits,w_bits,T", DECODED)
+def test_decoded_weight_route(env, d_in, d_out, a_bits, w_bits, T):
+    # the fused call from 1024 tokens on with its full workspace (weights
+    # decoded once, both operands by TMA) against the stage calls, the codes
+    # route and the oracle; with the least workspace it keeps decoding weights
+    # inside the contraction
+    torch, B = env
+    x_np = W.custom_activations(T, d_in, seed=d_in + T)
+    Wm = W.custom_weights(d_out, d_in, seed=d_out + 3)
+    rows = np.unique(np.concatenate([np.arange(8), np.arange(T - 8, T),
+                                     np.random.default_rng(T).choice(T, 48, replace=False)]))
+    _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, w_rows=np.arange(0, d_out, 5), y_rows=rows,
+               label=f"decoded {d_in}x{d_out} T={T}")
+    layer = B.oq_layer_create(d_in, d_out, 0, a_bits, w_bits, 0)
+    x_t, _ = _x_tensor(torch, x_np)
+    Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(Wm).cuda())
+    full = B.oq_linear_fused_workspace_size(layer, T)
+    assert full >= d_out * d_in * 2 + T * d_in * 2
+    y_full = B.oq_linear_fused(layer, x_t, Wc, r)
+    a16, s = B.oq_rotate_quantize_levels(layer, x_t)
+    y_stage = B.oq_linear_decoded(layer, a16, s, B.oq_weight_levels(layer, Wc), r)
+    least = full - ((d_out * d_in * 2 + 255) // 256) * 256
+    ws = torch.empty((least,), dtype=torch.uint8, device="cuda")
+    y_least = B.oq_linear_fused(layer, x_t, Wc, r, workspace=ws)
+    y_lv = B.oq_linear_levels(layer, a16, s, Wc, r)
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+    np.testing.assert_array_equal(y_full.cpu().numpy(), y_stage.cpu().numpy())
+    np.testing.assert_array_equal(y_least.cpu().numpy(), y_lv.cpu().numpy())
+    np.testing.assert_array_equal(y_full.cpu().numpy(), y_lv.cpu().numpy())
+    with pytest.raises(B.OrbitQuantError):
+        B.oq_linear_fused(layer, x_t, Wc, r, workspace=ws[:least - 256])
 
 
 def test_degenerate_tokens(env):
