@@ -44,8 +44,8 @@ def parse_args():
     ap.add_argument("--workload", default="dit_image")
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's token count (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--route", choices=["levels", "codes"], default="levels",
-                    help="hot-path route of the timed step (the other one is reported beside it)")
+    ap.add_argument("--route", choices=["levels", "levels_wdec", "codes"], default="levels",
+                    help="hot-path route of the timed step (the others are reported beside it)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -233,32 +233,38 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     a16 = torch.empty((T, d), dtype=torch.float16, device=dev)
+    w16 = torch.empty((dout, d), dtype=torch.float16, device=dev)
 
-    # the two routes of the hot path (both give the same y):
-    #   levels: oq_rotate_quantize_levels -> oq_linear_levels, the two stages of
-    #           oq_linear_fused (activation codes leave K1 as fp16 levels that
-    #           the contraction reads by TMA; only weight codes are decoded)
-    #   codes:  oq_rotate_quantize -> oq_linear (packed codes between them)
-    def stage1(route):
-        if route == "levels":
-            B.oq_rotate_quantize_levels(layer, x, a16, s)
-        else:
-            B.oq_rotate_quantize(layer, x, codes, s)
-
-    def stage2(route):
-        if route == "levels":
-            B.oq_linear_levels(layer, a16, s, Wc, r, y)
-        else:
-            B.oq_linear(layer, codes, s, Wc, r, y)
+    # the routes of the hot path (all give the same y):
+    #   levels:      the stages of oq_linear_fused at this batch size.  The
+    #                activation codes leave K1 as fp16 levels; from W16_MIN_T
+    #                tokens on the weight codes are decoded once into fp16
+    #                levels and both operands reach the MMAs by TMA
+    #                (oq_weight_levels + oq_linear_decoded), below it the
+    #                contraction decodes the weight codes (oq_linear_levels).
+    #   levels_wdec: oq_rotate_quantize_levels -> oq_linear_levels at any size
+    #   codes:       oq_rotate_quantize -> oq_linear (packed codes between them)
+    decoded = T >= B.W16_MIN_T and dout % 256 == 0
+    stages = {
+        "levels": [("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s))]
+        + ([("wlevels", lambda: B.oq_weight_levels(layer, Wc, w16)),
+            ("gemm", lambda: B.oq_linear_decoded(layer, a16, s, w16, r, y))] if decoded else
+           [("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]),
+        "levels_wdec": [("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s)),
+                        ("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))],
+        "codes": [("rq", lambda: B.oq_rotate_quantize(layer, x, codes, s)),
+                  ("gemm", lambda: B.oq_linear(layer, codes, s, Wc, r, y))],
+    }
 
     def timed(route, K, warmup, sample_clocks=False):
+        st = stages[route]
         for _ in range(warmup):
             flush.zero_()
-            stage1(route)
-            stage2(route)
+            for _, fn in st:
+                fn()
         torch.cuda.synchronize()
         B.oq_poll_error(layer)
-        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(st) + 1)] for _ in range(K)]
         clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) \
             if (rank == 0 and sample_clocks) else None
         if clocks:
@@ -271,27 +277,25 @@ def run_ours(args):
         for i in range(K):
             flush.zero_()                              # L2 flushed, outside the events
             ev[i][0].record(stream)
-            stage1(route)
-            ev[i][1].record(stream)
-            stage2(route)
-            ev[i][2].record(stream)
+            for j, (_, fn) in enumerate(st):
+                fn()
+                ev[i][j + 1].record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         wall = time.perf_counter() - wall0
         clk = clocks.stop() if clocks else None
-        t1 = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-        t2 = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+        per = {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)] for j, (name, _) in enumerate(st)}
         B.oq_poll_error(layer)
-        return t1, t2, wall, clk
+        return per, wall, clk
 
     K = args.steps
     route = args.route
-    other = "codes" if route == "levels" else "levels"
-    t_rq, t_mm, wall, clk = timed(route, K, args.warmup, sample_clocks=True)
-    total_ms = max_over_ranks(sum(a + b for a, b in zip(t_rq, t_mm)), dev)
-    o_rq, o_mm, _, _ = timed(other, K, max(3, args.warmup // 2))
-    other_ms = max_over_ranks(sum(a + b for a, b in zip(o_rq, o_mm)), dev)
+    others = [o for o in ("levels", "levels_wdec", "codes") if o != route]
+    per, wall, clk = timed(route, K, args.warmup, sample_clocks=True)
+    total_ms = max_over_ranks(sum(sum(v) for v in per.values()), dev)
+    other_per = {o: timed(o, K, max(3, args.warmup // 2))[0] for o in others}
+    other_ms = {o: max_over_ranks(sum(sum(v) for v in other_per[o].values()), dev) for o in others}
 
     # the fused call, same workload (one C call, both kernels)
     for _ in range(2):
@@ -332,26 +336,38 @@ def run_ours(args):
 
     def rq_bytes_per_launch(rt):
         # bf16 x read + A operand written (fp16 levels, or packed codes) + norms
-        return T * (2 * d + (2 * d if rt == "levels" else d * lay.a_bits / 8) + 4)
+        return T * (2 * d + (2 * d if rt != "codes" else d * lay.a_bits / 8) + 4)
 
-    mm_ms = statistics.mean(t_mm)
-    rq_ms = statistics.mean(t_rq)
+    def route_decoded(rt):
+        return rt == "levels" and decoded
+
+    wl_bytes = dout * d * (lay.w_bits / 8 + 2)     # weight codes read + fp16 levels written
+    mm_ms = statistics.mean(per["gemm"])
+    rq_ms = statistics.mean(per["rq"])
     rq_bytes = rq_bytes_per_launch(route)
     gemm_tf = flops / (mm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
-    kernels = {
-        "levels": ("codebook GEMM, fp16 A operand by TMA, weight codes decoded to fp16 in shared memory "
-                   "(tcgen05 CTA pair, fp32 TMEM accumulate)",
-                   "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes) writing the codes' fp16 levels"),
+    gemm_desc = {
+        "decoded": ("codebook GEMM on fp16 levels of both operands, both by TMA "
+                    "(tcgen05 CTA pair, fp32 TMEM accumulate)", "gemm_decoded"),
+        "levels_wdec": ("codebook GEMM, fp16 A operand by TMA, weight codes decoded to fp16 in shared memory "
+                        "(tcgen05 CTA pair, fp32 TMEM accumulate)", "gemm_levels"),
         "codes": ("codebook GEMM, both operands' codes decoded to fp16 in shared memory "
-                  "(tcgen05 CTA pair, fp32 TMEM accumulate)",
-                  "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes, pack)"),
+                  "(tcgen05 CTA pair, fp32 TMEM accumulate)", None),
+    }
+    gkey = "decoded" if route_decoded(route) else ("codes" if route == "codes" else "levels_wdec")
+    rq_desc = {
+        "levels": "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes) writing the codes' fp16 levels",
+        "codes": "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes, pack)",
     }
     steps_desc = {
-        "levels": "oq_rotate_quantize_levels + oq_linear_levels (the two stages of oq_linear_fused; "
-                  "weights prepared once, offline)",
+        "levels": ("oq_rotate_quantize_levels + oq_weight_levels + oq_linear_decoded" if decoded else
+                   "oq_rotate_quantize_levels + oq_linear_levels")
+        + " (the stages of oq_linear_fused at this batch size; weights prepared once, offline)",
+        "levels_wdec": "oq_rotate_quantize_levels + oq_linear_levels (weight codes decoded inside the contraction)",
         "codes": "oq_rotate_quantize + oq_linear (weights prepared once, offline)",
     }
+    full_size = T == wl.tokens
     out = {
         "metric": METRIC,
         "value": whole_job_rate(world, T, K, total_ms),
@@ -374,36 +390,45 @@ def run_ours(args):
             "step": steps_desc[route],
         },
         "roofline": {
-            "kernel": kernels[route][0],
+            "kernel": gemm_desc[gkey][0],
             "bound": "tensor", "achieved": gemm_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
             "frac": gemm_tf / peaks["bf16_tflops"],
-            "traffic": measured_traffic("gemm_levels") if (route == "levels" and T == wl.tokens) else None,
+            "traffic": measured_traffic(gemm_desc[gkey][1]) if (gemm_desc[gkey][1] and full_size) else None,
             "peak_source": f"{peaks['source']} bf16 dense burst (fp16 has the same tensor rate)",
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, profiles/traffic.json",
             "flops_per_launch": flops, "ms_per_launch": mm_ms,
         },
         "roofline_rotate_quantize": {
-            "kernel": kernels[route][1],
+            "kernel": rq_desc["codes" if route == "codes" else "levels"],
             "bound": "hbm", "achieved": rq_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": rq_gbs / peaks["hbm_gbs"],
-            "traffic": measured_traffic("rq_levels") if (route == "levels" and T == wl.tokens) else None,
+            "traffic": measured_traffic("rq_levels") if (route != "codes" and full_size) else None,
             "peak_source": f"{peaks['source']} HBM copy bandwidth",
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, profiles/traffic.json",
             "bytes_per_launch": rq_bytes, "ms_per_launch": rq_ms,
         },
+        **({"roofline_weight_levels": {
+            "kernel": "weight codes -> fp16 levels (once per call)",
+            "bound": "hbm", "achieved": wl_bytes / (statistics.mean(per["wlevels"]) * 1e-3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": wl_bytes / (statistics.mean(per["wlevels"]) * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "traffic": measured_traffic("weight_levels") if full_size else None,
+            "bytes_per_launch": wl_bytes, "ms_per_launch": statistics.mean(per["wlevels"]),
+        }} if "wlevels" in per else {}),
         "fused": {"value": T / (statistics.mean(t_fused) * 1e-3), "unit": UNIT,
                   "ms_per_call": statistics.mean(t_fused), "call": "oq_linear_fused"},
-        "other_route": {"route": other, "step": steps_desc[other],
-                        "value": whole_job_rate(world, T, K, other_ms), "unit": UNIT, "ms_per_step": other_ms / K,
-                        "gemm_tflops": flops / (statistics.mean(o_mm) * 1e-3) / 1e12,
-                        "gemm_ms": statistics.mean(o_mm),
-                        "rq_gbs": rq_bytes_per_launch(other) / (statistics.mean(o_rq) * 1e-3) / 1e9,
-                        "rq_ms": statistics.mean(o_rq)},
+        "other_routes": [{"route": o, "step": steps_desc[o],
+                          "value": whole_job_rate(world, T, K, other_ms[o]), "unit": UNIT,
+                          "ms_per_step": other_ms[o] / K,
+                          "gemm_tflops": flops / (statistics.mean(other_per[o]["gemm"]) * 1e-3) / 1e12,
+                          "gemm_ms": statistics.mean(other_per[o]["gemm"]),
+                          "rq_gbs": rq_bytes_per_launch(o) / (statistics.mean(other_per[o]["rq"]) * 1e-3) / 1e9,
+                          "rq_ms": statistics.mean(other_per[o]["rq"])} for o in others],
         "e2e": {"value": whole_job_rate(world, T, K, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()),
                 "path": "pinned host x -> device, oq_linear_fused, y -> pinned host"},
-        "gpu_launches": 2 * K,
+        "gpu_launches": len(stages[route]) * K,
         "wall_s_timed_region": wall,
         "clocks": clk,
     }

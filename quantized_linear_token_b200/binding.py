@@ -23,6 +23,9 @@ OQ_FLAG_SIGNS = 1
 OQ_FLAG_GAUSSIAN_MARGINAL = 2
 OQ_FLAG_WEIGHT_ONLY_INT4 = 4
 OQ_FLAG_FP8_CONTRACTION = 8
+# oq_linear_fused decodes the weight codes once per call from this many tokens
+# on (bf16 x, d_out % 256 == 0, a workspace of oq_linear_fused_workspace_size)
+W16_MIN_T = 1024
 
 # every symbol include/orbitquant.h declares
 EXPORTS = (

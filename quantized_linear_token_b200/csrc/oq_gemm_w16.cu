@@ -1,17 +1,11 @@
-// Decode-then-contract route for large batches.
-//
-// (1) levels_kernel expands packed codes rows [R, K] into their fp16 operand
-//     values alpha * C[code] (row-major [R, K]): one pass over the codes, HBM
-//     bound.  For the weights this is once per call instead of once per
-//     256-token tile inside the contraction, and the 2 d_out d_in bytes it
-//     writes stay in L2 for the contraction that follows.
-// (2) gemm_w16_kernel contracts two fp16 level operands on CTA pairs
-//     (tcgen05 cta_group::2, M = 256, N = 256, K = 16 per MMA):
-//       y[m, n] = a_scale[m] b_scale[n] out_scale sum_k A[m, k] B[n, k]
-//     (gecl notes Method 2 and Takeaway 3: the product of the two codebook
-//     operands in the shared rotated basis; the dequantised levels are exact
-//     in fp16 up to the codebook's fp16 scale, and the tensor cores add them in
-//     fp32).
+// Decode-then-contract route for large batches, second kernel: the
+// contraction of two fp16 level operands on CTA pairs (tcgen05 cta_group::2,
+// M = 256, N = 256, K = 16 per MMA):
+//   y[m, n] = a_scale[m] b_scale[n] out_scale sum_k A[m, k] B[n, k]
+// (gecl notes Method 2 and Takeaway 3: the product of the two codebook
+// operands in the shared rotated basis; the levels are exact in fp16 up to the
+// codebook's fp16 scale, and the tensor cores add them in fp32).  The weight
+// operand comes from oq_levels.cu, decoded once per call.
 //
 // Each CTA of a pair loads its 128 A rows and 128 B rows of every K block of
 // 64 by TMA into its own shared memory and counts the bytes on the even CTA's
@@ -29,64 +23,12 @@
 #include <algorithm>
 #include <cstring>
 
-#include "oq_decode.cuh"
 #include "oq_internal.h"
 #include "oq_ptx.cuh"
 #include "oq_tmap.cuh"
 
 namespace oq {
 namespace {
-
-// ------------------------------------------------------------------ (1) levels
-
-template <int BITS>
-__global__ void __launch_bounds__(256) levels_kernel(const uint32_t* __restrict__ codes, int64_t rows, int K,
-                                                     int wpr, uint4 tabv, DecK kc, const uint16_t* lut8_g,
-                                                     uint16_t* __restrict__ out) {
-  __shared__ uint16_t lut8[256];
-  if constexpr (BITS == 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = lut8_g[i];
-    __syncthreads();
-  }
-  const uint32_t t[4] = {tabv.x, tabv.y, tabv.z, tabv.w};
-  constexpr int QP = Fmt<BITS>::QP, CPP = Fmt<BITS>::CPP;
-  const int nkb = (K + DEC_BK - 1) / DEC_BK;
-  const int64_t items = rows * nkb * QP;
-  // item = (row, K block, part): consecutive threads read consecutive code
-  // parts and write consecutive runs of CPP 16-byte chunks
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < items; i += (int64_t)gridDim.x * blockDim.x) {
-    const int q = (int)(i % QP);
-    const int64_t rk = i / QP;
-    const int kb = (int)(rk % nkb);
-    const int64_t r = rk / nkb;
-    const uint4 v = load_part<BITS>(codes + r * wpr, kb, q, K);
-    uint16_t* o = out + r * K + kb * DEC_BK + q * CPP * 8;
-#pragma unroll
-    for (int j = 0; j < CPP; ++j)
-      if (kb * DEC_BK + (q * CPP + j) * 8 < K)
-        *reinterpret_cast<uint4*>(o + j * 8) = decode_chunk_k<BITS>(v, j, t, lut8, kc);
-  }
-}
-
-template <int BITS>
-oq_status levels_launch_t(const uint32_t* codes, int64_t rows, int K, const uint16_t* levels_host,
-                          const uint16_t* levels_dev, uint16_t* out, void* stream) {
-  uint32_t t[4] = {0u, 0u, 0u, 0u};
-  make_decode_tables(BITS, levels_host, t);
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t items = rows * ((K + DEC_BK - 1) / DEC_BK) * Fmt<BITS>::QP;
-  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((items + 255) / 256, (int64_t)sms * 8));
-  levels_kernel<BITS><<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      codes, rows, K, K * BITS / 32, make_uint4(t[0], t[1], t[2], t[3]), make_deck(), levels_dev, out);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    set_error(std::string("levels launch: ") + cudaGetErrorString(e));
-    return OQ_ERR_CUDA;
-  }
-  return OQ_OK;
-}
 
 // ------------------------------------------------------------------ (2) contraction
 
@@ -297,19 +239,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
 }
 
 }  // namespace
-
-oq_status levels_launch(const uint32_t* codes, int64_t rows, int K, int bits, const uint16_t* levels_host,
-                        const uint16_t* levels_dev, uint16_t* out, void* stream) {
-  if (rows == 0) return OQ_OK;
-  if (K % 32 != 0) return OQ_ERR_UNSUPPORTED;
-  switch (bits) {
-    case 2: return levels_launch_t<2>(codes, rows, K, levels_host, levels_dev, out, stream);
-    case 3: return levels_launch_t<3>(codes, rows, K, levels_host, levels_dev, out, stream);
-    case 4: return levels_launch_t<4>(codes, rows, K, levels_host, levels_dev, out, stream);
-    case 8: return levels_launch_t<8>(codes, rows, K, levels_host, levels_dev, out, stream);
-    default: return OQ_ERR_UNSUPPORTED;
-  }
-}
 
 oq_status gemm_w16_launch(const GemmArgs& g, void* stream) {
   if (g.M == 0) return OQ_OK;
