@@ -301,26 +301,36 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 96)
 #pragma unroll
       for (int gi = 0; gi < E / 32; ++gi) {
         if constexpr (OUT16) {
-          // the codes' fp16 levels (the contraction's A operand), two per word
-          uint32_t o[16];
+          // the codes' fp16 levels (the contraction's A operand), two per
+          // word, eight per 16-byte chunk
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            uint32_t sel = 0u, pay[2];
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[4];
 #pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-              const float g = z[gi * 32 + i + e2] * ks;
-              int m = __float_as_int(g + 12582912.0f) + boffv;
-              m = min(max(m, 0), nb1);
-              const uint2 en = tbl[m];
-              pay[e2] = en.y;
-              const bool up = g > __uint_as_float(en.x);
-              sel |= (up ? 0x32u : 0x10u) << (8 * e2);
+            for (int i = 0; i < 8; i += 2) {
+              uint32_t sel = 0u, pay[2];
+#pragma unroll
+              for (int e2 = 0; e2 < 2; ++e2) {
+                const float g = z[gi * 32 + q * 8 + i + e2] * ks;
+                int m = __float_as_int(g + 12582912.0f) + boffv;
+                m = min(max(m, 0), nb1);
+                const uint2 en = tbl[m];
+                pay[e2] = en.y;
+                const bool up = g > __uint_as_float(en.x);
+                sel |= (up ? 0x32u : 0x10u) << (8 * e2);
+              }
+              o[i >> 1] = __byte_perm(pay[0], pay[1], sel | 0x4400u);
             }
-            o[i >> 1] = __byte_perm(pay[0], pay[1], sel | 0x4400u);
+            const uint4 ch = make_uint4(o[0], o[1], o[2], o[3]);
+            if constexpr (PASSES == 2) {
+              // into this thread's own exchange region (its z values are
+              // already in registers), slot swizzled by c so that both this
+              // store and the group reads below are free of bank conflicts
+              reinterpret_cast<uint4*>(work + j * (H + PAD) + c * E)[(gi * 4 + q) ^ (c & 7)] = ch;
+            } else {
+              reinterpret_cast<uint4*>(p.out16 + (size_t)t * d + pos0 + gi * 32)[q] = ch;
+            }
           }
-          uint4* dst = reinterpret_cast<uint4*>(p.out16 + (size_t)t * d + pos0 + gi * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
         } else {
           // 32 consecutive positions straight into BITS packed words
           uint32_t w[BITS];
@@ -352,6 +362,29 @@ __global__ void __maxnreg__(elems_per_thread(1 << LOG_H) == 64 ? 168 : 96)
         }
       }
       if (tid == 0) p.norms[t] = s;
+    }
+    if constexpr (OUT16 && PASSES == 2) {
+      // Each thread's 32 fp16 levels are 64 contiguous output bytes; stored
+      // directly, a warp's 16-byte stores would land 64 bytes apart and write
+      // every 32-byte sector in halves.  Instead the four threads of a group
+      // (consecutive c, one row, one warp) swap chunks through their exchange
+      // regions: in store qq lane i writes chunk i of thread c0 + qq, so each
+      // store of the group covers 64 contiguous bytes (two whole sectors).
+      __syncwarp();
+      if (valid) {
+        const int i4 = c & 3, c0 = c & ~3;
+        const float* base = work + j * (H + PAD) + c0 * E;
+        uint16_t* rowout = p.out16 + (size_t)t * d + j * H;
+#pragma unroll
+        for (int gi = 0; gi < E / 32; ++gi) {
+#pragma unroll
+          for (int qq = 0; qq < 4; ++qq) {
+            const int cs = c0 + qq;
+            const uint4 ch = reinterpret_cast<const uint4*>(base + qq * E)[(gi * 4 + i4) ^ (cs & 7)];
+            reinterpret_cast<uint4*>(rowout + cs * E + gi * 32)[i4] = ch;
+          }
+        }
+      }
     }
     __syncthreads();
   }
