@@ -309,22 +309,20 @@ def run_ours(args):
     torch.cuda.synchronize()
     t_fused = [evf[i][0].elapsed_time(evf[i][1]) for i in range(K)]
 
-    # end to end through the public API with host buffers: pinned x -> device,
-    # fused call, y -> pinned host, all inside the events
+    # end to end through the public API with host buffers: the host-buffer
+    # fused call copies pinned x in, computes and copies y out to pinned host
+    # memory, overlapped chunk by chunk; all of it inside the events
     x_host = x.cpu().pin_memory()
     y_host = torch.empty((T, dout), dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(x)
+    ws_host = torch.empty((max(B.oq_linear_fused_host_workspace_size(layer, B.OQ_DTYPE_BF16, T), 1),),
+                          dtype=torch.uint8, device=dev)
     eve = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     for i in range(max(2, args.warmup // 2)):
-        x_dev.copy_(x_host, non_blocking=True)
-        B.oq_linear_fused(layer, x_dev, Wc, r, y, ws)
-        y_host.copy_(y, non_blocking=True)
+        B.oq_linear_fused_host(layer, x_host, Wc, r, y_host, ws_host)
     torch.cuda.synchronize()
     for i in range(K):
         eve[i][0].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        B.oq_linear_fused(layer, x_dev, Wc, r, y, ws)
-        y_host.copy_(y, non_blocking=True)
+        B.oq_linear_fused_host(layer, x_host, Wc, r, y_host, ws_host)
         eve[i][1].record(stream)
     torch.cuda.synchronize()
     t_e2e = [eve[i][0].elapsed_time(eve[i][1]) for i in range(K)]
@@ -427,7 +425,7 @@ def run_ours(args):
         "e2e": {"value": whole_job_rate(world, T, K, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()),
-                "path": "pinned host x -> device, oq_linear_fused, y -> pinned host"},
+                "path": "oq_linear_fused_host: pinned host x -> device, fused call, y -> pinned host, overlapped in chunks of 1024 tokens"},
         "gpu_launches": len(stages[route]) * K,
         "wall_s_timed_region": wall,
         "clocks": clk,

@@ -310,6 +310,31 @@ oq_status oq_linear_decoded(const oq_layer* layer, const uint16_t* a16, const fl
 oq_status oq_linear_fused_static(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
                                  const uint32_t* Wcodes, const float* r, float* y, void* stream);
 
+/*
+ * oq_linear_fused_host -- oq_linear_fused with x and y in HOST memory (page-
+ * locked for the copies to overlap; pageable memory works but serialises
+ * them).  The pages have no counterpart; this is the interface for callers
+ * whose activations live in host memory.
+ *   x_host     host [T, d_in] bf16 (OQ_DTYPE_BF16) or fp32 (OQ_DTYPE_F32).
+ *   y_host     host [T, d_out] fp32.
+ *   Wcodes, r  device, from oq_weight_prepare.
+ *   workspace  device scratch of oq_linear_fused_host_workspace_size(layer,
+ *              x_dtype, T) bytes, 256-byte aligned.
+ * The batch runs in chunks of 1024 tokens: the copy of chunk i + 1 into the
+ * device, the computation of chunk i (on `stream`) and the copy of chunk i - 1
+ * out to the host overlap, on two copy streams that the layer creates on its
+ * first such call and keeps until oq_layer_destroy (make that first call before
+ * any stream capture).  Work queued on `stream` before the call runs first;
+ * work queued after it waits for y to be in host memory (synchronise `stream`
+ * before reading y_host).  y is exactly the y of oq_linear_fused on the whole
+ * batch.  Calls on one layer must not overlap (they share its copy streams).
+ * Errors: as oq_linear_fused; OQ_ERR_UNSUPPORTED on an INT4 weight-only layer.
+ */
+size_t oq_linear_fused_host_workspace_size(const oq_layer* layer, int32_t x_dtype, int64_t T);
+oq_status oq_linear_fused_host(const oq_layer* layer, const void* x_host, int32_t x_dtype, int64_t T,
+                               const uint32_t* Wcodes, const float* r, float* y_host, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
 /* Reads and clears the layer's device error word.  Synchronizes the device.
  * Returns OQ_OK, OQ_ERR_TIMEOUT or OQ_ERR_DEVICE. */
 oq_status oq_poll_error(const oq_layer* layer);

@@ -32,7 +32,7 @@ EXPORTS = (
     "oq_codebook_build", "oq_rotation_build", "oq_layer_create", "oq_layer_destroy", "oq_layer_get_info", "oq_layer_get_perm",
     "oq_rotate_quantize", "oq_weight_prepare", "oq_linear", "oq_linear_fused_workspace_size",
     "oq_linear_fused", "oq_rotate_quantize_levels", "oq_linear_levels", "oq_weight_levels", "oq_linear_decoded",
-    "oq_linear_fused_static",
+    "oq_linear_fused_static", "oq_linear_fused_host_workspace_size", "oq_linear_fused_host",
     "oq_poll_error", "oq_last_error", "oq_status_string",
 )
 
@@ -89,6 +89,8 @@ def load_library(path: str = LIB_PATH):
         "oq_rotate_quantize_levels": (i32, [vp, vp, i32, i64, vp, vp, vp]),
         "oq_linear_levels": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_weight_levels": (i32, [vp, vp, vp, vp]),
+        "oq_linear_fused_host_workspace_size": (ctypes.c_size_t, [vp, i32, i64]),
+        "oq_linear_fused_host": (i32, [vp, vp, i32, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]),
         "oq_linear_decoded": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
         "oq_poll_error": (i32, [vp]),
@@ -304,6 +306,41 @@ def oq_linear_decoded(layer: Layer, a16, s, w16, r, y=None):
     _check(load_library().oq_linear_decoded(layer.handle, _dev(a16, "a16"), _dev(s, "s"), T, _dev(w16, "w16"),
                                             _dev(r, "r"), _dev(y, "y"), _stream(a16)), "oq_linear_decoded")
     return y
+
+
+def oq_linear_fused_host_workspace_size(layer: Layer, x_dtype: int, T: int) -> int:
+    return int(load_library().oq_linear_fused_host_workspace_size(layer.handle, x_dtype, T))
+
+
+def _host(t, name: str):
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def oq_linear_fused_host(layer: Layer, x_host, Wcodes, r, y_host=None, workspace=None):
+    """x_host [T, d_in] bf16/fp32 in host memory (pinned for overlap) -> y_host
+    [T, d_out] fp32 in host memory: copies in, the fused call and copies out,
+    overlapped chunk by chunk, queued on the current stream of Wcodes' device.
+    Synchronise that stream before reading y_host."""
+    torch = _torch()
+    T = x_host.shape[0]
+    if x_host.dim() != 2 or x_host.shape[1] != layer.d_in:
+        raise ValueError("x_host must be [T, d_in]")
+    if y_host is None:
+        y_host = torch.empty((T, layer.d_out), dtype=torch.float32, pin_memory=True)
+    code = _dtype_code(x_host)
+    need = oq_linear_fused_host_workspace_size(layer, code, T)
+    if workspace is None:
+        workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Wcodes.device)
+    _check(load_library().oq_linear_fused_host(layer.handle, _host(x_host, "x_host"), code, T,
+                                               _dev(Wcodes, "Wcodes"), _dev(r, "r"), _host(y_host, "y_host"),
+                                               _dev(workspace, "workspace"),
+                                               workspace.numel() * workspace.element_size(), _stream(Wcodes)),
+           "oq_linear_fused_host")
+    return y_host
 
 
 def oq_linear_fused_static(layer: Layer, x, Wcodes, r, y=None):

@@ -85,6 +85,7 @@ static oq_status check_shape(int32_t d_in, int32_t d_out, int32_t a_bits, int32_
 
 void oq_layer_destroy(oq_layer* L) {
   if (!L) return;
+  io_release(L);
   cudaFree(L->d_gather_a);
   cudaFree(L->d_signmask);
   cudaFree(L->d_levels_a);
@@ -533,25 +534,20 @@ static oq_status int4_linear(const oq_layer* L, const void* x, int32_t x_dtype, 
   return OQ_OK;
 }
 
-oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                          const float* r, float* y, void* workspace, size_t workspace_bytes, void* stream) {
-  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: layer is null");
-  if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: T < 0");
-  if (T == 0) return OQ_OK;
-  oq_status st = check_rows_input(x, x_dtype, "oq_linear_fused");
-  if (st != OQ_OK) return st;
-  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, y, stream);
-  if (!Wcodes || !r || !y || !workspace) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: null pointer");
-  if (!aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(r, 16) || !aligned(workspace, 256))
-    return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: misaligned pointer (workspace needs 256 bytes)");
+// The fused call's body on checked arguments.  w16_ready: the weights' fp16
+// levels, already decoded by the caller (oq_linear_fused_host decodes them
+// once for all its chunks), or null.
+static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                              const float* r, float* y, unsigned char* ws, size_t workspace_bytes, void* stream,
+                              const uint16_t* w16_ready) {
+  oq_status st;
   const size_t need = min_workspace(L, T);
-  if (workspace_bytes < need) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
   if (fused_f16_route(L, x_dtype)) {
     uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
     float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
     st = rq_levels(L, x, x_dtype, T, a16, s, stream);
     if (st != OQ_OK) return st;
+    if (w16_ready) return linear_w16(L, a16, s, T, w16_ready, r, y, stream);
     // large batches with room for the decoded weights: decode them once, then
     // contract two fp16 operands; otherwise decode weights inside the contraction
     if (fused_w16_route(L, x_dtype, T) && workspace_bytes >= round256(need) + fused_w16_bytes(L)) {
@@ -563,10 +559,35 @@ oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int
     return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
   }
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws);
-  float* s = reinterpret_cast<float*>(ws + ((fused_codes_bytes(L, T) + 255) & ~(size_t)255));
+  float* s = reinterpret_cast<float*>(ws + round256(fused_codes_bytes(L, T)));
   st = rq(L, x, x_dtype, T, L->a_bits, L->bins_a, codes, s, stream);
   if (st != OQ_OK) return st;
   return linear_impl(L, codes, s, T, Wcodes, r, y, stream);
+}
+
+static oq_status fused_checks(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                              const float* r, const float* y, const void* workspace, const char* who) {
+  const std::string w(who);
+  if (!L) return fail(OQ_ERR_INVALID_ARG, w + ": layer is null");
+  if (T < 0) return fail(OQ_ERR_INVALID_ARG, w + ": T < 0");
+  if (T == 0) return OQ_OK;
+  const oq_status st = check_rows_input(x, x_dtype, who);
+  if (st != OQ_OK) return st;
+  if (L->int4_only) return OQ_OK;
+  if (!Wcodes || !r || !y || !workspace) return fail(OQ_ERR_INVALID_ARG, w + ": null pointer");
+  if (!aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(r, 16) || !aligned(workspace, 256))
+    return fail(OQ_ERR_INVALID_ARG, w + ": misaligned pointer (workspace needs 256 bytes)");
+  return OQ_OK;
+}
+
+oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                          const float* r, float* y, void* workspace, size_t workspace_bytes, void* stream) {
+  oq_status st = fused_checks(L, x, x_dtype, T, Wcodes, r, y, workspace, "oq_linear_fused");
+  if (st != OQ_OK || T == 0) return st;
+  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, y, stream);
+  if (workspace_bytes < min_workspace(L, T)) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
+  return fused_device(L, x, x_dtype, T, Wcodes, r, y, static_cast<unsigned char*>(workspace), workspace_bytes,
+                      stream, nullptr);
 }
 
 oq_status oq_poll_error(const oq_layer* L) {
@@ -588,4 +609,18 @@ oq_status oq_poll_error(const oq_layer* L) {
 
 namespace oq {
 size_t fused_min_workspace(const oq_layer* L, int64_t T) { return min_workspace(L, T); }
+size_t fused_w16_workspace(const oq_layer* L, int64_t T) { return round256(min_workspace(L, T)) + fused_w16_bytes(L); }
+bool fused_decodes_weights(const oq_layer* L, int32_t x_dtype, int64_t T) { return fused_w16_route(L, x_dtype, T); }
+oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                           const float* r, const float* y, const void* workspace, const char* who) {
+  return fused_checks(L, x, x_dtype, T, Wcodes, r, y, workspace, who);
+}
+oq_status fused_run(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                    const float* r, float* y, void* ws, size_t ws_bytes, void* stream, const uint16_t* w16_ready) {
+  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, y, stream);
+  return fused_device(L, x, x_dtype, T, Wcodes, r, y, static_cast<unsigned char*>(ws), ws_bytes, stream, w16_ready);
+}
+oq_status decode_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* w16, void* stream) {
+  return levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
+}
 }  // namespace oq

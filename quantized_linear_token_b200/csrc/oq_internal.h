@@ -45,6 +45,11 @@ struct oq_layer {
   int* d_error;                       // device error word
   oq_bin_table bins_a, bins_w;       // threshold search tables (activation / weight codebook)
   int* d_counters;                    // split-K hand-off counters of the small-batch contraction (zero at rest)
+  // host-buffer pipeline (oq_linear_fused_host): two copy streams and their
+  // events, created on the first call (opaque CUDA handles)
+  void* io_stream[2];
+  void* io_event[8];
+  bool io_ready;
 };
 
 namespace oq {
@@ -129,8 +134,20 @@ oq_status levels_launch(const uint32_t* codes, int64_t rows, int K, int bits, co
 oq_status gemm_w16_launch(const GemmArgs& g, void* stream);
 // the fused call decodes the weights once per call from this many tokens on
 constexpr int64_t W16_MIN_T = 1024;
-// the least workspace oq_linear_fused accepts (oq_api.cu)
+// the fused call's pieces for the host-buffer pipeline (oq_api.cu): the least
+// workspace; the workspace with the decoded weights after it; whether the
+// fused call decodes the weights once at this batch size; argument checks;
+// the call on checked arguments (w16_ready: weights already decoded, or null)
 size_t fused_min_workspace(const oq_layer* L, int64_t T);
+size_t fused_w16_workspace(const oq_layer* L, int64_t T);
+bool fused_decodes_weights(const oq_layer* L, int32_t x_dtype, int64_t T);
+oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                           const float* r, const float* y, const void* workspace, const char* who);
+oq_status fused_run(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                    const float* r, float* y, void* ws, size_t ws_bytes, void* stream, const uint16_t* w16_ready);
+oq_status decode_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* w16, void* stream);
+// host-buffer pipeline resources of a layer (oq_host_io.cu)
+void io_release(oq_layer* L);
 // prmt decode tables of a codebook's fp16 levels (oq_gemm.cu)
 void make_decode_tables(int bits, const uint16_t* levels, uint32_t* t);
 

@@ -325,6 +325,51 @@ def test_decoded_weight_route(env, d_in, d_out, a_bits, w_bits, T):
         B.oq_linear_fused(layer, x_t, Wc, r, workspace=ws[:least - 256])
 
 
+HOST_IO = [
+    # d_in, d_out, a, w, T, x dtype: several chunks with a ragged last one on
+    # the decoded-weight route; one chunk below the decode threshold; a batch
+    # of the small-batch kernel; fp32 x (packed-code route) over three chunks;
+    # d_out not a multiple of 256 (code route, one-SM contraction)
+    (3072, 768, 4, 4, 2600, "bf16"),
+    (640, 512, 3, 3, 700, "bf16"),
+    (1024, 256, 4, 2, 37, "bf16"),
+    (256, 256, 4, 4, 2100, "f32"),
+    (512, 384, 4, 4, 1500, "bf16"),
+]
+
+
+@pytest.mark.parametrize("d_in,d_out,a_bits,w_bits,T,xdt", HOST_IO)
+def test_host_buffer_pipeline(env, d_in, d_out, a_bits, w_bits, T, xdt):
+    # x and y in pinned host memory, copies overlapped with the computation
+    # chunk by chunk: y equals the device-buffer fused call's y bit for bit
+    torch, B = env
+    x_np = W.custom_activations(T, d_in, seed=d_in + 7 * T)
+    if xdt == "f32":
+        x_np = W.bf16_bits_to_f32(x_np)
+    Wm = W.custom_weights(d_out, d_in, seed=d_out + 11)
+    layer = B.oq_layer_create(d_in, d_out, 0, a_bits, w_bits, 0)
+    x_t, _ = _x_tensor(torch, x_np)
+    Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(Wm).cuda())
+    y_dev = B.oq_linear_fused(layer, x_t, Wc, r)
+    x_host = x_t.cpu().pin_memory()
+    ys = []
+    for _ in range(2):                  # a second call reuses the layer's copy streams
+        y_host = torch.full((T, d_out), float("nan"), dtype=torch.float32).pin_memory()
+        B.oq_linear_fused_host(layer, x_host, Wc, r, y_host)
+        torch.cuda.current_stream().synchronize()
+        ys.append(y_host.numpy().copy())
+    B.oq_poll_error(layer)
+    ref = y_dev.cpu().numpy()
+    for y in ys:
+        np.testing.assert_array_equal(y, ref)
+    need = B.oq_linear_fused_host_workspace_size(layer, B.OQ_DTYPE_BF16 if xdt == "bf16" else B.OQ_DTYPE_F32, T)
+    small = torch.empty((need - 256,), dtype=torch.uint8, device="cuda")
+    with pytest.raises(B.OrbitQuantError):
+        B.oq_linear_fused_host(layer, x_host, Wc, r, workspace=small)
+    with pytest.raises(ValueError):
+        B.oq_linear_fused_host(layer, x_t, Wc, r)
+
+
 def test_degenerate_tokens(env):
     # a zero token (s = 0, every code L/2 - 1, y = 0) and tokens with very
     # small and very large norms
