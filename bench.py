@@ -43,6 +43,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="dit_image")
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's token count (profiling)")
+    ap.add_argument("--layer", default="", help="layer of the workload by name (default: its first)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--route", choices=["levels", "levels_wdec", "codes"], default="levels",
                     help="hot-path route of the timed step (the others are reported beside it)")
@@ -218,7 +219,7 @@ def run_ours(args):
     B.load_library()
 
     wl = W.WORKLOADS[args.workload]
-    lay = wl.layers[0]
+    lay = next(l for l in wl.layers if l.name == args.layer) if args.layer else wl.layers[0]
     T, d, dout = (args.tokens or wl.tokens), lay.d_in, lay.d_out
     x_np = rank_batch(wl, d, T, rank)
     Wm = W.weights(wl, lay)
@@ -400,7 +401,7 @@ def run_ours(args):
         "dtype": "f16",
         "data": "synthetic",
         "config": {
-            "workload": f"{args.workload}: {wl.title}",
+            "workload": f"{args.workload}: {wl.title}", "layer": lay.name,
             "tokens_per_gpu": T, "d_in": d, "d_out": dout, "a_bits": lay.a_bits, "w_bits": lay.w_bits,
             "h": d & -d, "x_dtype": "bf16", "y_dtype": "fp32",
             "parallelism": f"token-sharded x{world}, weights replicated",
@@ -471,7 +472,7 @@ def run_reference(args):
         return
     from quantized_linear_token_b200 import workloads as W
     wl = W.WORKLOADS[args.workload]
-    lay = wl.layers[0]
+    lay = next(l for l in wl.layers if l.name == args.layer) if args.layer else wl.layers[0]
     per_step = max(1.0, 60.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_cpu_rate(wl, lay, min(per_step, 2.0))

@@ -208,13 +208,12 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
 
 /*
  * oq_linear_fused -- x -> y in one call: the rotate-quantize step produces
- * the A operand of the contraction (the same codes as oq_rotate_quantize
- * followed by oq_linear, and the same y; for batches of at most 256 tokens the
- * contraction runs a split-K kernel whose fp32 sums come in another order, so
- * y agrees to rounding).  With bf16 x and d_out % 256 == 0 the rotate-quantize
- * kernel writes the fp16 levels of the activation codes, which the contraction
- * reads with TMA (only the weight codes are decoded in the contraction);
- * otherwise the packed codes pass through the workspace.  `workspace` is
+ * the A operand of the contraction.  With bf16 x and d_out % 256 == 0 the
+ * rotate-quantize kernel writes the fp16 levels of the activation codes (as
+ * oq_rotate_quantize_levels), which the contraction reads with TMA (only the
+ * weight codes are decoded in the contraction); otherwise the packed codes of
+ * oq_rotate_quantize pass through the workspace and y is that of oq_linear
+ * (bit for bit).  `workspace` is
  * caller-owned device scratch, 256-byte aligned, that may be reused between
  * calls on one stream.  oq_linear_fused_workspace_size(layer, T) gives the
  * bytes of the fastest route: the A operand and the norms, and from 1024
@@ -245,6 +244,12 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  *   x    device [T, d_in] bf16 (OQ_DTYPE_BF16 only, else OQ_ERR_UNSUPPORTED).
  *   a16  device [T, d_in] uint16 (fp16 bits), 16-byte aligned.
  *   s    device [T] fp32 token norms.
+ * For h = 1024 without OQ_FLAG_SIGNS the block transform runs on the tensor
+ * cores (H_1024 = H_32 (x) H_32 as two rounds of warp MMAs, the second on a
+ * two-term tf32 split of the fp32 intermediate): its fp32 rounding differs
+ * from oq_rotate_quantize's, so a code may differ from that call's where the
+ * coordinate lies within rounding of a decision threshold, and s may differ
+ * in the last bits.  Both meet the same bounds against the exact transform.
  *
  * oq_linear_levels -- oq_linear with the A operand given as those fp16
  * levels (read by TMA; only the weight codes are decoded):

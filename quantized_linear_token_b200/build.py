@@ -19,7 +19,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "liborbitquant.so")
 
-SOURCES = ["oq_api.cu", "oq_rotate_quantize.cu", "oq_gemm.cu", "oq_gemm_pair.cu", "oq_gemm_skinny.cu", "oq_gemm_w16.cu",
+SOURCES = ["oq_api.cu", "oq_rotate_quantize.cu", "oq_rotate_quantize_tc.cu", "oq_gemm.cu", "oq_gemm_pair.cu", "oq_gemm_skinny.cu", "oq_gemm_w16.cu",
            "oq_levels.cu", "oq_host_io.cu", "oq_int4.cu",
            "oq_noalloc.cu", "oq_host.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

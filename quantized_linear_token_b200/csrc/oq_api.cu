@@ -87,6 +87,7 @@ void oq_layer_destroy(oq_layer* L) {
   if (!L) return;
   io_release(L);
   cudaFree(L->d_gather_a);
+  cudaFree(L->d_gather_tc);
   cudaFree(L->d_signmask);
   cudaFree(L->d_levels_a);
   cudaFree(L->d_levels_w);
@@ -212,6 +213,14 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   st = cuda_check(cudaMalloc(&L->d_gather_a, gather.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
   if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_gather_a, gather.data(), gather.size() * sizeof(uint16_t),
                                               cudaMemcpyHostToDevice), "upload gather");
+  if (st == OQ_OK && L->h == 1024 && !signed_rot && d_in / 1024 <= 8) {
+    std::vector<uint16_t> gather_tc;
+    rqtc_build_gather(d_in, L->perm_host, gather_tc);
+    st = cuda_check(cudaMalloc(&L->d_gather_tc, gather_tc.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
+    if (st == OQ_OK)
+      st = cuda_check(cudaMemcpy(L->d_gather_tc, gather_tc.data(), gather_tc.size() * sizeof(uint16_t),
+                                 cudaMemcpyHostToDevice), "upload gather");
+  }
   if (st == OQ_OK && signed_rot) {
     st = cuda_check(cudaMalloc(&L->d_signmask, signmask.size() * sizeof(uint32_t)), "cudaMalloc(signs)");
     if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_signmask, signmask.data(), signmask.size() * sizeof(uint32_t),
@@ -428,6 +437,8 @@ static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, in
   a.out16 = a16;
   a.norms = s;
   a.err = L->d_error;
+  a.gather_tc = L->d_gather_tc;
+  if (rqtc_supported(a)) return rqtc_launch(a, stream);
   return rq_launch(a, stream);
 }
 

@@ -16,11 +16,15 @@ namespace {
 // chunk i of the flat output is chunk i % CPP of flat code part i / CPP.  One
 // chunk (16 output bytes) per thread and step: consecutive lanes write
 // consecutive 16-byte pieces, and the CPP lanes of a part load the same bytes
-// (one L1 line serves them).
+// (one L1 line serves them).  Each thread takes UNROLL steps of the grid
+// stride at a time and issues their loads before any decode, so that several
+// loads per thread are in flight (one at a time left the kernel bound by
+// load latency).
 template <int BITS>
 __global__ void __launch_bounds__(256) levels_flat_kernel(const uint32_t* __restrict__ codes, int64_t chunks,
                                                           uint4 tabv, DecK kc, const uint16_t* lut8_g,
                                                           uint4* __restrict__ out) {
+  constexpr int UNROLL = 4;
   __shared__ uint16_t lut8[256];
   if constexpr (BITS == 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = lut8_g[i];
@@ -28,17 +32,28 @@ __global__ void __launch_bounds__(256) levels_flat_kernel(const uint32_t* __rest
   }
   const uint32_t t[4] = {tabv.x, tabv.y, tabv.z, tabv.w};
   constexpr int CPP = Fmt<BITS>::CPP;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < chunks; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t part = i / CPP;
-    const int j = (int)(i % CPP);
-    uint4 v;
-    if constexpr (BITS == 3) {
-      const uint32_t* pw = codes + part * 3;   // 32 codes in three words
-      v = make_uint4(__ldg(pw), __ldg(pw + 1), __ldg(pw + 2), 0u);
-    } else {
-      v = __ldg(reinterpret_cast<const uint4*>(codes) + part);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < chunks; i0 += UNROLL * stride) {
+    uint4 v[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (i < chunks) {
+        const int64_t part = i / CPP;
+        if constexpr (BITS == 3) {
+          const uint32_t* pw = codes + part * 3;   // 32 codes in three words
+          v[u] = make_uint4(__ldg(pw), __ldg(pw + 1), __ldg(pw + 2), 0u);
+        } else {
+          v[u] = __ldg(reinterpret_cast<const uint4*>(codes) + part);
+        }
+      }
     }
-    out[i] = decode_chunk_k<BITS>(v, j, t, lut8, kc);
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < chunks) out[i] = decode_chunk_k<BITS>(v[u], (int)(i % CPP), t, lut8, kc);
+    }
   }
 }
 

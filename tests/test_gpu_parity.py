@@ -62,23 +62,22 @@ def _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, flags=0, seed=0, w_ro
     # contraction on the GPU's own codes
     y_np, yf_np = y.cpu().numpy(), yf.cpu().numpy()
     lin = check_linear(y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, label + " y", rows=y_rows)
-    # the fused call computes the same codes, so the same y: bit for bit when
-    # both run the CTA-pair kernel; for small batches the fused route runs the
-    # split-K small-batch kernel (another summation order), which is checked
-    # against the oracle itself and against the codes route to fp32 rounding
-    _same_y(yf_np, y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, T_small=_small_batch(x_np, d_out),
-            label=label + " fused", rows=y_rows)
     if x_np.dtype == np.uint16 and d_out % 256 == 0:
-        _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in,
-                            Wc_np, r_np, cb_w, y_rows, label)
+        # fp16-level route: its rotate-quantize kernel may be the tensor-core
+        # FWHT one (h = 1024), whose fp32 rounding differs from the code
+        # route's, so its codes are checked against the oracle on their own;
+        # the fused call runs that route and gives its y bit for bit
+        y2 = _check_level_stages(env, layer, x_t, Wc, r, x64, perm, h, signs, cb_a, a_bits, d_in,
+                                 Wc_np, r_np, cb_w, y_rows, label)
+        np.testing.assert_array_equal(yf_np, y2)
+    else:
+        # the fused call computes the code route's codes, so the same y
+        _same_y(yf_np, y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, T_small=False,
+                label=label + " fused", rows=y_rows)
     return st, lin
 
 
 SKINNY_MAX_T = 256   # batches up to this size take the small-batch kernel on the fp16-level route
-
-
-def _small_batch(x_np, d_out):
-    return x_np.dtype == np.uint16 and x_np.shape[0] <= SKINNY_MAX_T and d_out % 128 == 0
 
 
 def _same_y(y_new, y_ref, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, T_small, label, rows=None):
@@ -93,36 +92,50 @@ def _same_y(y_new, y_ref, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in, T_small
     assert float((diff / np.where(bound > 0, bound, 1.0)).max()) <= 1e-5, label
 
 
-def _check_level_stages(env, layer, x_t, Wc, r, codes_np, s_np, y_np, cb_a, a_bits, d_in, Wc_np, r_np, cb_w,
+def levels_to_codes(a16_bits: np.ndarray, levels_f16: np.ndarray, label: str) -> np.ndarray:
+    """Codes of an fp16 level operand: every value must be one of the
+    codebook's fp16 levels (which are distinct)."""
+    order = np.argsort(levels_f16)
+    pos = np.searchsorted(levels_f16[order], a16_bits)
+    pos = np.minimum(pos, len(order) - 1)
+    ok = levels_f16[order][pos] == a16_bits
+    assert ok.all(), f"{label}: {int((~ok).sum())} values that are no codebook level"
+    return order[pos].astype(np.int64)
+
+
+def _check_level_stages(env, layer, x_t, Wc, r, x64, perm, h, signs, cb_a, a_bits, d_in, Wc_np, r_np, cb_w,
                         y_rows, label):
-    """The fused call's fp16 route as two calls: the A operand holds exactly the
-    fp16 value of a_scale times the level of each code, the norms are the
-    same, and the contraction gives the same y."""
+    """The fused call's fp16 route as two calls: the A operand holds exactly
+    the fp16 value of a_scale times the level of a code, those codes and the
+    norms match the oracle (same bounds as the code route), and the
+    contraction of the operand matches the oracle on those codes.  Returns
+    the route's y."""
     torch, B = env
     a16, s2 = B.oq_rotate_quantize_levels(layer, x_t)
     y2 = B.oq_linear_levels(layer, a16, s2, Wc, r)
     torch.cuda.synchronize()
     B.oq_poll_error(layer)
-    np.testing.assert_array_equal(s2.cpu().numpy(), s_np)
-    c = O.unpack_codes(codes_np, a_bits, d_in)
-    want = (layer.a_scale * np.asarray(cb_a.levels, dtype=np.float64))[c].astype(np.float16).view(np.uint16)
-    np.testing.assert_array_equal(a16.cpu().numpy().view(np.uint16), want)
+    lv = (layer.a_scale * np.asarray(cb_a.levels, dtype=np.float64)).astype(np.float16).view(np.uint16)
+    c16 = levels_to_codes(a16.cpu().numpy().view(np.uint16), lv, label + " levels")
+    words16, s2_np = O.pack_codes(c16, a_bits), s2.cpu().numpy()
+    check_codes(words16, x64, perm, h, cb_a, a_bits, signs, s2_np, label + " levels x")
+    y2_np = y2.cpu().numpy()
+    check_linear(y2_np, words16, s2_np, Wc_np, r_np, cb_a, cb_w, d_in, label + " levels y", rows=y_rows)
     # the split-K small-batch path adds its splits in a fixed order: repeat
     # calls give the same bits
     y3 = B.oq_linear_levels(layer, a16, s2, Wc, r)
     torch.cuda.synchronize()
-    np.testing.assert_array_equal(y3.cpu().numpy(), y2.cpu().numpy())
-    _same_y(y2.cpu().numpy(), y_np, codes_np, s_np, Wc_np, r_np, cb_a, cb_w, d_in,
-            T_small=codes_np.shape[0] <= SKINNY_MAX_T and Wc_np.shape[0] % 128 == 0, label=label + " levels",
-            rows=y_rows)
-    _check_decoded(env, layer, a16, s2, Wc, r, codes_np, s_np, y_np, d_in, Wc_np, r_np, cb_a, cb_w, y_rows, label)
+    np.testing.assert_array_equal(y3.cpu().numpy(), y2_np)
+    _check_decoded(env, layer, a16, s2, Wc, r, words16, s2_np, y2_np, d_in, Wc_np, r_np, cb_a, cb_w, y_rows, label)
+    return y2_np
 
 
 def _check_decoded(env, layer, a16, s, Wc, r, codes_np, s_np, y_np, d_in, Wc_np, r_np, cb_a, cb_w, y_rows, label):
     """The decode-then-contract route: the weights' fp16 levels hold exactly
     fp16(w_scale C_w[code]), and the contraction of the two fp16 operands gives
-    the codes route's y (the same MMAs in the same order on CTA pairs; to fp32
-    summation order against the small-batch kernel)."""
+    the y of oq_linear_levels on the same A operand (the same MMAs in the same
+    order on CTA pairs; to fp32 summation order against the small-batch
+    kernel)."""
     torch, B = env
     w16 = B.oq_weight_levels(layer, Wc)
     y4 = B.oq_linear_decoded(layer, a16, s, w16, r)
@@ -192,6 +205,9 @@ EDGE = [
     (3072, 512, 4, 4, 96, 3),      # image-DiT width, signed RPBH and Gaussian marginal together
     (2048, 128, 4, 2, 70, 0),      # h = 2048 (64 per thread, two passes)
     (6144, 512, 3, 4, 33, 0),      # h = 2048, k = 3
+    (1024, 256, 4, 4, 1, 0),       # h = 1024 tensor-core FWHT: one block, one token
+    (7168, 256, 3, 3, 37, 0),      # h = 1024 tensor-core FWHT: seven blocks (warps) per row
+    (5120, 768, 2, 2, 300, 0),     # h = 1024 tensor-core FWHT: 2-bit codebook
 ]
 
 
@@ -370,11 +386,13 @@ def test_host_buffer_pipeline(env, d_in, d_out, a_bits, w_bits, T, xdt):
         B.oq_linear_fused_host(layer, x_t, Wc, r)
 
 
-def test_degenerate_tokens(env):
+@pytest.mark.parametrize("d_in,d_out", [(256, 128), (1024, 256)])
+def test_degenerate_tokens(env, d_in, d_out):
     # a zero token (s = 0, every code L/2 - 1, y = 0) and tokens with very
-    # small and very large norms
+    # small and very large norms; d_in = 1024 takes the tensor-core FWHT on the
+    # fp16-level route
     torch, B = env
-    d_in, d_out, T = 256, 128, 6
+    T = 6
     x = W.bf16_bits_to_f32(W.custom_activations(T, d_in, seed=5))
     x[1] = 0.0
     x[2] *= 1e-12
@@ -383,12 +401,16 @@ def test_degenerate_tokens(env):
     x[4, 17] = -3.0                      # one-hot token
     x_np = W.f32_to_bf16_bits(x)
     Wm = W.custom_weights(d_out, d_in, seed=9)
-    _run_layer(env, d_in, d_out, 4, 4, x_np, Wm, label="degenerate")
+    _run_layer(env, d_in, d_out, 4, 4, x_np, Wm, label=f"degenerate {d_in}")
     layer = B.oq_layer_create(d_in, d_out, 0, 4, 4, 0)
     xt = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).cuda()
     codes, s = B.oq_rotate_quantize(layer, xt)
     c = O.unpack_codes(to_numpy_u32(codes), 4, d_in)
     assert float(s[1]) == 0.0 and np.all(c[1] == 7)
+    if d_out % 256 == 0:
+        a16, s2 = B.oq_rotate_quantize_levels(layer, xt)
+        mid = np.float16(layer.a_scale * O.lloyd_max(d_in, 4).levels[7]).view(np.uint16)
+        assert float(s2[1]) == 0.0 and np.all(a16[1].cpu().numpy().view(np.uint16) == mid)
 
 
 def test_empty_batch(env):
