@@ -95,6 +95,7 @@ void oq_layer_destroy(oq_layer* L) {
   cudaFree(L->bins_a.d_levels);
   cudaFree(L->bins_w.d_codes);
   cudaFree(L->bins_w.d_levels);
+  cudaFree(L->bins_a_full.d_levels);
   cudaFree(L->d_counters);
   cudaFree(L->d_error);
   delete L;
@@ -210,6 +211,24 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
     return st;
   }
 
+  // full-range activation table for the tensor-core rotate-quantize kernel
+  // (kept in shared memory: at most 2048 bins)
+  std::vector<uint32_t> taf_codes, taf_levels;
+  bool full_table = false;
+  if (L->h == 1024 && !signed_rot && d_in / 1024 <= 8) {
+    float kf = 0.f;
+    int b0f = 0, nbf = 0;
+    const std::string saved = g_last_error;   // a table too large for this use is not an error
+    if (build_bin_table(L->cb_a, d_in, L->h, lv_a, &kf, &b0f, &nbf, taf_codes, taf_levels, true) == OQ_OK &&
+        nbf <= 2048 && kf == L->bins_a.kscale) {
+      full_table = true;
+      L->bins_a_full.kscale = kf;
+      L->bins_a_full.b0 = b0f;
+      L->bins_a_full.nb = nbf;
+    }
+    g_last_error = saved;
+  }
+
   st = cuda_check(cudaMalloc(&L->d_gather_a, gather.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
   if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_gather_a, gather.data(), gather.size() * sizeof(uint16_t),
                                               cudaMemcpyHostToDevice), "upload gather");
@@ -239,6 +258,7 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   upload(&L->bins_a.d_levels, ta_levels);
   upload(&L->bins_w.d_codes, tw_codes);
   upload(&L->bins_w.d_levels, tw_levels);
+  if (full_table) upload(&L->bins_a_full.d_levels, taf_levels);
   if (st == OQ_OK && d_out % 128 == 0) {
     const size_t cb = (size_t)(d_out / 32) * sizeof(int);
     st = cuda_check(cudaMalloc(&L->d_counters, cb), "cudaMalloc(split counters)");
@@ -438,6 +458,9 @@ static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, in
   a.norms = s;
   a.err = L->d_error;
   a.gather_tc = L->d_gather_tc;
+  a.bins_full = L->bins_a_full.d_levels;
+  a.nb_full = L->bins_a_full.nb;
+  a.b0_full = L->bins_a_full.b0;
   if (rqtc_supported(a)) return rqtc_launch(a, stream);
   return rq_launch(a, stream);
 }

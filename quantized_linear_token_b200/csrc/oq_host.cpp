@@ -395,9 +395,12 @@ double choose_fp16_scale(const oq_codebook& cb) {
 // Threshold search table (see oq_bin_table): the smallest power of two K for
 // which consecutive scaled thresholds (as fp32, the values the kernel compares
 // against) lie more than one bin apart, then per bin the number of thresholds
-// in earlier bins and the one threshold inside it (+inf if none).
+// in earlier bins and the one threshold inside it (+inf if none).  With
+// full_range the bins cover every g a finite token can produce: |u| <= 1, so
+// |g| <= K sqrt(d), plus a margin for fp32 rounding of z and s; a kernel can
+// then index it without clamping.
 oq_status build_bin_table(const oq_codebook& cb, int d, int h, const uint16_t* lv16, float* kscale, int* b0, int* nb,
-                          std::vector<uint32_t>& codes, std::vector<uint32_t>& levels) {
+                          std::vector<uint32_t>& codes, std::vector<uint32_t>& levels, bool full_range) {
   const int L = 1 << cb.bits;
   const double sd = std::sqrt((double)d);
   auto bits_of = [](float f) {
@@ -412,7 +415,12 @@ oq_status build_bin_table(const oq_codebook& cb, int d, int h, const uint16_t* l
     bool apart = true;
     for (int j = 1; j < L - 1 && apart; ++j) apart = (double)tk[j] - (double)tk[j - 1] > 1.0;
     if (!apart) continue;
-    const int lo = (int)std::nearbyint(tk[0]) - 1, hi = (int)std::nearbyint(tk[L - 2]) + 1;
+    int lo = (int)std::nearbyint(tk[0]) - 1, hi = (int)std::nearbyint(tk[L - 2]) + 1;
+    if (full_range) {
+      const int bound = (int)std::ceil(K * sd * (1.0 + 1e-4)) + 2;
+      lo = std::min(lo, -bound);
+      hi = std::max(hi, bound);
+    }
     const int n = hi - lo + 1;
     if (n > OQ_MAX_BINS) break;
     codes.assign(2 * (size_t)n, 0u);

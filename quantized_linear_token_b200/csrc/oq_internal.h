@@ -45,6 +45,7 @@ struct oq_layer {
   uint16_t lv_a[256], lv_w[256];      // host copies of the two level tables
   int* d_error;                       // device error word
   oq_bin_table bins_a, bins_w;       // threshold search tables (activation / weight codebook)
+  oq_bin_table bins_a_full;           // activation table over the full range of g (levels only), or d_levels null
   int* d_counters;                    // split-K hand-off counters of the small-batch contraction (zero at rest)
   // host-buffer pipeline (oq_linear_fused_host): two copy streams and their
   // events, created on the first call (opaque CUDA handles)
@@ -70,7 +71,7 @@ double choose_fp8_scale(const oq_codebook& cb, double* worst);
 // threshold search table of a codebook (host copies; words interleaved TK, payload)
 constexpr int OQ_MAX_BINS = 4096;
 oq_status build_bin_table(const oq_codebook& cb, int d, int h, const uint16_t* lv16, float* kscale, int* b0, int* nb,
-                          std::vector<uint32_t>& codes, std::vector<uint32_t>& levels);
+                          std::vector<uint32_t>& codes, std::vector<uint32_t>& levels, bool full_range = false);
 
 // rotate + quantize launch (oq_rotate_quantize.cu): rows of `src` -> packed codes + norms
 struct RQArgs {
@@ -80,6 +81,8 @@ struct RQArgs {
   int d, h, log_h, bits;
   const uint16_t* gather;    // per-thread gather offsets (kernel order)
   const uint16_t* gather_tc; // offsets in the tensor-core kernel's order, or null
+  const uint32_t* bins_full; // full-range levels table (no clamping needed), or null
+  int nb_full, b0_full;
   const uint32_t* signmask;  // or null
   const uint32_t* bins;      // device threshold search table (codes, or levels for out16)
   int nb, b0;

@@ -67,6 +67,7 @@ struct TCParams {
   int* err;
   const uint2* bins;   // {threshold bits, fp16 level pair}
   int nb, b0;
+  int full;            // the table spans every g of a token with a normal fp32 norm
   float kscale;
 };
 
@@ -129,6 +130,37 @@ __device__ __forceinline__ void sumsq2(float& s0, float& s1, float a0, float a1)
 
 __device__ __forceinline__ uint32_t hbit(int r, int c) { return (__popc(r & c) & 1) ? 0xBF80u : 0x3F80u; }
 __device__ __forceinline__ uint32_t hbit32(int r, int c) { return (__popc(r & c) & 1) ? 0xBF800000u : 0x3F800000u; }
+
+// Quantizes the warp's 32 x 32 block Z (round-2 accumulators: rows a' =
+// 16 mt + g + 8 half, columns b' = 8 nt + 2q + {0, 1}) with the bin table and
+// stores the fp16 level pairs as words of the output row.
+template <bool CLAMP>
+__device__ __forceinline__ void quantize_store(const float (&D2)[2][4][4], float ks, float magic, int bin_lo,
+                                               int bin_hi, uint32_t tbl_shift, uint16_t* rowout, int g) {
+#pragma unroll
+  for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        float g0, g1, t0, t1;
+        mul2(g0, g1, D2[mt][nt][2 * half], D2[mt][nt][2 * half + 1], ks);
+        add2(t0, t1, g0, g1, magic);
+        int m0 = __float_as_int(t0), m1 = __float_as_int(t1);
+        if (CLAMP) {
+          m0 = min(max(m0, bin_lo), bin_hi);
+          m1 = min(max(m1, bin_lo), bin_hi);
+        }
+        const uint2 e0 = lds_v2(tbl_shift + 8u * (uint32_t)m0);
+        const uint2 e1 = lds_v2(tbl_shift + 8u * (uint32_t)m1);
+        // byte selector: bytes 0-1 from e0's level pair (upper level if g0 is
+        // above the bin's threshold), bytes 2-3 likewise from e1's
+        const uint32_t sel = 0x5410u | (gt_mask(g0, __uint_as_float(e0.x)) & 0x22u) |
+                             (gt_mask(g1, __uint_as_float(e1.x)) & 0x2200u);
+        const int a = 16 * mt + g + 8 * half;
+        *reinterpret_cast<uint32_t*>(rowout + 32 * a + 8 * nt) = __byte_perm(e0.y, e1.y, sel);
+      }
+}
 
 __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -292,26 +324,14 @@ __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCPar
     // (the bin-table search of rq_kernel), fp16 level pairs stored as words
     const float ks = (s > 0.f) ? p.kscale / s : 0.f;
     uint16_t* rowout = p.out16 + (size_t)t * p.d + (size_t)warp * 1024 + 2 * q;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int half = 0; half < 2; ++half)
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          float g0, g1, t0, t1;
-          mul2(g0, g1, D2[mt][nt][2 * half], D2[mt][nt][2 * half + 1], ks);
-          add2(t0, t1, g0, g1, magic);
-          const int m0 = min(max(__float_as_int(t0), bin_lo), bin_hi);
-          const int m1 = min(max(__float_as_int(t1), bin_lo), bin_hi);
-          const uint2 e0 = lds_v2(tbl_shift + 8u * (uint32_t)m0);
-          const uint2 e1 = lds_v2(tbl_shift + 8u * (uint32_t)m1);
-          // byte selector: bytes 0-1 from e0's level pair (upper level if g0
-          // is above the bin's threshold), bytes 2-3 likewise from e1's
-          const uint32_t sel = 0x5410u | (gt_mask(g0, __uint_as_float(e0.x)) & 0x22u) |
-                               (gt_mask(g1, __uint_as_float(e1.x)) & 0x2200u);
-          const int a = 16 * mt + g + 8 * half;
-          *reinterpret_cast<uint32_t*>(rowout + 32 * a + 8 * nt) = __byte_perm(e0.y, e1.y, sel);
-        }
+    // With a full-range table every finite g of a token whose squared norm is
+    // a normal fp32 number lies inside it (|g| <= K sqrt(d) up to rounding),
+    // so the bin index needs no clamp.  Other tokens (a norm that under- or
+    // overflowed in fp32, non-finite values, zero) take the clamped search.
+    if (p.full && s2 >= 1e-30f && s2 <= 1e30f)
+      quantize_store<false>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+    else
+      quantize_store<true>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
     if (tid == 0) p.norms[t] = s;
   }
 }
@@ -337,12 +357,19 @@ oq_status rqtc_launch(const RQArgs& a, void* stream) {
   p.out16 = a.out16;
   p.norms = a.norms;
   p.err = a.err;
-  p.bins = reinterpret_cast<const uint2*>(a.bins);
-  p.nb = a.nb;
-  p.b0 = a.b0;
+  if (a.bins_full) {
+    p.bins = reinterpret_cast<const uint2*>(a.bins_full);
+    p.nb = a.nb_full;
+    p.b0 = a.b0_full;
+    p.full = 1;
+  } else {
+    p.bins = reinterpret_cast<const uint2*>(a.bins);
+    p.nb = a.nb;
+    p.b0 = a.b0;
+  }
   p.kscale = a.kscale;
   const int threads = p.nw * 32;
-  const size_t gtab_off = (80 + 8 * (size_t)a.nb + 15) & ~(size_t)15;
+  const size_t gtab_off = (80 + 8 * (size_t)p.nb + 15) & ~(size_t)15;
   const size_t smem = ((gtab_off + 64 * (size_t)threads + 127) & ~(size_t)127) + 2 * (size_t)p.stage_bytes;
   cudaError_t e = cudaFuncSetAttribute(rqtc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e == cudaSuccess)
