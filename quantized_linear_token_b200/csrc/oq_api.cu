@@ -215,7 +215,8 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   // (kept in shared memory: at most 2048 bins)
   std::vector<uint32_t> taf_codes, taf_levels;
   bool full_table = false;
-  if (L->h == 1024 && !signed_rot && d_in / 1024 <= 8) {
+  const bool tc_rq = ((L->h == 1024 && d_in / L->h <= 8) || (L->h == 512 && d_in / L->h <= 32)) && !signed_rot;
+  if (tc_rq) {
     float kf = 0.f;
     int b0f = 0, nbf = 0;
     const std::string saved = g_last_error;   // a table too large for this use is not an error
@@ -232,9 +233,9 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   st = cuda_check(cudaMalloc(&L->d_gather_a, gather.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
   if (st == OQ_OK) st = cuda_check(cudaMemcpy(L->d_gather_a, gather.data(), gather.size() * sizeof(uint16_t),
                                               cudaMemcpyHostToDevice), "upload gather");
-  if (st == OQ_OK && L->h == 1024 && !signed_rot && d_in / 1024 <= 8) {
+  if (st == OQ_OK && tc_rq) {
     std::vector<uint16_t> gather_tc;
-    rqtc_build_gather(d_in, L->perm_host, gather_tc);
+    rqtc_build_gather(d_in, L->h, L->perm_host, gather_tc);
     st = cuda_check(cudaMalloc(&L->d_gather_tc, gather_tc.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
     if (st == OQ_OK)
       st = cuda_check(cudaMemcpy(L->d_gather_tc, gather_tc.data(), gather_tc.size() * sizeof(uint16_t),
@@ -461,7 +462,10 @@ static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, in
   a.bins_full = L->bins_a_full.d_levels;
   a.nb_full = L->bins_a_full.nb;
   a.b0_full = L->bins_a_full.b0;
-  if (rqtc_supported(a)) return rqtc_launch(a, stream);
+  if (rqtc_supported(a)) {
+    const oq_status st = rqtc_launch(a, stream);
+    if (st != OQ_ERR_UNSUPPORTED) return st;   // else (shared memory too small): the two-pass kernel
+  }
   return rq_launch(a, stream);
 }
 

@@ -38,7 +38,7 @@ struct oq_layer {
   std::vector<int8_t> signs_host;     // +-1 by rotated position (OQ_FLAG_SIGNS)
   // device tables (owned)
   uint16_t* d_gather_a;               // rotate-quantize gather offsets, kernel order
-  uint16_t* d_gather_tc;              // the same for the tensor-core FWHT kernel (h = 1024), or null
+  uint16_t* d_gather_tc;              // the same for the tensor-core FWHT kernel (h = 1024 or 512), or null
   uint32_t* d_signmask;               // sign bits in kernel order, or null
   uint16_t* d_levels_a;               // fp16 bits of a_scale * activation levels
   uint16_t* d_levels_w;               // fp16 bits of w_scale * weight levels
@@ -97,9 +97,9 @@ int rq_elems_per_thread(int h);
 void rq_build_gather(int d, int h, const std::vector<uint32_t>& perm, const std::vector<int8_t>* signs,
                      std::vector<uint16_t>& gather, std::vector<uint32_t>& signmask);
 oq_status rq_launch(const RQArgs& a, void* stream);
-// rotate-quantize with the block FWHT on the tensor cores (h = 1024, bf16
-// input, fp16-level output, no signs; oq_rotate_quantize_tc.cu)
-void rqtc_build_gather(int d, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather);
+// rotate-quantize with the block FWHT on the tensor cores (h = 1024 or 512,
+// bf16 input, fp16-level output, no signs; oq_rotate_quantize_tc.cu)
+void rqtc_build_gather(int d, int h, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather);
 bool rqtc_supported(const RQArgs& a);
 oq_status rqtc_launch(const RQArgs& a, void* stream);
 

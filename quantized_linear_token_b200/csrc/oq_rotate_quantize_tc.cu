@@ -1,18 +1,18 @@
 // Rotate + quantize with the block Walsh-Hadamard transform on the tensor
-// cores, for blocks of h = 1024 and bf16 activations, writing the fp16 levels
+// cores, for blocks of h = 1024 or 512 and bf16 activations, writing the fp16 levels
 // of the codes (the A operand of the fused layer call).  Same arithmetic
 // contract as rq_kernel (gecl notes Method 1, 3, 4; pith Supplementary A):
 //   s = ||x||_2,  y = P_pi x,  z_j = H_h y_j (block j, unnormalised),
 //   code_i = #{k : t_k < z_i / (s sqrt(h))},  output fp16(a_scale C[code_i]).
 //
-// Sylvester's H_1024 is H_32 (x) H_32: with a block viewed as a 32 x 32
-// matrix Y[a][b] = y[32 a + b], its transform is Z = H_32 Y H_32.  One warp
-// owns one block and computes it with two rounds of warp-level MMAs
-// (m16n8k16, bf16 operands, fp32 accumulate):
-//   round 1: P^T = H_32 Y^T.  The B operand is Y^T, gathered through pi
+// Sylvester's H_h is H_A (x) H_32 (A = h / 32 = 32 or 16): with a block
+// viewed as an A x 32 matrix Y[a][b] = y[32 a + b], its transform is
+// Z = H_A Y H_32.  One warp owns one block and computes it with two rounds of
+// warp-level MMAs:
+//   round 1: P^T = H_32 Y^T (m16n8k16, bf16 operands, fp32 accumulate).  The B operand is Y^T, gathered through pi
 //            straight into the fragment registers: bf16 inputs and +-1
 //            entries, so the products are exact.
-//   round 2: Z = H_32 P.  The accumulator layout of round 1 already holds,
+//   round 2: Z = H_A P.  The accumulator layout of round 1 already holds,
 //            in every lane, the pairs of P that its round-2 B fragments need,
 //            so P never leaves the registers.  P is fp32; it enters as two
 //            tf32 terms, hi = P with its low 13 mantissa bits cleared and
@@ -22,7 +22,7 @@
 //            chosen to match the pairs a lane holds).
 // The norm comes from round 1: sum P^2 = 32 sum y^2 per block.  Then every
 // coordinate is quantized with the same bin-table search as rq_kernel and its
-// fp16 level stored.  One CTA = d / 1024 warps = one row at a time; rows
+// fp16 level stored.  One CTA = d / h warps = one row at a time; rows
 // stream through shared memory with double-buffered bulk copies.
 #include <cuda_bf16.h>
 
@@ -34,23 +34,24 @@
 
 namespace oq {
 
-// Gather table of the tensor-core kernel: entry (w * 32 + lane) * 32 + e is
-// the byte offset (2 x the input channel) of in-block position 32 a + b of
-// block w in the staged bf16 row, with
-// e = (kt * 4 + nt) * 4 + i, a = 8 nt + lane / 4 and
+// Gather table of the tensor-core kernel (block size h, A = h / 32 values per
+// lane): entry (w * 32 + lane) * A + e is the byte offset (2 x the input
+// channel) of in-block position 32 a + b of block w in the staged bf16 row,
+// with e = (kt * A / 8 + nt) * 4 + i, a = 8 nt + lane / 4 and
 // b = 16 kt + 2 (lane % 4) + {0, 1, 8, 9}[i]: the order in which a lane fills
 // its round-1 B fragments.
-void rqtc_build_gather(int d, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather) {
+void rqtc_build_gather(int d, int h, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather) {
   static const int boff[4] = {0, 1, 8, 9};
+  const int A = h / 32, NT = A / 8;
   gather.assign((size_t)d, 0);
-  for (int w = 0; w < d / 1024; ++w)
+  for (int w = 0; w < d / h; ++w)
     for (int lane = 0; lane < 32; ++lane)
       for (int kt = 0; kt < 2; ++kt)
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
           for (int i = 0; i < 4; ++i) {
             const int a = 8 * nt + lane / 4, b = 16 * kt + 2 * (lane % 4) + boff[i];
-            const int e = (kt * 4 + nt) * 4 + i;
-            gather[((size_t)w * 32 + lane) * 32 + e] = (uint16_t)(2 * perm[(size_t)w * 1024 + 32 * a + b]);
+            const int e = (kt * NT + nt) * 4 + i;
+            gather[((size_t)w * 32 + lane) * A + e] = (uint16_t)(2 * perm[(size_t)w * h + 32 * a + b]);
           }
 }
 
@@ -59,7 +60,7 @@ namespace {
 struct TCParams {
   const void* src;     // [rows, d] bf16
   int64_t rows;
-  int d, nw;           // nw = d / 1024 warps per CTA
+  int d, nw;           // nw = d / h warps per CTA
   int stage_bytes;     // per row buffer
   const uint16_t* gather;
   uint16_t* out16;     // fp16 levels [rows, d]
@@ -131,14 +132,14 @@ __device__ __forceinline__ void sumsq2(float& s0, float& s1, float a0, float a1)
 __device__ __forceinline__ uint32_t hbit(int r, int c) { return (__popc(r & c) & 1) ? 0xBF80u : 0x3F80u; }
 __device__ __forceinline__ uint32_t hbit32(int r, int c) { return (__popc(r & c) & 1) ? 0xBF800000u : 0x3F800000u; }
 
-// Quantizes the warp's 32 x 32 block Z (round-2 accumulators: rows a' =
+// Quantizes the warp's A x 32 block Z (round-2 accumulators: rows a' =
 // 16 mt + g + 8 half, columns b' = 8 nt + 2q + {0, 1}) with the bin table and
 // stores the fp16 level pairs as words of the output row.
-template <bool CLAMP>
-__device__ __forceinline__ void quantize_store(const float (&D2)[2][4][4], float ks, float magic, int bin_lo,
+template <bool CLAMP, int MT2>
+__device__ __forceinline__ void quantize_store(const float (&D2)[MT2][4][4], float ks, float magic, int bin_lo,
                                                int bin_hi, uint32_t tbl_shift, uint16_t* rowout, int g) {
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
+  for (int mt = 0; mt < MT2; ++mt)
 #pragma unroll
     for (int half = 0; half < 2; ++half)
 #pragma unroll
@@ -162,24 +163,28 @@ __device__ __forceinline__ void quantize_store(const float (&D2)[2][4][4], float
       }
 }
 
-__global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCParams p) {
+// A = rows of the block matrix (h / 32): NT1 = A / 8 round-1 column tiles,
+// MT2 = A / 16 round-2 row tiles
+template <int A>
+__global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid_constant__ TCParams p) {
+  constexpr int NT1 = A / 8, MT2 = A / 16, H = 32 * A;
   extern __shared__ __align__(128) unsigned char smem[];
   const int nw = p.nw, nthreads = nw * 32;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, q = lane & 3, g = lane >> 2;
 
-  // shared memory: mbarriers | norm partials [2][8] | threshold table |
-  // gather offsets [4][threads] (uint4) | two row buffers
+  // shared memory: mbarriers | norm partials [2][32] | threshold table |
+  // gather offsets [A / 8][threads] (uint4) | two row buffers
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem);
   float* red = reinterpret_cast<float*>(smem + 16);
-  uint2* tbl = reinterpret_cast<uint2*>(smem + 80);
-  const int gtab_off = (80 + 8 * p.nb + 15) & ~15;
+  uint2* tbl = reinterpret_cast<uint2*>(smem + 272);
+  const int gtab_off = (272 + 8 * p.nb + 15) & ~15;
   uint4* gtab = reinterpret_cast<uint4*>(smem + gtab_off);
-  unsigned char* stage = smem + ((gtab_off + 64 * nthreads + 127) & ~127);
+  unsigned char* stage = smem + ((gtab_off + 2 * A * nthreads + 127) & ~127);
   const uint32_t stage_addr0 = smem_u32(stage);
 
-  for (int i = tid; i < 4 * nthreads; i += nthreads) {
+  for (int i = tid; i < (A / 8) * nthreads; i += nthreads) {
     const int t = i % nthreads, qq = i / nthreads;
-    gtab[i] = __ldg(reinterpret_cast<const uint4*>(p.gather) + (size_t)t * 4 + qq);
+    gtab[i] = __ldg(reinterpret_cast<const uint4*>(p.gather) + (size_t)t * (A / 8) + qq);
   }
   for (int i = tid; i < p.nb; i += nthreads) tbl[i] = __ldg(p.bins + i);
   if (tid == 0) {
@@ -234,9 +239,9 @@ __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCPar
     const uint32_t sa = stage_addr0 + (uint32_t)(buf * p.stage_bytes);
 
     // ---- gather through pi into round-1 B fragments (bf16 pairs)
-    uint32_t B1[2][4][2];
+    uint32_t B1[2][NT1][2];
 #pragma unroll
-    for (int qq = 0; qq < 4; ++qq) {
+    for (int qq = 0; qq < A / 8; ++qq) {
       const uint4 gq = gtab[qq * nthreads + tid];
       const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
 #pragma unroll
@@ -244,24 +249,24 @@ __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCPar
         uint16_t v0, v1;
         asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v0) : "r"(sa + (gw[hpair] & 0xFFFFu)));
         asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v1) : "r"(sa + (gw[hpair] >> 16)));
-        // slots e = 8 qq + 2 hpair, +1: (kt, nt) = divmod(2 qq + hpair / 2, 4), register hpair % 2
-        const int kn = 2 * qq + (hpair >> 1), kt = kn >> 2, nt = kn & 3;
+        // slots e = 8 qq + 2 hpair, +1: (kt, nt) = divmod(2 qq + hpair / 2, NT1), register hpair % 2
+        const int kn = 2 * qq + (hpair >> 1), kt = kn / NT1, nt = kn % NT1;
         B1[kt][nt][hpair & 1] = (uint32_t)v0 | ((uint32_t)v1 << 16);
       }
     }
 
     // ---- round 1: P^T = H_32 Y^T (rows b', columns a)
-    float D1[2][4][4];
+    float D1[2][NT1][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+      for (int nt = 0; nt < NT1; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) D1[mt][nt][i] = 0.f;
 #pragma unroll
     for (int kt = 0; kt < 2; ++kt)
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
+      for (int nt = 0; nt < NT1; ++nt)
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) mma_bf16_16816(D1[mt][nt], (mt & kt) ? hn : hp, B1[kt][nt][0], B1[kt][nt][1]);
 
@@ -270,28 +275,28 @@ __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCPar
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
+      for (int nt = 0; nt < NT1; ++nt) {
         sumsq2(ss0, ss1, D1[mt][nt][0], D1[mt][nt][1]);
         sumsq2(ss0, ss1, D1[mt][nt][2], D1[mt][nt][3]);
       }
     float ss = ss0 + ss1;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if (lane == 0) red[buf * 8 + warp] = ss;
+    if (lane == 0) red[buf * 32 + warp] = ss;
 
     // ---- round 2: Z = H_32 P in tf32, P as hi + lo.  K tile nt of the
     // contraction over a takes a = 8 nt + 2q + {0, 1} from lane (g, q): the
     // pair D1[mt][nt][2h], D1[mt][nt][2h + 1] = P[8 nt + 2q + {0, 1}][16 mt + g
     // + 8 h] is the B fragment of (k tile nt, n tile 2 mt + h).
-    float D2[2][4][4];
+    float D2[MT2][4][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mt = 0; mt < MT2; ++mt)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i) D2[mt][nt][i] = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < NT1; ++nt)
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -302,7 +307,7 @@ __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCPar
           sub2(lo0, lo1, x0, x1, __uint_as_float(hi0), __uint_as_float(hi1));
           const int nt2 = 2 * mt + h;
 #pragma unroll
-          for (int mt2 = 0; mt2 < 2; ++mt2) {
+          for (int mt2 = 0; mt2 < MT2; ++mt2) {
             const bool na = mt2 & (nt >> 1), nh = na ^ (nt & 1);
             const uint32_t a0 = na ? un : u, a1 = nh ? un : u, a2 = na ? vn : v, a3 = nh ? vn : v;
             mma_tf32_1688(D2[mt2][nt2], a0, a1, a2, a3, hi0, hi1);
@@ -317,21 +322,21 @@ __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCPar
       break;
     }
     float s2 = 0.f;
-    for (int w = 0; w < nw; ++w) s2 += red[buf * 8 + w];
+    for (int w = 0; w < nw; ++w) s2 += red[buf * 32 + w];
     const float s = sqrtf(s2 * (1.0f / 32.0f));
 
     // ---- quantize: Z[a'][b'] for a' = 16 mt + g + 8 half, b' = 8 nt + 2q + {0, 1}
     // (the bin-table search of rq_kernel), fp16 level pairs stored as words
     const float ks = (s > 0.f) ? p.kscale / s : 0.f;
-    uint16_t* rowout = p.out16 + (size_t)t * p.d + (size_t)warp * 1024 + 2 * q;
+    uint16_t* rowout = p.out16 + (size_t)t * p.d + (size_t)warp * H + 2 * q;
     // With a full-range table every finite g of a token whose squared norm is
     // a normal fp32 number lies inside it (|g| <= K sqrt(d) up to rounding),
     // so the bin index needs no clamp.  Other tokens (a norm that under- or
     // overflowed in fp32, non-finite values, zero) take the clamped search.
     if (p.full && s2 >= 1e-30f && s2 <= 1e30f)
-      quantize_store<false>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+      quantize_store<false, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
     else
-      quantize_store<true>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+      quantize_store<true, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
     if (tid == 0) p.norms[t] = s;
   }
 }
@@ -339,8 +344,38 @@ __global__ void __launch_bounds__(256) rqtc_kernel(const __grid_constant__ TCPar
 }  // namespace
 
 bool rqtc_supported(const RQArgs& a) {
-  return a.out16 && a.h == 1024 && a.src_dtype == OQ_DTYPE_BF16 && !a.signmask && a.gather_tc &&
-         a.d % 1024 == 0 && a.d / 1024 >= 1 && a.d / 1024 <= 8 && a.nb >= 1 && a.nb <= OQ_MAX_BINS;
+  return a.out16 && (a.h == 1024 || a.h == 512) && a.src_dtype == OQ_DTYPE_BF16 && !a.signmask && a.gather_tc &&
+         a.d % a.h == 0 && a.d / a.h >= 1 && a.d / a.h <= (a.h == 1024 ? 8 : 32) && a.nb >= 1 &&
+         a.nb <= OQ_MAX_BINS;
+}
+
+template <int A>
+static oq_status rqtc_launch_t(const TCParams& p, void* stream) {
+  const int threads = p.nw * 32;
+  const size_t gtab_off = (272 + 8 * (size_t)p.nb + 15) & ~(size_t)15;
+  const size_t smem = ((gtab_off + 2 * A * (size_t)threads + 127) & ~(size_t)127) + 2 * (size_t)p.stage_bytes;
+  if (smem > 227 * 1024) return OQ_ERR_UNSUPPORTED;
+  auto kern = rqtc_kernel<A>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) {
+    set_error(std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
+    return OQ_ERR_CUDA;
+  }
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem);
+  if (per_sm < 1) per_sm = 1;
+  const int64_t grid = std::min<int64_t>(p.rows, (int64_t)sms * per_sm);
+  kern<<<(unsigned)grid, threads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error(std::string("rotate_quantize (tensor-core FWHT) launch: ") + cudaGetErrorString(e));
+    return OQ_ERR_CUDA;
+  }
+  return OQ_OK;
 }
 
 oq_status rqtc_launch(const RQArgs& a, void* stream) {
@@ -351,7 +386,7 @@ oq_status rqtc_launch(const RQArgs& a, void* stream) {
   p.src = a.src;
   p.rows = a.rows;
   p.d = a.d;
-  p.nw = a.d / 1024;
+  p.nw = a.d / a.h;
   p.stage_bytes = (a.d * 2 + 127) & ~127;
   p.gather = a.gather_tc;
   p.out16 = a.out16;
@@ -368,30 +403,7 @@ oq_status rqtc_launch(const RQArgs& a, void* stream) {
     p.b0 = a.b0;
   }
   p.kscale = a.kscale;
-  const int threads = p.nw * 32;
-  const size_t gtab_off = (80 + 8 * (size_t)p.nb + 15) & ~(size_t)15;
-  const size_t smem = ((gtab_off + 64 * (size_t)threads + 127) & ~(size_t)127) + 2 * (size_t)p.stage_bytes;
-  cudaError_t e = cudaFuncSetAttribute(rqtc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(rqtc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) {
-    set_error(std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-    return OQ_ERR_CUDA;
-  }
-  int dev = 0, sms = 0, per_sm = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rqtc_kernel, threads, smem);
-  if (per_sm < 1) per_sm = 1;
-  const int64_t grid = std::min<int64_t>(a.rows, (int64_t)sms * per_sm);
-  rqtc_kernel<<<(unsigned)grid, threads, smem, static_cast<cudaStream_t>(stream)>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    set_error(std::string("rotate_quantize (tensor-core FWHT) launch: ") + cudaGetErrorString(e));
-    return OQ_ERR_CUDA;
-  }
-  return OQ_OK;
+  return a.h == 1024 ? rqtc_launch_t<32>(p, stream) : rqtc_launch_t<16>(p, stream);
 }
 
 }  // namespace oq

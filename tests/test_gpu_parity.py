@@ -208,6 +208,8 @@ EDGE = [
     (1024, 256, 4, 4, 1, 0),       # h = 1024 tensor-core FWHT: one block, one token
     (7168, 256, 3, 3, 37, 0),      # h = 1024 tensor-core FWHT: seven blocks (warps) per row
     (5120, 768, 2, 2, 300, 0),     # h = 1024 tensor-core FWHT: 2-bit codebook
+    (512, 256, 3, 3, 17, 0),       # h = 512 tensor-core FWHT (H_16 x H_32): one block
+    (1536, 256, 4, 4, 130, 2),     # h = 512 tensor-core FWHT: three blocks, Gaussian-marginal codebook
 ]
 
 
