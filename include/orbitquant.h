@@ -245,7 +245,7 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  *   a16  device [T, d_in] uint16 (fp16 bits), 16-byte aligned.
  *   s    device [T] fp32 token norms.
  * For h = 1024 without OQ_FLAG_SIGNS the block transform runs on the tensor
- * cores (H_1024 = H_32 (x) H_32 as two rounds of warp MMAs, the second on a
+ * cores (H_1024 = H_32 (x) H_32 as two passes of warp MMAs, the second on a
  * two-term tf32 split of the fp32 intermediate): its fp32 rounding differs
  * from oq_rotate_quantize's, so a code may differ from that call's where the
  * coordinate lies within rounding of a decision threshold, and s may differ

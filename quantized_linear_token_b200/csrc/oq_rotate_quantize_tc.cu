@@ -7,20 +7,21 @@
 //
 // Sylvester's H_h is H_A (x) H_32 (A = h / 32 = 32 or 16): with a block
 // viewed as an A x 32 matrix Y[a][b] = y[32 a + b], its transform is
-// Z = H_A Y H_32.  One warp owns one block and computes it with two rounds of
+// Z = H_A Y H_32.  One warp owns one block and computes it with two passes of
 // warp-level MMAs:
-//   round 1: P^T = H_32 Y^T (m16n8k16, bf16 operands, fp32 accumulate).  The B operand is Y^T, gathered through pi
-//            straight into the fragment registers: bf16 inputs and +-1
-//            entries, so the products are exact.
-//   round 2: Z = H_A P.  The accumulator layout of round 1 already holds,
-//            in every lane, the pairs of P that its round-2 B fragments need,
+//   pass 1: P^T = H_32 Y^T (m16n8k16, bf16 operands, fp32 accumulate).
+//            The B operand is Y^T, gathered through pi straight into the
+//            fragment registers: bf16 inputs and +-1 entries, so the
+//            products are exact.
+//   pass 2: Z = H_A P.  The accumulator layout of pass 1 already holds,
+//            in every lane, the pairs of P that its pass-2 B fragments need,
 //            so P never leaves the registers.  P is fp32; it enters as two
 //            tf32 terms, hi = P with its low 13 mantissa bits cleared and
 //            lo = P - hi (which the tensor core reads to 11 bits), so the
 //            operand is P to 2^-20 of its value; both products accumulate
 //            into the same fp32 result (m16n8k8 tf32 MMAs, whose K order is
 //            chosen to match the pairs a lane holds).
-// The norm comes from round 1: sum P^2 = 32 sum y^2 per block.  Then every
+// The norm comes from pass 1: sum P^2 = 32 sum y^2 per block.  Then every
 // coordinate is quantized with the same bin-table search as rq_kernel and its
 // fp16 level stored.  One CTA = d / h warps = one row at a time; rows
 // stream through shared memory with double-buffered bulk copies.
@@ -39,7 +40,7 @@ namespace oq {
 // channel) of in-block position 32 a + b of block w in the staged bf16 row,
 // with e = (kt * A / 8 + nt) * 4 + i, a = 8 nt + lane / 4 and
 // b = 16 kt + 2 (lane % 4) + {0, 1, 8, 9}[i]: the order in which a lane fills
-// its round-1 B fragments.
+// its pass-1 B fragments.
 void rqtc_build_gather(int d, int h, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather) {
   static const int boff[4] = {0, 1, 8, 9};
   const int A = h / 32, NT = A / 8;
@@ -132,7 +133,7 @@ __device__ __forceinline__ void sumsq2(float& s0, float& s1, float a0, float a1)
 __device__ __forceinline__ uint32_t hbit(int r, int c) { return (__popc(r & c) & 1) ? 0xBF80u : 0x3F80u; }
 __device__ __forceinline__ uint32_t hbit32(int r, int c) { return (__popc(r & c) & 1) ? 0xBF800000u : 0x3F800000u; }
 
-// Quantizes the warp's A x 32 block Z (round-2 accumulators: rows a' =
+// Quantizes the warp's A x 32 block Z (pass-2 accumulators: rows a' =
 // 16 mt + g + 8 half, columns b' = 8 nt + 2q + {0, 1}) with the bin table and
 // stores the fp16 level pairs as words of the output row.
 template <bool CLAMP, int MT2>
@@ -163,8 +164,8 @@ __device__ __forceinline__ void quantize_store(const float (&D2)[MT2][4][4], flo
       }
 }
 
-// A = rows of the block matrix (h / 32): NT1 = A / 8 round-1 column tiles,
-// MT2 = A / 16 round-2 row tiles
+// A = rows of the block matrix (h / 32): NT1 = A / 8 pass-1 column tiles,
+// MT2 = A / 16 pass-2 row tiles
 template <int A>
 __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid_constant__ TCParams p) {
   constexpr int NT1 = A / 8, MT2 = A / 16, H = 32 * A;
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
   hp[3] = hbit(g + 8, 2 * q + 8) | hbit(g + 8, 2 * q + 9) << 16;
 #pragma unroll
   for (int i = 0; i < 4; ++i) hn[i] = hp[i] ^ 0x80008000u;
-  // round 2 (tf32, K order of k-tile nt: k = q <-> a = 8 nt + 2q, k = q + 4
+  // pass 2 (tf32, K order of k-tile nt: k = q <-> a = 8 nt + 2q, k = q + 4
   // <-> a = 8 nt + 2q + 1): A[a'][k] = H_32[a'][a].  For rows a' = 16 mt + g
   // + 8 h the sign is sgn(g & a) times (-1)^(mt & nt >> 1) times (-1)^(h &
   // nt & 1), so four values cover every fragment.
@@ -238,7 +239,7 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
     const bool ok = mbar_wait(&mbar[buf], (uint32_t)(it >> 1) & 1u, p.err);
     const uint32_t sa = stage_addr0 + (uint32_t)(buf * p.stage_bytes);
 
-    // ---- gather through pi into round-1 B fragments (bf16 pairs)
+    // ---- gather through pi into pass-1 B fragments (bf16 pairs)
     uint32_t B1[2][NT1][2];
 #pragma unroll
     for (int qq = 0; qq < A / 8; ++qq) {
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
       }
     }
 
-    // ---- round 1: P^T = H_32 Y^T (rows b', columns a)
+    // ---- pass 1: P^T = H_32 Y^T (rows b', columns a)
     float D1[2][NT1][4];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt)
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
     for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if (lane == 0) red[buf * 32 + warp] = ss;
 
-    // ---- round 2: Z = H_32 P in tf32, P as hi + lo.  K tile nt of the
+    // ---- pass 2: Z = H_A P in tf32, P as hi + lo.  K tile nt of the
     // contraction over a takes a = 8 nt + 2q + {0, 1} from lane (g, q): the
     // pair D1[mt][nt][2h], D1[mt][nt][2h + 1] = P[8 nt + 2q + {0, 1}][16 mt + g
     // + 8 h] is the B fragment of (k tile nt, n tile 2 mt + h).

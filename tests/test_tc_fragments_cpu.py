@@ -1,9 +1,9 @@
 """The index algebra of the tensor-core block transform, on the CPU.
 
 The rotate-quantize kernel for h = 512 and 1024 computes z = H_h y of one
-block as Z = H_A Y H_32 (Y[a][b] = y[32 a + b], A = h / 32) with two rounds of
-warp MMAs, and feeds round 1's accumulator registers to round 2 as B
-fragments after choosing round 2's K order to match.  This emulates those
+block as Z = H_A Y H_32 (Y[a][b] = y[32 a + b], A = h / 32) with two passes of
+warp MMAs, and feeds pass 1's accumulator registers to pass 2 as B
+fragments after choosing pass 2's K order to match.  This emulates those
 fragment layouts (the m16n8k16 and m16n8k8 register maps of the PTX warp MMA
 instructions) lane by lane in numpy and checks that the assembled result is
 the Sylvester transform of the flattened block.  It pins the derivation the
@@ -20,11 +20,11 @@ def _hb(r: int, c: int) -> float:
 
 
 @pytest.mark.parametrize("A", [16, 32])
-def test_two_round_fragment_transform(A):
+def test_two_pass_fragment_transform(A):
     NT1, MT2 = A // 8, A // 16
     Y = np.random.default_rng(A).standard_normal((A, 32))
     H32, HA = O.sylvester_hadamard(32), O.sylvester_hadamard(A)
-    # round 1: P^T = H_32 Y^T; lane (g, q) of tile (kt, nt) holds Y[8nt + g][16kt + 2q + 8r + {0, 1}]
+    # pass 1: P^T = H_32 Y^T; lane (g, q) of tile (kt, nt) holds Y[8nt + g][16kt + 2q + 8r + {0, 1}]
     D1 = {}
     for mt in range(2):
         for nt in range(NT1):
@@ -40,7 +40,7 @@ def test_two_round_fragment_transform(A):
             for lane in range(32):
                 g, q = lane >> 2, lane & 3
                 D1[lane, mt, nt] = (acc[g][2 * q], acc[g][2 * q + 1], acc[g + 8][2 * q], acc[g + 8][2 * q + 1])
-    # round 2: Z = H_A P, k tile nt with k = q <-> a = 8nt + 2q and k = q + 4 <-> a = 8nt + 2q + 1
+    # pass 2: Z = H_A P, k tile nt with k = q <-> a = 8nt + 2q and k = q + 4 <-> a = 8nt + 2q + 1
     z = O.sylvester_hadamard(32 * A) @ Y.reshape(-1)
     for mt2 in range(MT2):
         for nt2 in range(4):
