@@ -219,6 +219,9 @@ def run_ours(args):
     B.load_library()
 
     wl = W.WORKLOADS[args.workload]
+    if wl.x_dtype != "bf16":
+        raise SystemExit(f"bench.py times bf16-activation workloads; {args.workload} ({wl.x_dtype} activations) "
+                         "is a parity case of the tests")
     lay = next(l for l in wl.layers if l.name == args.layer) if args.layer else wl.layers[0]
     T, d, dout = (args.tokens or wl.tokens), lay.d_in, lay.d_out
     x_np = rank_batch(wl, d, T, rank)
@@ -401,10 +404,7 @@ def run_ours(args):
         "dtype": "f16",
         "data": "synthetic",
         "config": {
-            "workload": f"{args.workload}: {wl.title}", "layer": lay.name,
-            "tokens_per_gpu": T, "d_in": d, "d_out": dout, "a_bits": lay.a_bits, "w_bits": lay.w_bits,
-            "h": d & -d, "x_dtype": "bf16", "y_dtype": "fp32",
-            "parallelism": f"token-sharded x{world}, weights replicated",
+            **workload_config(args, wl, lay, T, world),
             "l2": "flushed (256 MiB write) before every step, outside the timed events",
             "step": "one oq_linear_fused call (x -> y: " + steps_desc[route].split(" (")[0] + ")",
         },
@@ -465,6 +465,16 @@ def run_ours(args):
 
 
 # ------------------------------------------------------------------ reference arm
+def workload_config(args, wl, lay, T, world):
+    """The config keys both arms report for one workload and layer."""
+    return {
+        "workload": f"{args.workload}: {wl.title}", "layer": lay.name,
+        "tokens_per_gpu": T, "d_in": lay.d_in, "d_out": lay.d_out, "a_bits": lay.a_bits, "w_bits": lay.w_bits,
+        "h": lay.d_in & -lay.d_in, "x_dtype": wl.x_dtype, "y_dtype": "fp32",
+        "parallelism": f"token-sharded x{world}, weights replicated",
+    }
+
+
 def run_reference(args):
     """The oracle timed on the host cores, on this arm's workload/metric."""
     rank = int(os.environ.get("RANK", "0"))
@@ -488,8 +498,9 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {wl.title}", "d_in": lay.d_in, "d_out": lay.d_out,
-                   "a_bits": lay.a_bits, "w_bits": lay.w_bits},
+        "config": {**workload_config(args, wl, lay, args.tokens or wl.tokens, args.gpus),
+                   "step": "the oracle (fp64 numpy): rotate_quantize + linear_from_codes on a bounded "
+                           "sample of the workload's tokens, weight rows prepared beforehand"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                          "sample": f"{total_tok} tokens, {args.steps} steps of ~{per_step:.1f} s, chunks of 32"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

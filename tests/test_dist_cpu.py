@@ -57,3 +57,19 @@ def test_single_process_helpers():
     import bench
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.whole_job_rate(1, 100, 2, 10.0) == pytest.approx(20000.0)
+
+
+def test_both_arms_report_the_same_workload_config():
+    # the reference arm and this arm describe a run by the same config keys
+    import argparse
+
+    import bench
+    from quantized_linear_token_b200 import workloads as W
+    for key in ("dit_image", "dit_mlp", "video_dit", "stress"):
+        wl = W.WORKLOADS[key]
+        for lay in wl.layers:
+            args = argparse.Namespace(workload=key, layer=lay.name, tokens=0, gpus=2)
+            cfg = bench.workload_config(args, wl, lay, wl.tokens, 2)
+            assert cfg["layer"] == lay.name and cfg["tokens_per_gpu"] == wl.tokens
+            assert cfg["h"] == lay.d_in & -lay.d_in and cfg["x_dtype"] == "bf16"
+            assert cfg["parallelism"].startswith("token-sharded x2")
