@@ -244,9 +244,10 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  *   x    device [T, d_in] bf16 (OQ_DTYPE_BF16 only, else OQ_ERR_UNSUPPORTED).
  *   a16  device [T, d_in] uint16 (fp16 bits), 16-byte aligned.
  *   s    device [T] fp32 token norms.
- * For h = 1024 without OQ_FLAG_SIGNS the block transform runs on the tensor
- * cores (H_1024 = H_32 (x) H_32 as two passes of warp MMAs, the second on a
- * two-term tf32 split of the fp32 intermediate): its fp32 rounding differs
+ * For h = 1024 (d_in <= 8192) or h = 512 (d_in <= 16384) without
+ * OQ_FLAG_SIGNS the block transform runs on the tensor cores (H_h =
+ * H_{h/32} (x) H_32 as two passes of warp MMAs, the second on a two-term tf32
+ * split of the fp32 intermediate): its fp32 rounding differs
  * from oq_rotate_quantize's, so a code may differ from that call's where the
  * coordinate lies within rounding of a decision threshold, and s may differ
  * in the last bits.  Both meet the same bounds against the exact transform.
