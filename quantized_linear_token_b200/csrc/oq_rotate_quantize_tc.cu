@@ -1,6 +1,6 @@
 // Rotate + quantize with the block Walsh-Hadamard transform on the tensor
-// cores, for blocks of h = 1024 or 512 and bf16 activations, writing the fp16 levels
-// of the codes (the A operand of the fused layer call).  Same arithmetic
+// cores, for blocks of h = 1024 or 512 and bf16 activations, writing the fp16
+// levels of the codes (the A operand of the fused layer call).  Same arithmetic
 // contract as rq_kernel (gecl notes Method 1, 3, 4; pith Supplementary A):
 //   s = ||x||_2,  y = P_pi x,  z_j = H_h y_j (block j, unnormalised),
 //   code_i = #{k : t_k < z_i / (s sqrt(h))},  output fp16(a_scale C[code_i]).
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
 #pragma unroll
   for (int i = 0; i < 4; ++i) hn[i] = hp[i] ^ 0x80008000u;
   // pass 2 (tf32, K order of k-tile nt: k = q <-> a = 8 nt + 2q, k = q + 4
-  // <-> a = 8 nt + 2q + 1): A[a'][k] = H_32[a'][a].  For rows a' = 16 mt + g
+  // <-> a = 8 nt + 2q + 1): A[a'][k] = H_A[a'][a].  For rows a' = 16 mt + g
   // + 8 h the sign is sgn(g & a) times (-1)^(mt & nt >> 1) times (-1)^(h &
   // nt & 1), so four values cover every fragment.
   const uint32_t u = hbit32(g, 2 * q), v = hbit32(g, 2 * q + 1);
