@@ -137,6 +137,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ oracle timing (host)
+def oracle_cpu_rate_single_thread(wl, lay, seconds: float):
+    """oracle_cpu_rate with numpy's thread pools limited to one thread."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=1):
+        rate, el, done, _ = oracle_cpu_rate(wl, lay, seconds)
+    return rate, el, done
+
+
 def oracle_cpu_rate(wl, lay, seconds: float, chunk: int = 32):
     """Tokens/s of the fp64 oracle (as it stands) on this host's cores, on a
     bounded sample of the workload: chunks of `chunk` tokens, until `seconds`
@@ -453,10 +461,14 @@ def run_ours(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, el, done, threads = oracle_cpu_rate(wl, lay, args.cpu_seconds)
+        rate1, el1, done1 = oracle_cpu_rate_single_thread(wl, lay, max(1.0, args.cpu_seconds / 4))
         out["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": threads, "kind": "oracle",
                                "sample": f"{done} tokens of {args.workload} in chunks of 32 "
                                          f"({el:.1f} s): oracle rotate_quantize + linear_from_codes, "
-                                         f"fp64 numpy; weight rows prepared beforehand"}
+                                         f"fp64 numpy; weight rows prepared beforehand",
+                               "single_thread": {"value": rate1, "unit": UNIT, "cores": 1,
+                                                 "sample": f"{done1} tokens ({el1:.1f} s), numpy limited to "
+                                                           f"one thread"}}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
