@@ -21,12 +21,14 @@
  * Conventions for every call below:
  *   - Pointers named "device" must point to CUDA device memory of the current
  *     device, be 16-byte aligned and be contiguous row-major.  The caller owns
- *     them.  The library owns only what an oq_layer holds (the permutation,
- *     codebook tables, an error word).
+ *     them.  The library owns only what an oq_layer holds (the permutation and
+ *     gather tables, codebook and threshold tables, split-K counters, an error
+ *     word, and the copy streams of oq_linear_fused_host).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; the return value reports
- *     argument checks and launch errors only.  No call allocates memory except
- *     oq_layer_create.
+ *     argument checks and launch errors only.  No call allocates device memory
+ *     except oq_layer_create; oq_linear_fused_host creates its layer's two
+ *     copy streams and their events on its first call.
  *   - Faults the kernels detect themselves (a bounded wait that ran out, an
  *     index out of range) set the layer's device error word, read back by
  *     oq_poll_error.
