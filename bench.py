@@ -136,6 +136,87 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+class NvmlClockSampler:
+    """SM clock, power and throttle reasons polled through NVML about every
+    half millisecond, with host timestamps, so that the summary covers the
+    timed region itself (a few milliseconds here, shorter than nvidia-smi's
+    sampling period).  stop(t0, t1) summarises the samples taken between the
+    host times t0 and t1 (perf_counter), or, if the region held none, the
+    samples closest to it."""
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+
+    def __init__(self, gpu_uuid: str, period_s: float = 0.0005):
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(gpu_uuid)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(pynvml, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        self.period = period_s
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.thread = None
+        # one reading of each query now, so that a query this driver lacks
+        # fails here (and the caller falls back) rather than in the thread
+        pynvml.nvmlDeviceGetClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.reasons_fn(self.h)
+        pynvml.nvmlDeviceGetPowerUsage(self.h)
+
+    def _poll(self):
+        nv = self.nv
+        try:
+            while not self.stop_flag.is_set():
+                t = time.perf_counter()
+                sm = float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                mask = int(self.reasons_fn(self.h))
+                power = float(nv.nvmlDeviceGetPowerUsage(self.h)) / 1000.0
+                self.samples.append((t, sm, mask, power))
+                self.stop_flag.wait(self.period)
+        except Exception:        # sampling ends; what was gathered is kept
+            return
+
+    def start(self):
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+
+    def stop(self, t0: float, t1: float):
+        self.stop_flag.set()
+        if self.thread is not None:
+            self.thread.join(timeout=2.0)
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        window = "timed region"
+        if not inside and self.samples:
+            mid = 0.5 * (t0 + t1)
+            inside = sorted(self.samples, key=lambda x: abs(x[0] - mid))[:3]
+            window = "the samples nearest the timed region"
+        reasons = sorted({n for _, _, m, _ in inside for n, bit in self.REASONS if m & bit})
+        return {"sm_mhz": statistics.median([x[1] for x in inside]) if inside else None,
+                "sm_max_mhz": self.max_mhz,
+                "power_w_max": max(x[3] for x in inside) if inside else None,
+                "reasons": reasons, "samples": len(inside), "source": f"NVML, {window}"}
+
+
+def start_clock_sampler(uuid: str):
+    """NVML sampling of the timed region if NVML answers, else nvidia-smi."""
+    try:
+        c = NvmlClockSampler(uuid)
+        c.start()
+        return c
+    except Exception:
+        c = ClockSampler(uuid)
+        c.start()
+        time.sleep(0.3)
+        return c
+
+
+def stop_clock_sampler(c, t0: float, t1: float):
+    if isinstance(c, NvmlClockSampler):
+        return c.stop(t0, t1)
+    return c.stop()
+
+
 # ------------------------------------------------------------------ oracle timing (host)
 def oracle_cpu_rate_single_thread(wl, lay, seconds: float):
     """oracle_cpu_rate with numpy's thread pools limited to one thread."""
@@ -312,10 +393,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     B.oq_poll_error(layer)
     evf = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    clocks = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
-    if clocks:
-        clocks.start()
-        time.sleep(0.3)
+    clocks = start_clock_sampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -328,8 +406,9 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    wall = time.perf_counter() - wall0
-    clk = clocks.stop() if clocks else None
+    wall1 = time.perf_counter()
+    wall = wall1 - wall0
+    clk = stop_clock_sampler(clocks, wall0, wall1) if clocks else None
     B.oq_poll_error(layer)
     t_fused = [evf[i][0].elapsed_time(evf[i][1]) for i in range(K)]
     total_ms = max_over_ranks(sum(t_fused), dev)
