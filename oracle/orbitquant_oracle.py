@@ -18,11 +18,38 @@ section:
                       Incoherence".
 
 Each function follows the method's steps in the pages' order, in fp64.  Where
-the pages are silent the function says which reading it takes (the readings
-are numbered D1..D17 in the design notes).  Library primitives used as single
-steps: ``numpy`` gathers/matmul, ``np.searchsorted`` (a sorted search),
-``scipy.special.betainc`` / ``erfc`` (the regularised incomplete beta function
-and the complementary error function) and ``math.lgamma``.
+the pages are silent, ambiguous or at odds with one another, the function
+names the reading it takes; the readings are:
+
+* D1  marginal: the exact law of one coordinate of a uniform point on
+      S^{d-1} (pith referee minor comment 1); N(0, 1/d) of pith Figure 2 as
+      an option.
+* D2  Lloyd-Max solver: Lloyd's alternation from N(0, 3/d) quantiles until
+      no level moves by 1e-11/sqrt(d).
+* D3  nearest level through midpoint thresholds.
+* D4  codes unsigned and ascending with the level; a value exactly on a
+      threshold takes the lower code.
+* D5  a zero token has s = 0 and every coordinate u = 0.
+* D6  the permutation is a gather, y_i = x_{pi(i)}, drawn by SplitMix64(seed)
+      driving a descending Fisher-Yates shuffle.
+* D7  Rademacher signs (pith Supplementary A) optional, drawn after the
+      shuffle, -1 when bit 63 of the draw is set.
+* D8  Sylvester natural order, scale 1/sqrt(h), block j = rotated positions
+      [j h, (j+1) h).
+* D9  h = the largest power of two dividing d.
+* D10 normalise, then rotate (equal to the reverse order).
+* D11 weights use the same Lloyd-Max quantizer with row norm r.
+* D12 no bias and no renormalisation of the dequantised directions.
+* D13 32 codes per little-endian bit stream of 32*b bits, b uint32 words.
+* D14 inputs read as their exact values (bf16 / fp32), all arithmetic fp64.
+* D15 the codebook's dimension is d_in, not h.
+* D18 AdaLN exception path: symmetric per-row INT4 round-to-nearest.
+(D16 and D17, the output and code tolerances, belong to the parity tests.)
+
+Library primitives used as single steps: ``numpy`` gathers/matmul,
+``np.searchsorted`` (a sorted search), ``scipy.special.betainc`` / ``erfc``
+(the regularised incomplete beta function and the complementary error
+function) and ``math.lgamma``.
 """
 
 from __future__ import annotations

@@ -254,6 +254,59 @@ def test_threshold_count_equals_nearest_level():
     assert O.quantize(np.array([-1.0, 1.0]), cb.thresholds).tolist() == [0, 15]
 
 
+@pytest.mark.parametrize("d", [256, 3072])
+@pytest.mark.parametrize("b", [2, 3, 4, 8])
+def test_threshold_distance_is_brute_force_minimum(d, b):
+    # threshold_distance decides which GPU code mismatches the parity bound
+    # excuses (a coordinate within 1e-5/sqrt(d) of a decision threshold).  Pin
+    # it to its definition min_j |u - t_j| taken by brute force over every
+    # threshold, on random coordinates, on coordinates exactly at and just
+    # beside each threshold (where a wrong searchsorted side or an
+    # off-by-one neighbour shows), and on coordinates past the outermost
+    # thresholds and past +-1.
+    cb = O.lloyd_max(d, b)
+    t = cb.thresholds
+    rng = np.random.default_rng(d + b)
+    step = 1e-7 / math.sqrt(d)
+    u = np.concatenate([
+        rng.standard_normal(50000) / math.sqrt(d),
+        t, t + step, t - step, np.nextafter(t, np.inf), np.nextafter(t, -np.inf),
+        0.5 * (t[:-1] + t[1:]),                         # equidistant from two thresholds
+        [t[0] - 1.0, t[-1] + 1.0, t[0] - step, t[-1] + step, -1.0, 1.0, -5.0, 5.0, 0.0],
+    ])
+    brute = np.min(np.abs(u[:, None] - t[None, :]), axis=1)
+    np.testing.assert_array_equal(O.threshold_distance(u, t), brute)
+    # the band test of the parity checks: exactly the coordinates whose
+    # nearest threshold is closer than the band
+    band = 1e-5 / math.sqrt(d)
+    np.testing.assert_array_equal(O.threshold_distance(u, t) < band, brute < band)
+    assert np.all(O.threshold_distance(t, t) == 0.0)
+
+
+@pytest.mark.parametrize("d", [3, 4, 16, 256, 3072])
+@pytest.mark.parametrize("gaussian", [False, True])
+def test_partial_moment_equals_quadrature(d, gaussian):
+    # the closed-form first moment of each half-line cell (exact sphere
+    # marginal: the antiderivative of t (1 - t^2)^((d-3)/2); Gaussian: of
+    # t phi(t)) against adaptive quadrature of t f_d(t) over the same interval
+    sig = 1.0 / math.sqrt(d)
+    top = 1.0 if not gaussian else 12.0 * sig
+    edges = [(0.0, 0.3 * sig), (0.3 * sig, 1.1 * sig), (1.1 * sig, 2.7 * sig), (0.0, top),
+             (2.7 * sig, top), (0.5 * sig, 0.5 * sig)]
+    for a, b in edges:
+        a, b = min(a, top), min(b, top)
+        want, _ = integrate.quad(lambda t: t * O.marginal_pdf(t, d, gaussian), a, b, epsabs=0, epsrel=1e-12,
+                                 limit=200)
+        got = float(O.marginal_partial_moment(a, b, d, gaussian))
+        assert abs(got - want) <= 1e-10 * (abs(want) + sig * 1e-3), (a, b, got, want)
+    # the half-line moment E[T; T > 0] in closed form: for the sphere
+    # Gamma(d/2) / (sqrt(pi) Gamma((d-1)/2) (d-1)), for N(0, 1/d) 1/sqrt(2 pi d)
+    half = float(O.marginal_partial_moment(0.0, math.inf if gaussian else 1.0, d, gaussian))
+    want_half = (1.0 / math.sqrt(2 * math.pi * d) if gaussian else
+                 math.exp(math.lgamma(d / 2) - math.lgamma((d - 1) / 2)) / (math.sqrt(math.pi) * (d - 1)))
+    assert abs(half - want_half) <= 1e-13 * want_half
+
+
 def test_quantizer_mse_matches_design():
     d = 256
     g = np.random.default_rng(9).standard_normal((20000, d))
