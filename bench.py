@@ -444,8 +444,13 @@ def run_ours(args):
     flops = 2.0 * T * d * dout
 
     def rq_bytes_per_launch(rt):
-        # bf16 x read + A operand written (fp16 levels, or packed codes) + norms
+        # the bytes this route's kernel moves: bf16 x read + its A operand
+        # written (fp16 levels, or packed codes) + norms
         return T * (2 * d + (2 * d if rt != "codes" else d * lay.a_bits / 8) + 4)
+
+    # the method's algorithmic bytes of rotate + quantize, whatever the route
+    # writes: bf16 x read, packed codes and the norm written
+    rq_alg_bytes = T * (2 * d + d * lay.a_bits / 8 + 4)
 
     def route_decoded(rt):
         return rt == "levels" and decoded
@@ -506,12 +511,17 @@ def run_ours(args):
         },
         "roofline_rotate_quantize": {
             "kernel": rq_desc["codes" if route == "codes" else "levels"],
-            "bound": "hbm", "achieved": rq_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": rq_gbs / peaks["hbm_gbs"],
-            "traffic": measured_traffic("rq_levels") if (route != "codes" and full_size) else None,
+            "bound": "hbm", "achieved": rq_alg_bytes / (rq_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": rq_alg_bytes / (rq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "bytes_per_launch": rq_alg_bytes,
+            "bytes_rule": "algorithmic: 2 d (bf16 x) + d a_bits / 8 (packed codes) + 4 (norm) per token",
+            "traffic": measured_traffic("rq_levels" if route != "codes" else "rq_codes") if full_size else None,
             "peak_source": f"{peaks['source']} HBM copy bandwidth",
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, profiles/traffic.json",
-            "bytes_per_launch": rq_bytes, "ms_per_launch": rq_ms,
+            "ms_per_launch": rq_ms,
+            "route_bytes_per_launch": rq_bytes, "route_achieved": rq_gbs, "route_frac": rq_gbs / peaks["hbm_gbs"],
+            "route_bytes_rule": ("the bytes this route's kernel moves: its A operand is written as fp16 levels, "
+                                 "2 d bytes per token" if route != "codes" else "same as algorithmic"),
         },
         **({"roofline_weight_levels": {
             "kernel": "weight codes -> fp16 levels (once per call)",
@@ -528,7 +538,8 @@ def run_ours(args):
                           "ms_per_step": other_ms[o] / K,
                           "gemm_tflops": flops / (statistics.mean(other_per[o]["gemm"]) * 1e-3) / 1e12,
                           "gemm_ms": statistics.mean(other_per[o]["gemm"]),
-                          "rq_gbs": rq_bytes_per_launch(o) / (statistics.mean(other_per[o]["rq"]) * 1e-3) / 1e9,
+                          "rq_gbs": rq_alg_bytes / (statistics.mean(other_per[o]["rq"]) * 1e-3) / 1e9,
+                          "rq_route_gbs": rq_bytes_per_launch(o) / (statistics.mean(other_per[o]["rq"]) * 1e-3) / 1e9,
                           "rq_ms": statistics.mean(other_per[o]["rq"])} for o in others],
         "e2e": {"value": whole_job_rate(world, T, K, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),

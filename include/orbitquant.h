@@ -21,9 +21,10 @@
  * Conventions for every call below:
  *   - Pointers named "device" must point to CUDA device memory of the current
  *     device, be 16-byte aligned and be contiguous row-major.  The caller owns
- *     them.  The library owns only what an oq_layer holds (the permutation and
+ *     them.  The library owns what an oq_layer holds (the permutation and
  *     gather tables, codebook and threshold tables, split-K counters, an error
- *     word, and the copy streams of oq_linear_fused_host).
+ *     word, and the copy streams of oq_linear_fused_host), and the fixed
+ *     scratch array of oq_linear_fused_static on every GPU that loads it.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Work is enqueued asynchronously; the return value reports
  *     argument checks and launch errors only.  No call allocates device memory
@@ -296,10 +297,11 @@ oq_status oq_linear_decoded(const oq_layer* layer, const uint16_t* a16, const fl
 
 /*
  * oq_linear_fused_static -- the same computation as oq_linear_fused for
- * callers that cannot allocate device memory: code running inside a CUDA
- * graph capture, runtimes that give plug-ins no allocator, loops where an
- * allocation or the synchronisation it implies is not allowed.  (The pages
- * have no counterpart; this is an interface for such callers.)
+ * callers that cannot allocate device memory: inference runtimes that give
+ * plug-ins no allocator, deployments whose device memory is fixed at start-
+ * up, loops where an allocation or the synchronisation it implies is not
+ * allowed.  (The pages have no counterpart; this is an interface for such
+ * callers.)
  *   The scratch that oq_linear_fused takes as `workspace` comes instead from a
  *   fixed array of OQ_STATIC_SCRATCH_BYTES bytes in device memory that the
  *   library reserves on every GPU that loads it, until the process exits.
@@ -308,11 +310,13 @@ oq_status oq_linear_decoded(const oq_layer* layer, const uint16_t* a16, const fl
  *   that device current); make that first call before any stream capture.
  *   Every call shares the array: calls that overlap on the GPU (different
  *   streams or host threads) race and give wrong results.
- *   Arguments as for oq_linear_fused; the array serves as its least
- *   workspace (A operand and norms), so weights are decoded inside the
- *   contraction.  Errors: OQ_ERR_INVALID_ARG when the batch needs more
- *   scratch than the array holds (at d_in = 3072 with d_out % 256 == 0 about
- *   2700 tokens).
+ *   Arguments as for oq_linear_fused.  The array serves as its least
+ *   workspace (the A operand and the norms), so the weights are decoded
+ *   inside the contraction at every batch size and y is that of
+ *   oq_linear_fused given that least workspace, bit for bit.  Errors:
+ *   OQ_ERR_INVALID_ARG when the batch needs more scratch than the array holds
+ *   (2 d_in + 4 bytes per token with bf16 x and d_out % 256 == 0: about 2700
+ *   tokens at d_in = 3072).
  */
 #define OQ_STATIC_SCRATCH_BYTES (16u << 20)
 oq_status oq_linear_fused_static(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,

@@ -23,6 +23,7 @@ SOURCES = ["oq_api.cu", "oq_rotate_quantize.cu", "oq_rotate_quantize_tc.cu", "oq
            "oq_levels.cu", "oq_host_io.cu", "oq_int4.cu",
            "oq_noalloc.cu", "oq_host.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-lineinfo", "-std=c++17"]
 
 
 def nvcc() -> str:
@@ -38,11 +39,30 @@ def _deps():
     return files
 
 
+STAMP = LIB + ".srchash"
+
+
+def source_hash() -> str:
+    """SHA-256 over every source and header the library is built from, and
+    the compiler flags, in a fixed order: the identity of a build."""
+    import hashlib
+    m = hashlib.sha256()
+    m.update(" ".join(ARCH + FLAGS).encode())
+    for f in sorted(_deps()):
+        m.update(os.path.basename(f).encode() + b"\0")
+        with open(f, "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    """The library exists and was built from exactly the sources present now
+    (a stamp with their hash is written beside it by every build); file times
+    are not trusted, since a copied tree keeps no build order."""
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(f) <= t for f in _deps())
+    with open(STAMP) as f:
+        return f.read().strip() == source_hash()
 
 
 def _run(cmd, verbose):
@@ -58,11 +78,12 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     """Compile every source for sm_100a (in parallel) and link the library."""
     if not force and up_to_date():
         return LIB
+    stamp = source_hash()
     from concurrent.futures import ThreadPoolExecutor
 
     objdir = os.path.join(ROOT, "_build")
     os.makedirs(objdir, exist_ok=True)
-    common = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
+    common = [nvcc(), *ARCH, *FLAGS, "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
     if ptxas_verbose:
         common += ["-Xptxas", "-v"]
     jobs = []
@@ -74,7 +95,12 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     if verbose or ptxas_verbose:
         sys.stdout.write("".join(outs))
     _run([nvcc(), *ARCH, "--shared", "-o", LIB + ".tmp"] + [o for o, _ in jobs], verbose)
+    if os.path.exists(STAMP):
+        os.remove(STAMP)
     os.replace(LIB + ".tmp", LIB)
+    with open(STAMP + ".tmp", "w") as f:
+        f.write(stamp + "\n")
+    os.replace(STAMP + ".tmp", STAMP)
     return LIB
 
 

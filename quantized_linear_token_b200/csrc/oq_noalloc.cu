@@ -1,12 +1,14 @@
 // oq_linear_fused_static: the fused layer call for callers that cannot
-// allocate device memory.  Some callers have no allocator to call: code that
-// runs while a CUDA graph is being captured for replay, inference runtimes
-// that hand out no device memory to plug-ins, and real-time loops in which an
-// allocation (and the synchronisation it can imply) is not allowed.  For them
-// the scratch that oq_linear_fused takes from the caller (the packed
-// activation codes and token norms passed from the rotate-quantize kernel to
-// the contraction) lives in a fixed array in device memory that belongs to
-// this library.
+// allocate device memory.  Some callers have no allocator to call: inference
+// runtimes that hand out no device memory to plug-ins, deployments whose
+// device memory is fixed when the process starts, and real-time loops in
+// which an allocation (and the synchronisation it can imply) is not allowed.
+// For them the scratch that oq_linear_fused takes from the caller lives in a
+// fixed array in device memory that belongs to this library.  That scratch is
+// the fused call's least workspace: the A operand that the rotate-quantize
+// kernel hands to the contraction (the fp16 levels of the activation codes
+// for bf16 x with d_out % 256 == 0, the packed codes otherwise) and the token
+// norms.
 //
 // The array is a file-scope static __device__ array of OQ_STATIC_SCRATCH_BYTES
 // bytes: every GPU that loads the library holds it until the process exits.
@@ -16,10 +18,10 @@
 // before any stream capture.  No call allocates or frees memory.
 //
 // All calls share the one array and it keeps the last call's contents.  Every
-// byte a call reads is written earlier in the same call (codes and norms of
-// its own tokens), so nothing needs clearing, but two calls that run at the
-// same time on the GPU (different streams, or different host threads) race on
-// the array and give wrong results.
+// byte a call reads is written earlier in the same call (the A operand and
+// norms of its own tokens), so nothing needs clearing, but two calls that run
+// at the same time on the GPU (different streams, or different host threads)
+// race on the array and give wrong results.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -74,8 +76,8 @@ extern "C" oq_status oq_linear_fused_static(const oq_layer* layer, const void* x
     return OQ_ERR_INVALID_ARG;
   }
   if (T == 0) return OQ_OK;
-  // the static array holds the fused call's least workspace (large batches
-  // then decode weights inside the contraction)
+  // the static array serves as the fused call's least workspace, so the
+  // weights are decoded inside the contraction at every batch size
   const size_t need = oq::fused_min_workspace(layer, T);
   if (need > (size_t)OQ_STATIC_SCRATCH_BYTES) {
     oq::set_error("oq_linear_fused_static: " + std::to_string(T) + " tokens need " + std::to_string(need) +
@@ -86,5 +88,5 @@ extern "C" oq_status oq_linear_fused_static(const oq_layer* layer, const void* x
   void* scratch = nullptr;
   const oq_status st = scratch_address(&scratch);
   if (st != OQ_OK) return st;
-  return oq_linear_fused(layer, x, x_dtype, T, Wcodes, r, y, scratch, (size_t)OQ_STATIC_SCRATCH_BYTES, stream);
+  return oq_linear_fused(layer, x, x_dtype, T, Wcodes, r, y, scratch, need, stream);
 }

@@ -66,6 +66,13 @@ def check_linear(y_gpu: np.ndarray, words_a: np.ndarray, s_gpu: np.ndarray, word
     rel = np.where(bound > 0, err / safe, err)
     worst = float(rel.max()) if rel.size else 0.0
     assert worst <= Y_TOL, f"{label}: max bound-relative error {worst:.3e} > {Y_TOL}"
-    big = np.abs(y_or) >= 1e-2 * math.sqrt(float(np.mean(y_or ** 2)) + 1e-300)
-    plain = float((err[big] / np.abs(y_or[big])).max()) if big.any() else 0.0
-    return {"max_bound_rel": worst, "max_plain_rel_large": plain}
+    # the plain relative error |dy| / |y| is reported, not bounded: the levels
+    # are irrational and the tensor cores multiply them as fp16 values (the
+    # level rounding, up to ~1e-4 relative at 4 bits and ~3.5e-4 at 8 bits,
+    # enters y scaled by bound / |y|, which grows without limit as y -> 0)
+    rms = math.sqrt(float(np.mean(y_or ** 2)) + 1e-300)
+    plain = {}
+    for name, frac in (("max_plain_rel_at_1pct_rms", 1e-2), ("max_plain_rel_at_rms", 1.0)):
+        big = np.abs(y_or) >= frac * rms
+        plain[name] = float((err[big] / np.abs(y_or[big])).max()) if big.any() else 0.0
+    return {"max_bound_rel": worst, **plain}
