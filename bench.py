@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--route", choices=["levels", "levels_wdec", "codes"], default="levels",
                     help="hot-path route of the timed step (the others are reported beside it)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--sweep", action="store_true",
+                    help="the stress workload's sweep (every token count x every layer): one JSON line per point")
     return ap.parse_args()
 
 
@@ -610,10 +612,109 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_sweep(args):
+    """The stress sweep on one GPU: 13824 -> 5120 at every token count of the
+    workload and every layer (W2A4, W3A3, W4A4, W4A8).  Per point: the step
+    (one oq_linear_fused call, L2 flushed before each), then the same path as
+    stage calls with an event after each kernel for the rooflines.  One JSON
+    line per point."""
+    import numpy as np
+    import torch
+
+    from quantized_linear_token_b200 import binding as B
+    from quantized_linear_token_b200 import build as Bld
+    from quantized_linear_token_b200 import workloads as W
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    Bld.build()
+    B.load_library()
+    peaks = load_peaks()
+    wl = W.WORKLOADS["stress"]
+    sweep = wl.token_sweep
+    d = wl.layers[0].d_in
+    # the recipe does not depend on the batch size, so every smaller batch is
+    # the first rows of the largest one
+    x_all = torch.from_numpy(W.activations(wl, d, tokens=max(sweep)).view(np.int16)).view(torch.bfloat16).to(dev)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    K, warm = args.steps, max(3, args.warmup)
+    for lay in wl.layers:
+        dout = lay.d_out
+        layer = B.oq_layer_create(d, dout, W.ROTATION_SEED, lay.a_bits, lay.w_bits)
+        Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(W.weights(wl, lay)).to(dev))
+        for T in sweep:
+            x = x_all[:T]
+            y = torch.empty((T, dout), dtype=torch.float32, device=dev)
+            ws = torch.empty((B.oq_linear_fused_workspace_size(layer, T),), dtype=torch.uint8, device=dev)
+            a16 = torch.empty((T, d), dtype=torch.float16, device=dev)
+            s = torch.empty((T,), dtype=torch.float32, device=dev)
+            decoded = T >= B.W16_MIN_T
+            w16 = torch.empty((dout, d), dtype=torch.float16, device=dev) if decoded else None
+            stages = [("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s))]
+            if decoded:
+                stages += [("wlevels", lambda: B.oq_weight_levels(layer, Wc, w16)),
+                           ("gemm", lambda: B.oq_linear_decoded(layer, a16, s, w16, r, y))]
+            else:
+                stages += [("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]
+            runs = {"step": [("step", lambda: B.oq_linear_fused(layer, x, Wc, r, y, ws))], "stages": stages}
+            times = {}
+            for name, st in runs.items():
+                for _ in range(warm):
+                    flush.zero_()
+                    for _, fn in st:
+                        fn()
+                ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(st) + 1)] for _ in range(K)]
+                torch.cuda.synchronize()
+                for i in range(K):
+                    flush.zero_()
+                    ev[i][0].record(stream)
+                    for j, (_, fn) in enumerate(st):
+                        fn()
+                        ev[i][j + 1].record(stream)
+                torch.cuda.synchronize()
+                for j, (kname, _) in enumerate(st):
+                    times[kname] = statistics.mean(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K))
+            B.oq_poll_error(layer)
+            flops = 2.0 * T * d * dout
+            rq_alg = T * (2 * d + d * lay.a_bits / 8 + 4)
+            line = {
+                "metric": METRIC, "sweep_point": True, "value": T / (times["step"] * 1e-3), "unit": UNIT,
+                "n_gpus": 1, "steps": K, "warmup": warm, "ms_per_step": times["step"],
+                "higher_is_better": True, "dtype": "f16", "data": "synthetic",
+                "config": {"workload": f"stress: {wl.title}", "layer": lay.name, "tokens_per_gpu": T, "d_in": d,
+                           "d_out": dout, "a_bits": lay.a_bits, "w_bits": lay.w_bits, "h": d & -d,
+                           "x_bytes": T * d * 2,
+                           "l2": "flushed (256 MiB write) before every step, outside the timed events",
+                           "contraction": "decoded weights, both operands by TMA" if decoded else
+                           ("small-batch split-K kernel" if T <= 256 else "CTA pair, weights decoded in the GEMM")},
+                "roofline": {"bound": "tensor", "achieved": flops / (times["gemm"] * 1e-3) / 1e12,
+                             "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": flops / (times["gemm"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                             "traffic": None, "ms_per_launch": times["gemm"]},
+                "roofline_rotate_quantize": {"bound": "hbm", "achieved": rq_alg / (times["rq"] * 1e-3) / 1e9,
+                                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                             "frac": rq_alg / (times["rq"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                             "bytes_per_launch": rq_alg, "ms_per_launch": times["rq"]},
+                "step_tflops": flops / (times["step"] * 1e-3) / 1e12,
+                "step_frac": flops / (times["step"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            }
+            if decoded:
+                wb = dout * d * (lay.w_bits / 8 + 2)
+                line["roofline_weight_levels"] = {"bound": "hbm", "achieved": wb / (times["wlevels"] * 1e-3) / 1e9,
+                                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                                  "frac": wb / (times["wlevels"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                                  "bytes_per_launch": wb, "ms_per_launch": times["wlevels"]}
+            print(json.dumps(line), flush=True)
+            del y, ws, a16, s, w16
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 

@@ -30,9 +30,9 @@
  *     argument checks and launch errors only.  No call allocates device memory
  *     except oq_layer_create; oq_linear_fused_host creates its layer's two
  *     copy streams and their events on its first call.
- *   - Faults the kernels detect themselves (a bounded wait that ran out, an
- *     index out of range) set the layer's device error word, read back by
- *     oq_poll_error.
+ *   - Every wait inside a kernel is bounded (1 s); a wait that runs out sets
+ *     the layer's device error word, and the kernel ends without its result.
+ *     oq_poll_error reads the word back (OQ_ERR_TIMEOUT).
  *   - Supported shapes: d_in % 32 == 0 with h = (largest power of two dividing
  *     d_in) in [32, 4096]; d_out % 16 == 0; a_bits in {2,3,4,8}; w_bits in
  *     {2,3,4}.  Anything else returns OQ_ERR_UNSUPPORTED.  T = 0 is a no-op.
@@ -59,7 +59,8 @@ typedef enum {
   OQ_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed          */
   OQ_ERR_TIMEOUT = 4,       /* a kernel's bounded wait ran out (device word) */
   OQ_ERR_NOMEM = 5,         /* oq_layer_create could not allocate            */
-  OQ_ERR_DEVICE = 6         /* a kernel's own bounds check fired             */
+  OQ_ERR_DEVICE = 6         /* the device error word holds a bit this version
+                               does not define (reserved)                    */
 } oq_status;
 
 enum { OQ_DTYPE_F32 = 0, OQ_DTYPE_BF16 = 1 };
@@ -348,8 +349,21 @@ oq_status oq_linear_fused_host(const oq_layer* layer, const void* x_host, int32_
                                size_t workspace_bytes, void* stream);
 
 /* Reads and clears the layer's device error word.  Synchronizes the device.
- * Returns OQ_OK, OQ_ERR_TIMEOUT or OQ_ERR_DEVICE. */
+ * Returns OQ_OK or OQ_ERR_TIMEOUT (OQ_ERR_DEVICE for a bit this version does
+ * not define). */
 oq_status oq_poll_error(const oq_layer* layer);
+
+/*
+ * oq_check_wait_timeout -- a self-test of the failure path shared by every
+ * kernel (the pages have no counterpart).  Launches one warp that waits, with
+ * the library's bounded-wait routine and a bound of `limit_us` microseconds
+ * (1 .. 1000000), on an mbarrier that no thread ever arrives on.  The wait runs
+ * out, sets the timeout bit of the layer's error word and returns; the kernel
+ * ends normally and the CUDA context stays usable.  The next oq_poll_error
+ * returns OQ_ERR_TIMEOUT and clears the word.  Asynchronous on `stream`.
+ * Errors: OQ_ERR_INVALID_ARG for a null layer or a bound out of range.
+ */
+oq_status oq_check_wait_timeout(const oq_layer* layer, uint32_t limit_us, void* stream);
 
 /* Message for the last error on the calling thread ("" if none). */
 const char* oq_last_error(void);

@@ -33,7 +33,7 @@ EXPORTS = (
     "oq_rotate_quantize", "oq_weight_prepare", "oq_linear", "oq_linear_fused_workspace_size",
     "oq_linear_fused", "oq_rotate_quantize_levels", "oq_linear_levels", "oq_weight_levels", "oq_linear_decoded",
     "oq_linear_fused_static", "oq_linear_fused_host_workspace_size", "oq_linear_fused_host",
-    "oq_poll_error", "oq_last_error", "oq_status_string",
+    "oq_poll_error", "oq_check_wait_timeout", "oq_last_error", "oq_status_string",
 )
 
 
@@ -94,6 +94,7 @@ def load_library(path: str = LIB_PATH):
         "oq_linear_decoded": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
         "oq_poll_error": (i32, [vp]),
+        "oq_check_wait_timeout": (i32, [vp, ctypes.c_uint32, vp]),
         "oq_last_error": (ctypes.c_char_p, []),
         "oq_status_string": (ctypes.c_char_p, [i32]),
     }
@@ -359,3 +360,12 @@ def oq_linear_fused_static(layer: Layer, x, Wcodes, r, y=None):
 
 def oq_poll_error(layer: Layer) -> None:
     _check(load_library().oq_poll_error(layer.handle), "oq_poll_error")
+
+
+def oq_check_wait_timeout(layer: Layer, limit_us: int) -> None:
+    """Launch the bounded-wait self-test on the current stream (its wait runs
+    out after limit_us microseconds; oq_poll_error then raises)."""
+    torch = _torch()
+    _check(load_library().oq_check_wait_timeout(
+        layer.handle, int(limit_us), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)),
+        "oq_check_wait_timeout")

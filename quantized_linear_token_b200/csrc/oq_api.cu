@@ -354,9 +354,13 @@ oq_status oq_weight_prepare(const oq_layer* L, const void* W, int32_t W_dtype, u
   return rq(L, W, W_dtype, L->d_out, L->w_bits, L->bins_w, Wcodes, r, stream);
 }
 
+// The contraction kernels address token rows with 32-bit TMA coordinates.
+constexpr int64_t MAX_TOKENS = ((int64_t)1 << 31) - 1024;
+
 static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T,
                              const uint32_t* Wcodes, const float* r, float* y, void* stream,
                              const uint16_t* a_f16 = nullptr) {
+  if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
   GemmArgs g{};
   g.a_codes = codes;
   g.a_f16 = a_f16;
@@ -510,6 +514,7 @@ oq_status oq_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* 
 
 static oq_status linear_w16(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
                             const float* r, float* y, void* stream) {
+  if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
   GemmArgs g{};
   g.a_f16 = a16;
   g.b_f16 = w16;
@@ -639,8 +644,15 @@ oq_status oq_poll_error(const oq_layer* L) {
   // a timed-out small-batch call can leave split counters mid-way
   if ((word & OQ_DEVERR_TIMEOUT) && L->d_counters) cudaMemset(L->d_counters, 0, (size_t)(L->d_out / 32) * sizeof(int));
   if (word & OQ_DEVERR_TIMEOUT) return fail(OQ_ERR_TIMEOUT, "a kernel's bounded wait ran out");
-  if (word & OQ_DEVERR_BOUNDS) return fail(OQ_ERR_DEVICE, "a kernel's bounds check fired");
+  if (word) return fail(OQ_ERR_DEVICE, "unknown bits in the device error word");
   return OQ_OK;
+}
+
+oq_status oq_check_wait_timeout(const oq_layer* L, uint32_t limit_us, void* stream) {
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_check_wait_timeout: layer is null");
+  if (limit_us < 1 || limit_us > 1000000)
+    return fail(OQ_ERR_INVALID_ARG, "oq_check_wait_timeout: limit must be 1 .. 1000000 microseconds");
+  return wait_timeout_launch(L->d_error, (uint64_t)limit_us * 1000u, stream);
 }
 
 }  // extern "C"

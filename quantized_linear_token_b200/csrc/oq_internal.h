@@ -7,9 +7,8 @@
 
 #include "orbitquant.h"
 
-// error word bits written by kernels into the layer's device word
+// error word bit written by kernels into the layer's device word
 #define OQ_DEVERR_TIMEOUT 1
-#define OQ_DEVERR_BOUNDS 2
 
 // Threshold search table of one codebook for the rotate-quantize kernel: with
 // g = K sqrt(d) u (u the unit-norm rotated coordinate, K a power of two bins
@@ -156,6 +155,8 @@ oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, in
 oq_status fused_run(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
                     const float* r, float* y, void* ws, size_t ws_bytes, void* stream, const uint16_t* w16_ready);
 oq_status decode_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* w16, void* stream);
+// a one-warp kernel whose bounded wait (limit_ns) runs out (oq_diag.cu)
+oq_status wait_timeout_launch(int* err, uint64_t limit_ns, void* stream);
 // host-buffer pipeline resources of a layer (oq_host_io.cu)
 void io_release(oq_layer* L);
 // prmt decode tables of a codebook's fp16 levels (oq_gemm.cu)

@@ -57,15 +57,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err) {
+// Bounded wait for the phase with the given parity to complete (limit_ns:
+// the bound, OQ_WAIT_NS unless a caller gives a shorter one).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,
+                                          uint64_t limit_ns = OQ_WAIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > OQ_WAIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       if (err) atomicOr(err, OQ_DEVERR_TIMEOUT);
       return false;
     }

@@ -69,8 +69,15 @@ WORKLOADS = {
 }
 
 
-def _rng(seed: int) -> np.random.Generator:
-    return np.random.Generator(np.random.Philox(seed))
+ROW_BLOCK = 1024   # activations are drawn in independent blocks of this many tokens
+
+
+def _rng(seed: int, block: int | None = None) -> np.random.Generator:
+    """Philox with a key made of the seed and (for activation rows) the row
+    block, so any block can be drawn without drawing the ones before it."""
+    if block is None:
+        return np.random.Generator(np.random.Philox(seed))
+    return np.random.Generator(np.random.Philox(key=np.array([seed, block + 1], dtype=np.uint64)))
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -89,37 +96,56 @@ def _gelu_tanh(x: np.ndarray) -> np.ndarray:
 
 
 def activations(wl: Workload, d: int, tokens: int | None = None, gelu: bool = False,
-                stream: int = 0) -> np.ndarray:
-    """Draw the [tokens, d] activations of a workload.  Returns fp32 values for
-    fp32 recipes and bfloat16 bit patterns (uint16) otherwise.  ``stream``
-    selects an independent draw (e.g. a second layer's input)."""
+                stream: int = 0, rows: tuple | None = None) -> np.ndarray:
+    """Draw the [tokens, d] activations of a workload, or only the rows
+    [rows[0], rows[1]) of that batch (the same values).  Returns fp32 values
+    for fp32 recipes and bfloat16 bit patterns (uint16) otherwise.
+    ``stream`` selects an independent draw (e.g. a second layer's input).
+
+    The recipe's outlier channels come from one generator; token rows come in
+    blocks of ROW_BLOCK, each from its own generator (with the per-token
+    values of its rows), so a slice of a large batch costs only its rows."""
     T = wl.tokens if tokens is None else int(tokens)
-    rng = _rng(wl.data_seed * 1000 + stream)
-    x = rng.standard_normal((T, d), dtype=np.float32)
+    r0, r1 = (0, T) if rows is None else (int(rows[0]), int(rows[1]))
+    if not 0 <= r0 <= r1 <= T:
+        raise ValueError("rows must lie inside the batch")
+    seed = wl.data_seed * 1000 + stream
+    meta = _rng(seed)
     if wl.recipe == "gauss_outlier4x30":
-        ch = rng.choice(d, 4, replace=False)
-        x[:, ch] *= np.float32(30.0)
+        ch = meta.choice(d, 4, replace=False)
     elif wl.recipe == "lognormal_token_t2":
-        n_out = int(round(0.01 * d))
-        ch = rng.choice(d, n_out, replace=False)
-        x[:, ch] = rng.standard_t(2.0, size=(T, n_out)).astype(np.float32) * np.float32(20.0)
-        x *= np.exp(rng.standard_normal((T, 1), dtype=np.float32))
-        if gelu:
-            x = _gelu_tanh(x)
+        ch = meta.choice(d, int(round(0.01 * d)), replace=False)
     elif wl.recipe == "frame_drift":
-        frames = 21
-        f = (np.arange(T) * frames) // max(T, 1)
-        x *= (0.5 + 3.5 * f / (frames - 1)).astype(np.float32)[:, None]
-        ch = rng.choice(d, 8, replace=False)
-        x[:, ch] *= np.float32(50.0)
+        ch = meta.choice(d, 8, replace=False)
     elif wl.recipe == "gauss_outlier_half_pct_x100":
-        ch = rng.choice(d, int(round(0.005 * d)), replace=False)
-        x[:, ch] *= np.float32(100.0)
+        ch = meta.choice(d, int(round(0.005 * d)), replace=False)
     else:
         raise ValueError(wl.recipe)
-    if wl.x_dtype == "fp32":
-        return x
-    return f32_to_bf16_bits(x)
+    out = np.empty((r1 - r0, d), dtype=np.float32 if wl.x_dtype == "fp32" else np.uint16)
+    for b in range(r0 // ROW_BLOCK, (r1 + ROW_BLOCK - 1) // ROW_BLOCK):
+        b0, b1 = b * ROW_BLOCK, min((b + 1) * ROW_BLOCK, T)
+        rng = _rng(seed, b)
+        x = rng.standard_normal((b1 - b0, d), dtype=np.float32)
+        if wl.recipe == "gauss_outlier4x30":
+            x[:, ch] *= np.float32(30.0)
+        elif wl.recipe == "lognormal_token_t2":
+            # heavy-tailed outlier channels, then a log-normal scale per token
+            x[:, ch] = rng.standard_t(2.0, size=(b1 - b0, len(ch))).astype(np.float32) * np.float32(20.0)
+            x *= np.exp(rng.standard_normal((b1 - b0, 1), dtype=np.float32))
+            if gelu:
+                x = _gelu_tanh(x)
+        elif wl.recipe == "frame_drift":
+            # 21 frames of equal token counts, scale drifting from x0.5 to x4
+            frames = 21
+            f = (np.arange(b0, b1) * frames) // max(T, 1)
+            x *= (0.5 + 3.5 * f / (frames - 1)).astype(np.float32)[:, None]
+            x[:, ch] *= np.float32(50.0)
+        else:
+            x[:, ch] *= np.float32(100.0)
+        lo, hi = max(b0, r0), min(b1, r1)
+        part = x[lo - b0:hi - b0]
+        out[lo - r0:hi - r0] = part if wl.x_dtype == "fp32" else f32_to_bf16_bits(part)
+    return out
 
 
 def weights(wl: Workload, layer: LayerShape) -> np.ndarray:

@@ -76,3 +76,31 @@ def check_linear(y_gpu: np.ndarray, words_a: np.ndarray, s_gpu: np.ndarray, word
         big = np.abs(y_or) >= frac * rms
         plain[name] = float((err[big] / np.abs(y_or[big])).max()) if big.any() else 0.0
     return {"max_bound_rel": worst, **plain}
+
+
+def check_code_rows(job):
+    """Oracle check of one block of rows of a large batch, run in a worker
+    process: draws the rows of the workload again (the generator draws any row
+    block on its own), rotates and quantizes them in fp64 and compares the
+    GPU's codes and norms.  Returns counts for the caller to bound."""
+    from quantized_linear_token_b200 import workloads as W
+    wl_key, layer_name, T, r0, r1, gelu, stream, codes_gpu, s_gpu = job
+    wl = W.WORKLOADS[wl_key]
+    lay = next(l for l in wl.layers if l.name == layer_name)
+    d = lay.d_in
+    x = W.activations(wl, d, tokens=T, gelu=gelu, stream=stream, rows=(r0, r1))
+    x64 = O.bf16_bits_to_f64(x) if x.dtype == np.uint16 else x.astype(np.float64)
+    cb = O.lloyd_max(d, lay.a_bits)
+    codes_or, s_or, u_or = O.rotate_quantize(x64, O.rpbh_permutation(d, W.ROTATION_SEED),
+                                             O.hadamard_block_size(d), cb)
+    mism = codes_gpu.astype(np.int64) != codes_or
+    n_mis = int(mism.sum())
+    outside = 0
+    max_step = 0
+    if n_mis:
+        band = O.threshold_distance(u_or[mism], cb.thresholds) < CODE_BAND / math.sqrt(d)
+        outside = int((~band).sum())
+        max_step = int(np.abs(codes_gpu.astype(np.int64)[mism] - codes_or[mism]).max())
+    norm_rel = float(np.max(np.abs(s_gpu.astype(np.float64) - s_or) / np.where(s_or > 0, s_or, 1.0)))
+    return {"rows": (r0, r1), "coords": int(codes_or.size), "mismatches": n_mis, "outside_band": outside,
+            "max_step": max_step, "norm_rel": norm_rel}

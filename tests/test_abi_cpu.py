@@ -103,6 +103,7 @@ def test_argument_checks(lib):
     assert lib.oq_linear_fused_host_workspace_size(None, 0, 10) == 0
     assert lib.oq_linear_fused_host(None, None, 0, 4, None, None, None, None, 0, None) == 1
     assert lib.oq_rotation_build(0, 0, 0, None, None) == 1
+    assert lib.oq_check_wait_timeout(None, 1000, None) == 1
     assert b"" != lib.oq_status_string(2)
     with pytest.raises(B.OrbitQuantError):
         B.oq_codebook_build(256, 9)

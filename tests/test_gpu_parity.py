@@ -448,6 +448,27 @@ def test_degenerate_tokens(env, d_in, d_out):
         assert float(s2[1]) == 0.0 and np.all(a16[1].cpu().numpy().view(np.uint16) == mid)
 
 
+def test_bounded_wait_timeout(env):
+    # the failure path every kernel shares: a bounded wait that runs out (an
+    # mbarrier nobody arrives on, 2 ms bound) sets the layer's error word and
+    # returns, the kernel ends, oq_poll_error reports OQ_ERR_TIMEOUT once and
+    # clears the word, and the context and the layer keep working
+    torch, B = env
+    x_np, Wm = _inputs("pr1", 256, 256, 64)
+    layer = B.oq_layer_create(256, 256, 0, 4, 4, 0)
+    B.oq_poll_error(layer)
+    B.oq_check_wait_timeout(layer, 2000)
+    with pytest.raises(B.OrbitQuantError) as err:
+        B.oq_poll_error(layer)
+    assert err.value.status == 4
+    B.oq_poll_error(layer)                      # cleared
+    with pytest.raises(B.OrbitQuantError):
+        B.oq_check_wait_timeout(layer, 0)
+    with pytest.raises(B.OrbitQuantError):
+        B.oq_check_wait_timeout(layer, 2_000_000)
+    _run_layer(env, 256, 256, 4, 4, x_np, Wm, label="after timeout")
+
+
 def test_empty_batch(env):
     torch, B = env
     layer = B.oq_layer_create(256, 256, 0, 4, 4, 0)
