@@ -72,7 +72,7 @@ def _levels_to_codes(a16_bits: np.ndarray, levels_f16: np.ndarray) -> np.ndarray
     pos = np.minimum(np.searchsorted(levels_f16[order], a16_bits), len(order) - 1)
     bad = levels_f16[order][pos] != a16_bits
     assert not bad.any(), f"{int(bad.sum())} values of the A operand are no codebook level"
-    return order[pos].astype(np.int8)
+    return order[pos].astype(np.uint8)          # codes of up to 8 bits
 
 
 @pytest.mark.parametrize("wl_key,layer_name,T,gelu,stream", FULL,
