@@ -429,6 +429,12 @@ static bool fused_w16_route(const oq_layer* L, int32_t x_dtype, int64_t T) {
 
 static size_t fused_w16_bytes(const oq_layer* L) { return round256((size_t)L->d_out * (size_t)L->d_in * 2); }
 
+// the workspace of the large-batch route: the least workspace, the decoded
+// weights, and the fused kernel's row-group flags
+static size_t full_workspace(const oq_layer* L, int64_t T, size_t base) {
+  return round256(base) + fused_w16_bytes(L) + round256(fused_flag_bytes(T));
+}
+
 // the least workspace oq_linear_fused accepts (without the decoded weights)
 static size_t min_workspace(const oq_layer* L, int64_t T) {
   if (!L || T <= 0 || L->int4_only) return 0;
@@ -439,12 +445,12 @@ static size_t min_workspace(const oq_layer* L, int64_t T) {
 
 size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
   const size_t base = min_workspace(L, T);
-  if (base && fused_w16_route(L, OQ_DTYPE_BF16, T)) return round256(base) + fused_w16_bytes(L);
+  if (base && fused_w16_route(L, OQ_DTYPE_BF16, T)) return full_workspace(L, T, base);
   return base;
 }
 
-static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint16_t* a16, float* s,
-                           void* stream) {
+static RQArgs rq_levels_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint16_t* a16,
+                             float* s) {
   RQArgs a{};
   a.src = x;
   a.src_dtype = x_dtype;
@@ -466,6 +472,12 @@ static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, in
   a.bins_full = L->bins_a_full.d_levels;
   a.nb_full = L->bins_a_full.nb;
   a.b0_full = L->bins_a_full.b0;
+  return a;
+}
+
+static oq_status rq_levels(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, uint16_t* a16, float* s,
+                           void* stream) {
+  const RQArgs a = rq_levels_args(L, x, x_dtype, T, a16, s);
   if (rqtc_supported(a)) {
     const oq_status st = rqtc_launch(a, stream);
     if (st != OQ_ERR_UNSUPPORTED) return st;   // else (shared memory too small): the two-pass kernel
@@ -512,9 +524,8 @@ oq_status oq_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* 
   return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_weight_levels: unsupported shape") : st;
 }
 
-static oq_status linear_w16(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
-                            const float* r, float* y, void* stream) {
-  if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
+static GemmArgs w16_args(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
+                         const float* r, float* y) {
   GemmArgs g{};
   g.a_f16 = a16;
   g.b_f16 = w16;
@@ -528,7 +539,13 @@ static oq_status linear_w16(const oq_layer* L, const uint16_t* a16, const float*
   g.a_bits = L->a_bits;
   g.b_bits = L->w_bits;
   g.err = L->d_error;
-  const oq_status st = gemm_w16_launch(g, stream);
+  return g;
+}
+
+static oq_status linear_w16(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
+                            const float* r, float* y, void* stream) {
+  if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
+  const oq_status st = gemm_w16_launch(w16_args(L, a16, s, T, w16, r, y), stream);
   return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_decoded: unsupported shape") : st;
 }
 
@@ -588,17 +605,30 @@ static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype,
   if (fused_f16_route(L, x_dtype)) {
     uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
     float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
-    st = rq_levels(L, x, x_dtype, T, a16, s, stream);
-    if (st != OQ_OK) return st;
-    if (w16_ready) return linear_w16(L, a16, s, T, w16_ready, r, y, stream);
+    if (w16_ready) {
+      st = rq_levels(L, x, x_dtype, T, a16, s, stream);
+      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16_ready, r, y, stream);
+    }
     // large batches with room for the decoded weights: decode them once, then
-    // contract two fp16 operands; otherwise decode weights inside the contraction
-    if (fused_w16_route(L, x_dtype, T) && workspace_bytes >= round256(need) + fused_w16_bytes(L)) {
+    // contract two fp16 operands -- in the fused kernel, whose producer teams
+    // write the A operand while the contraction runs, where it applies;
+    // otherwise decode weights inside the contraction
+    if (fused_w16_route(L, x_dtype, T) && workspace_bytes >= full_workspace(L, T, need)) {
+      if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
       uint16_t* w16 = reinterpret_cast<uint16_t*>(ws + round256(need));
       st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
       if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_fused: unsupported shape") : st;
-      return linear_w16(L, a16, s, T, w16, r, y, stream);
+      const RQArgs ra = rq_levels_args(L, x, x_dtype, T, a16, s);
+      if (fused_kernel_supported(ra, L->d_out)) {
+        int* flags = reinterpret_cast<int*>(ws + round256(need) + fused_w16_bytes(L));
+        st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y), flags, stream);
+        if (st != OQ_ERR_UNSUPPORTED) return st;
+      }
+      st = rq_levels(L, x, x_dtype, T, a16, s, stream);
+      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16, r, y, stream);
     }
+    st = rq_levels(L, x, x_dtype, T, a16, s, stream);
+    if (st != OQ_OK) return st;
     return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
   }
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws);
@@ -659,7 +689,7 @@ oq_status oq_check_wait_timeout(const oq_layer* L, uint32_t limit_us, void* stre
 
 namespace oq {
 size_t fused_min_workspace(const oq_layer* L, int64_t T) { return min_workspace(L, T); }
-size_t fused_w16_workspace(const oq_layer* L, int64_t T) { return round256(min_workspace(L, T)) + fused_w16_bytes(L); }
+size_t fused_w16_workspace(const oq_layer* L, int64_t T) { return full_workspace(L, T, min_workspace(L, T)); }
 bool fused_decodes_weights(const oq_layer* L, int32_t x_dtype, int64_t T) { return fused_w16_route(L, x_dtype, T); }
 oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
                            const float* r, const float* y, const void* workspace, const char* who) {

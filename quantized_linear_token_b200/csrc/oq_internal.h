@@ -143,6 +143,12 @@ oq_status levels_launch(const uint32_t* codes, int64_t rows, int K, int bits, co
 oq_status gemm_w16_launch(const GemmArgs& g, void* stream);
 // the fused call decodes the weights once per call from this many tokens on
 constexpr int64_t W16_MIN_T = 1024;
+// the fused layer kernel (oq_fused.cu): rotate-quantize producer teams inside
+// the CTA-pair contraction of the decoded weights.  `flags` is zeroed
+// workspace of fused_flag_bytes(T) bytes (cleared by the launch itself).
+bool fused_kernel_supported(const RQArgs& a, int N);
+size_t fused_flag_bytes(int64_t T);
+oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream);
 // the fused call's pieces for the host-buffer pipeline (oq_api.cu): the least
 // workspace; the workspace with the decoded weights after it; whether the
 // fused call decodes the weights once at this batch size; argument checks;
