@@ -84,12 +84,19 @@ struct FusedParams {
 constexpr int RG = 4;              // token rows per queue group: 32 groups per 128-row tile
 
 // Waits (bounded) until the `cnt` (<= 32) flags at f are all set, polling
-// with every lane of the warp.
+// with every lane of the warp.  Each lane turns the relaxed read that saw its
+// flag set into an acquire with a fence, and the warp then synchronises, so
+// everything the producers wrote before their releases is visible to the
+// lane that goes on to issue the TMA loads.
 __device__ __forceinline__ bool wait_flags(const int* f, int cnt, int lane, int* err) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     const int v = lane < cnt ? ld_relaxed_gpu(f + lane) : 1;
-    if (__all_sync(0xffffffffu, v != 0)) return true;
+    if (__all_sync(0xffffffffu, v != 0)) {
+      fence_acq_rel_gpu();
+      __syncwarp();
+      return true;
+    }
     // the lanes decide together, so the warp leaves the loop as one
     if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > OQ_WAIT_NS)) {
       if (lane == 0) atomicOr(err, OQ_DEVERR_TIMEOUT);
@@ -256,7 +263,6 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
       ok = wait_flags(p.flags + first, cnt, lane, p.err);
       if (!ok) break;
       if (lane == 0) {
-        fence_acq_rel_gpu();
         fence_proxy_async_global();
         for (int kb = 0; kb < nkb; ++kb) {
           if (n > 0 && !mbar_wait(&op_empty[s], (n - 1) & 1u, p.err)) {
