@@ -174,6 +174,29 @@ oq_status oq_layer_get_info(const oq_layer* layer, oq_layer_info* out);
 oq_status oq_layer_get_perm(const oq_layer* layer, uint32_t* perm);
 
 /*
+ * oq_weight_save / oq_weight_load -- prepared weights on disk, so that the
+ * offline step (oq_weight_prepare; hotpaper.ai abstract: the rotation is
+ * folded into the weight rows once) need not run again in a later process.
+ * The file carries the layer's d_in, d_out, a_bits, w_bits, flags and seed
+ * and a hash of both codebooks, then r [d_out] fp32 and Wcodes [d_out,
+ * d_in*w_bits/32] uint32 (little-endian, format version 1).
+ *   oq_weight_save  copies Wcodes and r (device, from oq_weight_prepare) to
+ *                   the host and writes `path` (through a temporary file that
+ *                   is renamed into place).  Synchronous.
+ *   oq_weight_load  reads `path`, checks every header field against `layer`,
+ *                   and copies the weights into Wcodes and r (device,
+ *                   caller-owned, the sizes oq_weight_prepare fills).
+ *                   Synchronous.
+ * Errors: OQ_ERR_INVALID_ARG for a null argument, a file that cannot be
+ * opened or written, a file that is not a prepared-weight file, is truncated
+ * or was prepared for a layer with other settings or codebooks;
+ * OQ_ERR_UNSUPPORTED for an unknown format version; OQ_ERR_CUDA for a failed
+ * copy.
+ */
+oq_status oq_weight_save(const oq_layer* layer, const uint32_t* Wcodes, const float* r, const char* path);
+oq_status oq_weight_load(const oq_layer* layer, const char* path, uint32_t* Wcodes, float* r);
+
+/*
  * oq_rotate_quantize -- online activation codec (gecl notes Method 1, 2, 4):
  *   s[t] = ||x[t]||_2,  u = R x[t] / s[t],  codes[t, i] = #{j : t_j < u_i}.
  *   x      device [T, d_in], bf16 (OQ_DTYPE_BF16) or fp32 (OQ_DTYPE_F32).
@@ -223,11 +246,18 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
  * bytes of the fastest route: the A operand and the norms, and from 1024
  * tokens on (bf16 x, d_out % 256 == 0) also 2 d_out d_in bytes for the
  * weights' fp16 levels, which are then decoded once per call
- * (oq_weight_levels) and contracted with oq_linear_decoded's kernel.  A
- * smaller workspace that still holds the A operand and the norms is accepted
- * and decodes the weights inside the contraction instead; the y values are
- * the same up to fp32 summation order.  Errors: OQ_ERR_INVALID_ARG when the
- * workspace is below that least size.
+ * (oq_weight_levels), and about T bytes of row-group flags.  That route
+ * contracts the two fp16 operands on CTA pairs; where the block size is 1024
+ * or 512 (at most 12 warps per token row) one kernel does both steps, its
+ * rotate-quantize warps writing the A operand while the contraction of
+ * earlier tiles runs, otherwise oq_rotate_quantize_levels' kernel and
+ * oq_linear_decoded's kernel run in turn; y is the same bit for bit.  A
+ * smaller workspace that still holds the A operand and the norms (the least
+ * size: 2 T d_in bytes rounded up to a multiple of 256, plus 4 T, on the
+ * fp16-level route) is accepted and decodes the weights inside the
+ * contraction instead; the y values are the same up to fp32 summation
+ * order.  Errors: OQ_ERR_INVALID_ARG when the workspace is below that least
+ * size.
  */
 size_t oq_linear_fused_workspace_size(const oq_layer* layer, int64_t T);
 oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,

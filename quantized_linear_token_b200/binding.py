@@ -30,7 +30,8 @@ W16_MIN_T = 1024
 # every symbol include/orbitquant.h declares
 EXPORTS = (
     "oq_codebook_build", "oq_rotation_build", "oq_layer_create", "oq_layer_destroy", "oq_layer_get_info", "oq_layer_get_perm",
-    "oq_rotate_quantize", "oq_weight_prepare", "oq_linear", "oq_linear_fused_workspace_size",
+    "oq_rotate_quantize", "oq_weight_prepare", "oq_weight_save", "oq_weight_load", "oq_linear",
+    "oq_linear_fused_workspace_size",
     "oq_linear_fused", "oq_rotate_quantize_levels", "oq_linear_levels", "oq_weight_levels", "oq_linear_decoded",
     "oq_linear_fused_static", "oq_linear_fused_host_workspace_size", "oq_linear_fused_host",
     "oq_poll_error", "oq_check_wait_timeout", "oq_last_error", "oq_status_string",
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH):
         "oq_linear_fused_host": (i32, [vp, vp, i32, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]),
         "oq_linear_decoded": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
         "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
+        "oq_weight_save": (i32, [vp, vp, vp, ctypes.c_char_p]),
+        "oq_weight_load": (i32, [vp, ctypes.c_char_p, vp, vp]),
         "oq_poll_error": (i32, [vp]),
         "oq_check_wait_timeout": (i32, [vp, ctypes.c_uint32, vp]),
         "oq_last_error": (ctypes.c_char_p, []),
@@ -356,6 +359,26 @@ def oq_linear_fused_static(layer: Layer, x, Wcodes, r, y=None):
                                                  _dev(Wcodes, "Wcodes"), _dev(r, "r"), _dev(y, "y"), _stream(x)),
            "oq_linear_fused_static")
     return y
+
+
+def oq_weight_save(layer: Layer, Wcodes, r, path: str) -> None:
+    """Write prepared weights (device Wcodes, r from oq_weight_prepare) to a file."""
+    _check(load_library().oq_weight_save(layer.handle, _dev(Wcodes, "Wcodes"), _dev(r, "r"),
+                                         os.fsencode(path)), "oq_weight_save")
+
+
+def oq_weight_load(layer: Layer, path: str, Wcodes=None, r=None):
+    """Read prepared weights saved for a layer with the same settings ->
+    (Wcodes, r) on the current CUDA device."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    if Wcodes is None:
+        Wcodes = torch.empty((layer.d_out, layer.w_words_per_row), dtype=torch.int32, device=dev)
+    if r is None:
+        r = torch.empty((layer.d_out,), dtype=torch.float32, device=dev)
+    _check(load_library().oq_weight_load(layer.handle, os.fsencode(path), _dev(Wcodes, "Wcodes"), _dev(r, "r")),
+           "oq_weight_load")
+    return Wcodes, r
 
 
 def oq_poll_error(layer: Layer) -> None:

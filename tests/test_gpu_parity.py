@@ -363,7 +363,8 @@ def test_decoded_weight_route(env, d_in, d_out, a_bits, w_bits, T):
     y_full = B.oq_linear_fused(layer, x_t, Wc, r)
     a16, s = B.oq_rotate_quantize_levels(layer, x_t)
     y_stage = B.oq_linear_decoded(layer, a16, s, B.oq_weight_levels(layer, Wc), r)
-    least = full - ((d_out * d_in * 2 + 255) // 256) * 256
+    # the least workspace: the fp16 A operand (rounded up to 256 bytes) and the norms
+    least = (T * d_in * 2 + 255) // 256 * 256 + T * 4
     ws = torch.empty((least,), dtype=torch.uint8, device="cuda")
     y_least = B.oq_linear_fused(layer, x_t, Wc, r, workspace=ws)
     y_lv = B.oq_linear_levels(layer, a16, s, Wc, r)
@@ -467,6 +468,40 @@ def test_bounded_wait_timeout(env):
     with pytest.raises(B.OrbitQuantError):
         B.oq_check_wait_timeout(layer, 2_000_000)
     _run_layer(env, 256, 256, 4, 4, x_np, Wm, label="after timeout")
+
+
+def test_prepared_weight_file(env, tmp_path):
+    # prepared weights saved with their layer's settings load back bit for bit
+    # into a layer built the same way, give the same y, and are refused by a
+    # layer with other settings or by a damaged file
+    torch, B = env
+    d_in, d_out, T = 1024, 256, 40
+    x_np = W.custom_activations(T, d_in, seed=21)
+    Wm = W.custom_weights(d_out, d_in, seed=22)
+    layer = B.oq_layer_create(d_in, d_out, 5, 4, 3, 0)
+    x_t, _ = _x_tensor(torch, x_np)
+    Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(Wm).cuda())
+    path = str(tmp_path / "w.oqw")
+    B.oq_weight_save(layer, Wc, r, path)
+    again = B.oq_layer_create(d_in, d_out, 5, 4, 3, 0)
+    Wc2, r2 = B.oq_weight_load(again, path)
+    torch.cuda.synchronize()
+    assert torch.equal(Wc2, Wc) and torch.equal(r2.view(torch.int32), r.view(torch.int32))
+    np.testing.assert_array_equal(B.oq_linear_fused(again, x_t, Wc2, r2).cpu().numpy(),
+                                  B.oq_linear_fused(layer, x_t, Wc, r).cpu().numpy())
+    for other in (B.oq_layer_create(d_in, d_out, 6, 4, 3, 0),                    # seed
+                  B.oq_layer_create(d_in, d_out, 5, 4, 4, 0),                    # weight bits
+                  B.oq_layer_create(d_in, d_out, 5, 4, 3, B.OQ_FLAG_GAUSSIAN_MARGINAL),   # codebooks
+                  B.oq_layer_create(d_in, 512, 5, 4, 3, 0)):                     # shape
+        with pytest.raises(B.OrbitQuantError):
+            B.oq_weight_load(other, path)
+    raw = open(path, "rb").read()
+    for bad in (raw[:-4], b"X" + raw[1:], raw + b"\0"):
+        with open(path, "wb") as f:
+            f.write(bad)
+        with pytest.raises(B.OrbitQuantError):
+            B.oq_weight_load(again, path)
+    B.oq_poll_error(layer)
 
 
 def test_empty_batch(env):
