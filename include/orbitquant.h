@@ -63,6 +63,8 @@ typedef enum {
                                does not define (reserved)                    */
 } oq_status;
 
+/* Element types of x, W and y.  y (the contraction calls' output) is fp32 or
+ * bf16 (rounded to nearest even in the epilogue, from the fp32 result). */
 enum { OQ_DTYPE_F32 = 0, OQ_DTYPE_BF16 = 1 };
 
 /* Layer / codebook flags. */
@@ -225,13 +227,14 @@ oq_status oq_weight_prepare(const oq_layer* layer, const void* W, int32_t W_dtyp
  * Method 1-2; pith Figure 2):
  *   y[t, o] = s[t] r[o] sum_i C_w[Wcodes[o, i]] C_a[codes[t, i]]
  *   codes, s   from oq_rotate_quantize; Wcodes, r from oq_weight_prepare.
- *   y          device [T, d_out] fp32.
+ *   y          device [T, d_out], fp32 (y_dtype OQ_DTYPE_F32) or bf16
+ *              (OQ_DTYPE_BF16: the fp32 result rounded to nearest even).
  * Runs on the tcgen05 tensor cores: both operands are decoded to fp16 levels
  * (scaled per codebook for exact-as-possible fp16 values), accumulated in
  * fp32 in tensor memory, and rescaled in the epilogue.
  */
 oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s, int64_t T,
-                    const uint32_t* Wcodes, const float* r, float* y, void* stream);
+                    const uint32_t* Wcodes, const float* r, void* y, int32_t y_dtype, void* stream);
 
 /*
  * oq_linear_fused -- x -> y in one call: the rotate-quantize step produces
@@ -261,7 +264,7 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
  */
 size_t oq_linear_fused_workspace_size(const oq_layer* layer, int64_t T);
 oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
-                          const uint32_t* Wcodes, const float* r, float* y,
+                          const uint32_t* Wcodes, const float* r, void* y, int32_t y_dtype,
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
@@ -289,7 +292,8 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  * oq_linear_levels -- oq_linear with the A operand given as those fp16
  * levels (read by TMA; only the weight codes are decoded):
  *   y[t, o] = s[t] r[o] / (a_scale w_scale) sum_i a16[t, i] fp16(w_scale C_w[Wcodes[o, i]])
- *   Needs d_out % 256 == 0 (else OQ_ERR_UNSUPPORTED); y 16-byte aligned.
+ *   Needs d_out % 256 == 0 (else OQ_ERR_UNSUPPORTED); y 16-byte aligned,
+ *   fp32 or bf16 as y_dtype says.
  *
  * oq_weight_levels -- the weights' operand as fp16 levels, decoded once
  * (gecl notes Limitation 3: the centroid lookup of every code):
@@ -303,8 +307,9 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  * for large batches):
  *   y[t, o] = s[t] r[o] / (a_scale w_scale) sum_i a16[t, i] w16[o, i]
  *   a16, s from oq_rotate_quantize_levels; w16 from oq_weight_levels; r from
- *   oq_weight_prepare (16-byte aligned); y device [T, d_out] fp32, 16-byte
- *   aligned.  Needs d_out % 256 == 0 (else OQ_ERR_UNSUPPORTED).
+ *   oq_weight_prepare (16-byte aligned); y device [T, d_out], fp32 or bf16
+ *   as y_dtype says, 16-byte aligned.  Needs d_out % 256 == 0 (else
+ *   OQ_ERR_UNSUPPORTED).
  *
  * oq_rotate_quantize_levels followed by oq_linear_levels gives exactly the y
  * of oq_linear_fused for T < 1024, and followed by oq_weight_levels +
@@ -316,15 +321,16 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  * across the SMs (the batch-1 / GEMV end of the workload sweep); the splits of
  * a tile add into y in a fixed order through per-layer counters, so results
  * repeat bit for bit, and calls on one layer must not overlap on the GPU
- * (different streams or host threads).
+ * (different streams or host threads).  With bf16 y those batches take the
+ * CTA-pair kernel instead (the splits add in fp32 in y itself).
  */
 oq_status oq_rotate_quantize_levels(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
                                     uint16_t* a16, float* s, void* stream);
 oq_status oq_linear_levels(const oq_layer* layer, const uint16_t* a16, const float* s, int64_t T,
-                           const uint32_t* Wcodes, const float* r, float* y, void* stream);
+                           const uint32_t* Wcodes, const float* r, void* y, int32_t y_dtype, void* stream);
 oq_status oq_weight_levels(const oq_layer* layer, const uint32_t* Wcodes, uint16_t* w16, void* stream);
 oq_status oq_linear_decoded(const oq_layer* layer, const uint16_t* a16, const float* s, int64_t T,
-                            const uint16_t* w16, const float* r, float* y, void* stream);
+                            const uint16_t* w16, const float* r, void* y, int32_t y_dtype, void* stream);
 
 /*
  * oq_linear_fused_static -- the same computation as oq_linear_fused for
@@ -341,7 +347,7 @@ oq_status oq_linear_decoded(const oq_layer* layer, const uint16_t* a16, const fl
  *   that device current); make that first call before any stream capture.
  *   Every call shares the array: calls that overlap on the GPU (different
  *   streams or host threads) race and give wrong results.
- *   Arguments as for oq_linear_fused.  The array serves as its least
+ *   Arguments as for oq_linear_fused, with fp32 y.  The array serves as its least
  *   workspace (the A operand and the norms), so the weights are decoded
  *   inside the contraction at every batch size and y is that of
  *   oq_linear_fused given that least workspace, bit for bit.  Errors:
@@ -359,7 +365,7 @@ oq_status oq_linear_fused_static(const oq_layer* layer, const void* x, int32_t x
  * them).  The pages have no counterpart; this is the interface for callers
  * whose activations live in host memory.
  *   x_host     host [T, d_in] bf16 (OQ_DTYPE_BF16) or fp32 (OQ_DTYPE_F32).
- *   y_host     host [T, d_out] fp32.
+ *   y_host     host [T, d_out], fp32 or bf16 as y_dtype says.
  *   Wcodes, r  device, from oq_weight_prepare.
  *   workspace  device scratch of oq_linear_fused_host_workspace_size(layer,
  *              x_dtype, T) bytes, 256-byte aligned.
@@ -375,8 +381,8 @@ oq_status oq_linear_fused_static(const oq_layer* layer, const void* x, int32_t x
  */
 size_t oq_linear_fused_host_workspace_size(const oq_layer* layer, int32_t x_dtype, int64_t T);
 oq_status oq_linear_fused_host(const oq_layer* layer, const void* x_host, int32_t x_dtype, int64_t T,
-                               const uint32_t* Wcodes, const float* r, float* y_host, void* workspace,
-                               size_t workspace_bytes, void* stream);
+                               const uint32_t* Wcodes, const float* r, void* y_host, int32_t y_dtype,
+                               void* workspace, size_t workspace_bytes, void* stream);
 
 /* Reads and clears the layer's device error word.  Synchronizes the device.
  * Returns OQ_OK or OQ_ERR_TIMEOUT (OQ_ERR_DEVICE for a bit this version does

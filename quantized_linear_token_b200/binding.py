@@ -84,15 +84,15 @@ def load_library(path: str = LIB_PATH):
         "oq_layer_get_perm": (i32, [vp, vp]),
         "oq_rotate_quantize": (i32, [vp, vp, i32, i64, vp, vp, vp]),
         "oq_weight_prepare": (i32, [vp, vp, i32, vp, vp, vp]),
-        "oq_linear": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
+        "oq_linear": (i32, [vp, vp, vp, i64, vp, vp, vp, i32, vp]),
         "oq_linear_fused_workspace_size": (sz, [vp, i64]),
-        "oq_linear_fused": (i32, [vp, vp, i32, i64, vp, vp, vp, vp, sz, vp]),
+        "oq_linear_fused": (i32, [vp, vp, i32, i64, vp, vp, vp, i32, vp, sz, vp]),
         "oq_rotate_quantize_levels": (i32, [vp, vp, i32, i64, vp, vp, vp]),
-        "oq_linear_levels": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
+        "oq_linear_levels": (i32, [vp, vp, vp, i64, vp, vp, vp, i32, vp]),
         "oq_weight_levels": (i32, [vp, vp, vp, vp]),
         "oq_linear_fused_host_workspace_size": (ctypes.c_size_t, [vp, i32, i64]),
-        "oq_linear_fused_host": (i32, [vp, vp, i32, i64, vp, vp, vp, vp, ctypes.c_size_t, vp]),
-        "oq_linear_decoded": (i32, [vp, vp, vp, i64, vp, vp, vp, vp]),
+        "oq_linear_fused_host": (i32, [vp, vp, i32, i64, vp, vp, vp, i32, vp, ctypes.c_size_t, vp]),
+        "oq_linear_decoded": (i32, [vp, vp, vp, i64, vp, vp, vp, i32, vp]),
         "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
         "oq_weight_save": (i32, [vp, vp, vp, ctypes.c_char_p]),
         "oq_weight_load": (i32, [vp, ctypes.c_char_p, vp, vp]),
@@ -232,14 +232,25 @@ def oq_weight_prepare(layer: Layer, W, Wcodes=None, r=None):
     return Wcodes, r
 
 
-def oq_linear(layer: Layer, codes, s, Wcodes, r, y=None):
-    """(codes, s, Wcodes, r) -> y [T, d_out] fp32."""
+def _y_out(y, T: int, d_out: int, y_dtype, device):
+    """The output tensor (given, or new of y_dtype: torch.float32 or
+    torch.bfloat16) and its C dtype code."""
     torch = _torch()
-    T = codes.shape[0]
     if y is None:
-        y = torch.empty((T, layer.d_out), dtype=torch.float32, device=codes.device)
+        y = torch.empty((T, d_out), dtype=torch.float32 if y_dtype is None else y_dtype, device=device)
+    if y.dtype == torch.float32:
+        return y, OQ_DTYPE_F32
+    if y.dtype == torch.bfloat16:
+        return y, OQ_DTYPE_BF16
+    raise ValueError("y must be float32 or bfloat16")
+
+
+def oq_linear(layer: Layer, codes, s, Wcodes, r, y=None, y_dtype=None):
+    """(codes, s, Wcodes, r) -> y [T, d_out] fp32 (or bf16)."""
+    T = codes.shape[0]
+    y, ycode = _y_out(y, T, layer.d_out, y_dtype, codes.device)
     _check(load_library().oq_linear(layer.handle, _dev(codes, "codes"), _dev(s, "s"), T, _dev(Wcodes, "Wcodes"),
-                                    _dev(r, "r"), _dev(y, "y"), _stream(codes)), "oq_linear")
+                                    _dev(r, "r"), _dev(y, "y"), ycode, _stream(codes)), "oq_linear")
     return y
 
 
@@ -247,17 +258,16 @@ def oq_linear_fused_workspace_size(layer: Layer, T: int) -> int:
     return int(load_library().oq_linear_fused_workspace_size(layer.handle, T))
 
 
-def oq_linear_fused(layer: Layer, x, Wcodes, r, y=None, workspace=None):
-    """x [T, d_in] -> y [T, d_out] fp32 in one call."""
+def oq_linear_fused(layer: Layer, x, Wcodes, r, y=None, workspace=None, y_dtype=None):
+    """x [T, d_in] -> y [T, d_out] fp32 (or bf16) in one call."""
     torch = _torch()
     T = x.shape[0]
-    if y is None:
-        y = torch.empty((T, layer.d_out), dtype=torch.float32, device=x.device)
+    y, ycode = _y_out(y, T, layer.d_out, y_dtype, x.device)
     need = oq_linear_fused_workspace_size(layer, T)
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=x.device)
     _check(load_library().oq_linear_fused(layer.handle, _dev(x, "x"), _dtype_code(x), T, _dev(Wcodes, "Wcodes"),
-                                          _dev(r, "r"), _dev(y, "y"), _dev(workspace, "workspace"),
+                                          _dev(r, "r"), _dev(y, "y"), ycode, _dev(workspace, "workspace"),
                                           workspace.numel() * workspace.element_size(), _stream(x)),
            "oq_linear_fused")
     return y
@@ -277,15 +287,13 @@ def oq_rotate_quantize_levels(layer: Layer, x, a16=None, s=None):
     return a16, s
 
 
-def oq_linear_levels(layer: Layer, a16, s, Wcodes, r, y=None):
-    """(a16 fp16 levels, s, Wcodes, r) -> y [T, d_out] fp32: the second stage of
-    the fused call's fp16 route."""
-    torch = _torch()
+def oq_linear_levels(layer: Layer, a16, s, Wcodes, r, y=None, y_dtype=None):
+    """(a16 fp16 levels, s, Wcodes, r) -> y [T, d_out] fp32 (or bf16): the
+    second stage of the fused call's fp16 route."""
     T = a16.shape[0]
-    if y is None:
-        y = torch.empty((T, layer.d_out), dtype=torch.float32, device=a16.device)
+    y, ycode = _y_out(y, T, layer.d_out, y_dtype, a16.device)
     _check(load_library().oq_linear_levels(layer.handle, _dev(a16, "a16"), _dev(s, "s"), T, _dev(Wcodes, "Wcodes"),
-                                           _dev(r, "r"), _dev(y, "y"), _stream(a16)), "oq_linear_levels")
+                                           _dev(r, "r"), _dev(y, "y"), ycode, _stream(a16)), "oq_linear_levels")
     return y
 
 
@@ -300,15 +308,13 @@ def oq_weight_levels(layer: Layer, Wcodes, w16=None):
     return w16
 
 
-def oq_linear_decoded(layer: Layer, a16, s, w16, r, y=None):
-    """(a16, s, w16, r) -> y [T, d_out] fp32: the contraction of two fp16 level
-    operands, both read by TMA."""
-    torch = _torch()
+def oq_linear_decoded(layer: Layer, a16, s, w16, r, y=None, y_dtype=None):
+    """(a16, s, w16, r) -> y [T, d_out] fp32 (or bf16): the contraction of two
+    fp16 level operands, both read by TMA."""
     T = a16.shape[0]
-    if y is None:
-        y = torch.empty((T, layer.d_out), dtype=torch.float32, device=a16.device)
+    y, ycode = _y_out(y, T, layer.d_out, y_dtype, a16.device)
     _check(load_library().oq_linear_decoded(layer.handle, _dev(a16, "a16"), _dev(s, "s"), T, _dev(w16, "w16"),
-                                            _dev(r, "r"), _dev(y, "y"), _stream(a16)), "oq_linear_decoded")
+                                            _dev(r, "r"), _dev(y, "y"), ycode, _stream(a16)), "oq_linear_decoded")
     return y
 
 
@@ -324,7 +330,7 @@ def _host(t, name: str):
     return ctypes.c_void_p(t.data_ptr())
 
 
-def oq_linear_fused_host(layer: Layer, x_host, Wcodes, r, y_host=None, workspace=None):
+def oq_linear_fused_host(layer: Layer, x_host, Wcodes, r, y_host=None, workspace=None, y_dtype=None):
     """x_host [T, d_in] bf16/fp32 in host memory (pinned for overlap) -> y_host
     [T, d_out] fp32 in host memory: copies in, the fused call and copies out,
     overlapped chunk by chunk, queued on the current stream of Wcodes' device.
@@ -334,13 +340,16 @@ def oq_linear_fused_host(layer: Layer, x_host, Wcodes, r, y_host=None, workspace
     if x_host.dim() != 2 or x_host.shape[1] != layer.d_in:
         raise ValueError("x_host must be [T, d_in]")
     if y_host is None:
-        y_host = torch.empty((T, layer.d_out), dtype=torch.float32, pin_memory=True)
+        y_host = torch.empty((T, layer.d_out), dtype=torch.float32 if y_dtype is None else y_dtype, pin_memory=True)
+    if y_host.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("y_host must be float32 or bfloat16")
+    ycode = OQ_DTYPE_F32 if y_host.dtype == torch.float32 else OQ_DTYPE_BF16
     code = _dtype_code(x_host)
     need = oq_linear_fused_host_workspace_size(layer, code, T)
     if workspace is None:
         workspace = torch.empty((max(need, 1),), dtype=torch.uint8, device=Wcodes.device)
     _check(load_library().oq_linear_fused_host(layer.handle, _host(x_host, "x_host"), code, T,
-                                               _dev(Wcodes, "Wcodes"), _dev(r, "r"), _host(y_host, "y_host"),
+                                               _dev(Wcodes, "Wcodes"), _dev(r, "r"), _host(y_host, "y_host"), ycode,
                                                _dev(workspace, "workspace"),
                                                workspace.numel() * workspace.element_size(), _stream(Wcodes)),
            "oq_linear_fused_host")

@@ -358,7 +358,7 @@ oq_status oq_weight_prepare(const oq_layer* L, const void* W, int32_t W_dtype, u
 constexpr int64_t MAX_TOKENS = ((int64_t)1 << 31) - 1024;
 
 static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T,
-                             const uint32_t* Wcodes, const float* r, float* y, void* stream,
+                             const uint32_t* Wcodes, const float* r, void* y, bool y_bf16, void* stream,
                              const uint16_t* a_f16 = nullptr) {
   if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
   GemmArgs g{};
@@ -379,6 +379,7 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
     g.out_scale = (float)(1.0 / (L->a8_scale * L->w8_scale));
   }
   g.y = y;
+  g.y_bf16 = y_bf16;
   g.M = T;
   g.N = L->d_out;
   g.K = L->d_in;
@@ -386,21 +387,29 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
   g.b_bits = L->w_bits;
   g.err = L->d_error;
   // a few hundred tokens or fewer: the small-batch kernel (weight rows as the
-  // MMA's M, split K); larger batches: the CTA-pair kernel
-  if (a_f16 && T <= SKINNY_MAX_T && L->d_counters) return gemm_skinny_launch(g, L->d_counters, stream);
+  // MMA's M, split K, its splits added in fp32 in y itself, so fp32 y only);
+  // larger batches and bf16 y: the CTA-pair kernel
+  if (a_f16 && T <= SKINNY_MAX_T && L->d_counters && !y_bf16) return gemm_skinny_launch(g, L->d_counters, stream);
   return gemm_launch(g, stream);
 }
 
+// fp32 or bf16 y
+static oq_status check_y_dtype(int32_t y_dtype, const char* who) {
+  if (y_dtype == OQ_DTYPE_F32 || y_dtype == OQ_DTYPE_BF16) return OQ_OK;
+  return fail(OQ_ERR_INVALID_ARG, std::string(who) + ": y_dtype must be OQ_DTYPE_F32 or OQ_DTYPE_BF16");
+}
+
 oq_status oq_linear(const oq_layer* L, const uint32_t* codes, const float* s, int64_t T, const uint32_t* Wcodes,
-                    const float* r, float* y, void* stream) {
+                    const float* r, void* y, int32_t y_dtype, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear: layer is null");
   if (L->int4_only) return not_for_int4(L, "oq_linear");
+  if (check_y_dtype(y_dtype, "oq_linear") != OQ_OK) return OQ_ERR_INVALID_ARG;
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear: T < 0");
   if (T == 0) return OQ_OK;
   if (!codes || !s || !Wcodes || !r || !y) return fail(OQ_ERR_INVALID_ARG, "oq_linear: null pointer");
   if (!aligned(codes, 16) || !aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(s, 4) || !aligned(r, 16))
     return fail(OQ_ERR_INVALID_ARG, "oq_linear: misaligned pointer");
-  return linear_impl(L, codes, s, T, Wcodes, r, y, stream);
+  return linear_impl(L, codes, s, T, Wcodes, r, y, y_dtype == OQ_DTYPE_BF16, stream);
 }
 
 // The fused call has two routes.  With bf16 activations and d_out % 256 == 0
@@ -501,8 +510,9 @@ oq_status oq_rotate_quantize_levels(const oq_layer* L, const void* x, int32_t x_
 }
 
 oq_status oq_linear_levels(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint32_t* Wcodes,
-                           const float* r, float* y, void* stream) {
+                           const float* r, void* y, int32_t y_dtype, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: layer is null");
+  if (check_y_dtype(y_dtype, "oq_linear_levels") != OQ_OK) return OQ_ERR_INVALID_ARG;
   if (L->int4_only) return not_for_int4(L, "oq_linear_levels");
   if (L->fp8) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_levels: the fp16-level route is not used in the FP8 mode");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: T < 0");
@@ -511,7 +521,7 @@ oq_status oq_linear_levels(const oq_layer* L, const uint16_t* a16, const float* 
   if (!aligned(a16, 16) || !aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(s, 4) || !aligned(r, 16))
     return fail(OQ_ERR_INVALID_ARG, "oq_linear_levels: misaligned pointer");
   if (L->d_out % 256 != 0) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_levels: needs d_out % 256 == 0");
-  return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
+  return linear_impl(L, nullptr, s, T, Wcodes, r, y, y_dtype == OQ_DTYPE_BF16, stream, a16);
 }
 
 oq_status oq_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* w16, void* stream) {
@@ -525,7 +535,7 @@ oq_status oq_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* 
 }
 
 static GemmArgs w16_args(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
-                         const float* r, float* y) {
+                         const float* r, void* y, bool y_bf16) {
   GemmArgs g{};
   g.a_f16 = a16;
   g.b_f16 = w16;
@@ -533,6 +543,7 @@ static GemmArgs w16_args(const oq_layer* L, const uint16_t* a16, const float* s,
   g.b_scale = r;
   g.out_scale = (float)(1.0 / (L->a_scale * L->w_scale));
   g.y = y;
+  g.y_bf16 = y_bf16;
   g.M = T;
   g.N = L->d_out;
   g.K = L->d_in;
@@ -543,15 +554,16 @@ static GemmArgs w16_args(const oq_layer* L, const uint16_t* a16, const float* s,
 }
 
 static oq_status linear_w16(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
-                            const float* r, float* y, void* stream) {
+                            const float* r, void* y, bool y_bf16, void* stream) {
   if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
-  const oq_status st = gemm_w16_launch(w16_args(L, a16, s, T, w16, r, y), stream);
+  const oq_status st = gemm_w16_launch(w16_args(L, a16, s, T, w16, r, y, y_bf16), stream);
   return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_decoded: unsupported shape") : st;
 }
 
 oq_status oq_linear_decoded(const oq_layer* L, const uint16_t* a16, const float* s, int64_t T, const uint16_t* w16,
-                            const float* r, float* y, void* stream) {
+                            const float* r, void* y, int32_t y_dtype, void* stream) {
   if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_decoded: layer is null");
+  if (check_y_dtype(y_dtype, "oq_linear_decoded") != OQ_OK) return OQ_ERR_INVALID_ARG;
   if (L->int4_only) return not_for_int4(L, "oq_linear_decoded");
   if (L->fp8) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_decoded: the fp16-level route is not used in the FP8 mode");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, "oq_linear_decoded: T < 0");
@@ -560,7 +572,7 @@ oq_status oq_linear_decoded(const oq_layer* L, const uint16_t* a16, const float*
   if (!aligned(a16, 16) || !aligned(w16, 16) || !aligned(y, 16) || !aligned(s, 4) || !aligned(r, 16))
     return fail(OQ_ERR_INVALID_ARG, "oq_linear_decoded: misaligned pointer");
   if (L->d_out % 256 != 0) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_decoded: needs d_out % 256 == 0");
-  return linear_w16(L, a16, s, T, w16, r, y, stream);
+  return linear_w16(L, a16, s, T, w16, r, y, y_dtype == OQ_DTYPE_BF16, stream);
 }
 
 // y = x (q r)^T for the INT4 weight-only layer: bf16 x straight into the
@@ -598,8 +610,8 @@ static oq_status int4_linear(const oq_layer* L, const void* x, int32_t x_dtype, 
 // levels, already decoded by the caller (oq_linear_fused_host decodes them
 // once for all its chunks), or null.
 static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                              const float* r, float* y, unsigned char* ws, size_t workspace_bytes, void* stream,
-                              const uint16_t* w16_ready) {
+                              const float* r, void* y, bool y_bf16, unsigned char* ws, size_t workspace_bytes,
+                              void* stream, const uint16_t* w16_ready) {
   oq_status st;
   const size_t need = min_workspace(L, T);
   if (fused_f16_route(L, x_dtype)) {
@@ -607,7 +619,7 @@ static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype,
     float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
     if (w16_ready) {
       st = rq_levels(L, x, x_dtype, T, a16, s, stream);
-      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16_ready, r, y, stream);
+      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16_ready, r, y, y_bf16, stream);
     }
     // large batches with room for the decoded weights: decode them once, then
     // contract two fp16 operands -- in the fused kernel, whose producer teams
@@ -621,32 +633,37 @@ static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype,
       const RQArgs ra = rq_levels_args(L, x, x_dtype, T, a16, s);
       if (fused_kernel_supported(ra, L->d_out)) {
         int* flags = reinterpret_cast<int*>(ws + round256(need) + fused_w16_bytes(L));
-        st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y), flags, stream);
+        st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), flags, stream);
         if (st != OQ_ERR_UNSUPPORTED) return st;
       }
       st = rq_levels(L, x, x_dtype, T, a16, s, stream);
-      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16, r, y, stream);
+      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16, r, y, y_bf16, stream);
     }
     st = rq_levels(L, x, x_dtype, T, a16, s, stream);
     if (st != OQ_OK) return st;
-    return linear_impl(L, nullptr, s, T, Wcodes, r, y, stream, a16);
+    return linear_impl(L, nullptr, s, T, Wcodes, r, y, y_bf16, stream, a16);
   }
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws);
   float* s = reinterpret_cast<float*>(ws + round256(fused_codes_bytes(L, T)));
   st = rq(L, x, x_dtype, T, L->a_bits, L->bins_a, codes, s, stream);
   if (st != OQ_OK) return st;
-  return linear_impl(L, codes, s, T, Wcodes, r, y, stream);
+  return linear_impl(L, codes, s, T, Wcodes, r, y, y_bf16, stream);
 }
 
 static oq_status fused_checks(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                              const float* r, const float* y, const void* workspace, const char* who) {
+                              const float* r, const void* y, int32_t y_dtype, const void* workspace,
+                              const char* who) {
   const std::string w(who);
   if (!L) return fail(OQ_ERR_INVALID_ARG, w + ": layer is null");
   if (T < 0) return fail(OQ_ERR_INVALID_ARG, w + ": T < 0");
   if (T == 0) return OQ_OK;
-  const oq_status st = check_rows_input(x, x_dtype, who);
+  oq_status st = check_rows_input(x, x_dtype, who);
   if (st != OQ_OK) return st;
-  if (L->int4_only) return OQ_OK;
+  if ((st = check_y_dtype(y_dtype, who)) != OQ_OK) return st;
+  if (L->int4_only) {
+    if (y_dtype != OQ_DTYPE_F32) return fail(OQ_ERR_UNSUPPORTED, w + ": the INT4 weight-only layer writes fp32 y");
+    return OQ_OK;
+  }
   if (!Wcodes || !r || !y || !workspace) return fail(OQ_ERR_INVALID_ARG, w + ": null pointer");
   if (!aligned(Wcodes, 16) || !aligned(y, 16) || !aligned(r, 16) || !aligned(workspace, 256))
     return fail(OQ_ERR_INVALID_ARG, w + ": misaligned pointer (workspace needs 256 bytes)");
@@ -654,13 +671,14 @@ static oq_status fused_checks(const oq_layer* L, const void* x, int32_t x_dtype,
 }
 
 oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                          const float* r, float* y, void* workspace, size_t workspace_bytes, void* stream) {
-  oq_status st = fused_checks(L, x, x_dtype, T, Wcodes, r, y, workspace, "oq_linear_fused");
+                          const float* r, void* y, int32_t y_dtype, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  oq_status st = fused_checks(L, x, x_dtype, T, Wcodes, r, y, y_dtype, workspace, "oq_linear_fused");
   if (st != OQ_OK || T == 0) return st;
-  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, y, stream);
+  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, static_cast<float*>(y), stream);
   if (workspace_bytes < min_workspace(L, T)) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
-  return fused_device(L, x, x_dtype, T, Wcodes, r, y, static_cast<unsigned char*>(workspace), workspace_bytes,
-                      stream, nullptr);
+  return fused_device(L, x, x_dtype, T, Wcodes, r, y, y_dtype == OQ_DTYPE_BF16,
+                      static_cast<unsigned char*>(workspace), workspace_bytes, stream, nullptr);
 }
 
 oq_status oq_poll_error(const oq_layer* L) {
@@ -692,13 +710,15 @@ size_t fused_min_workspace(const oq_layer* L, int64_t T) { return min_workspace(
 size_t fused_w16_workspace(const oq_layer* L, int64_t T) { return full_workspace(L, T, min_workspace(L, T)); }
 bool fused_decodes_weights(const oq_layer* L, int32_t x_dtype, int64_t T) { return fused_w16_route(L, x_dtype, T); }
 oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                           const float* r, const float* y, const void* workspace, const char* who) {
-  return fused_checks(L, x, x_dtype, T, Wcodes, r, y, workspace, who);
+                           const float* r, const void* y, int32_t y_dtype, const void* workspace, const char* who) {
+  return fused_checks(L, x, x_dtype, T, Wcodes, r, y, y_dtype, workspace, who);
 }
 oq_status fused_run(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                    const float* r, float* y, void* ws, size_t ws_bytes, void* stream, const uint16_t* w16_ready) {
-  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, y, stream);
-  return fused_device(L, x, x_dtype, T, Wcodes, r, y, static_cast<unsigned char*>(ws), ws_bytes, stream, w16_ready);
+                    const float* r, void* y, bool y_bf16, void* ws, size_t ws_bytes, void* stream,
+                    const uint16_t* w16_ready) {
+  if (L->int4_only) return int4_linear(L, x, x_dtype, T, Wcodes, r, static_cast<float*>(y), stream);
+  return fused_device(L, x, x_dtype, T, Wcodes, r, y, y_bf16, static_cast<unsigned char*>(ws), ws_bytes, stream,
+                      w16_ready);
 }
 oq_status decode_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* w16, void* stream) {
   return levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);

@@ -32,6 +32,7 @@
 #include <cstring>
 
 #include "oq_internal.h"
+#include "oq_epilogue.cuh"
 #include "oq_ptx.cuh"
 #include "oq_rqtc_dev.cuh"
 #include "oq_tmap.cuh"
@@ -61,6 +62,7 @@ struct FusedParams {
   CUtensorMap y_map;   // fp32 y [M, N], boxes of 32 x 32
   const float* b_scale;
   float out_scale;
+  bool y_bf16;         // y is bf16 (else fp32)
   int64_t M;
   int N, K, n_tiles, nkb;
   int64_t tiles;
@@ -307,17 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
         unsigned char* buf = ebuf + (cc & 1) * (32 * 32 * 4);
         if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
-        const uint32_t rb = smem_u32(buf) + (uint32_t)lane * 128u;
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const float4 rr = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + k4);
-          uint4 o;
-          o.x = __float_as_uint(__uint_as_float(v[4 * k4 + 0]) * srow * rr.x);
-          o.y = __float_as_uint(__uint_as_float(v[4 * k4 + 1]) * srow * rr.y);
-          o.z = __float_as_uint(__uint_as_float(v[4 * k4 + 2]) * srow * rr.z);
-          o.w = __float_as_uint(__uint_as_float(v[4 * k4 + 3]) * srow * rr.w);
-          st_shared_v4(rb + ((uint32_t)(k4 ^ (lane & 7)) << 4), o);
-        }
+        stage_y_chunk(v, srow, p.b_scale + nb, smem_u32(buf), lane, p.y_bf16);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -408,6 +400,7 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* str
   std::memset(&kp, 0, sizeof(kp));
   kp.b_scale = g.b_scale;
   kp.out_scale = g.out_scale;
+  kp.y_bf16 = g.y_bf16;
   kp.M = g.M;
   kp.N = g.N;
   kp.K = g.K;
@@ -433,26 +426,33 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* str
   const int A = a.h / 32;
   kp.nw = a.d / a.h;
   kp.stage_bytes = (a.d * 2 + 127) & ~127;
-  // as many teams as the warp budget and shared memory allow
+  auto kern = A == 32 ? fused_kernel<32> : fused_kernel<16>;
+  // as many teams as the warp budget, shared memory and the SM's registers
+  // allow (the occupancy query says whether one CTA of that shape fits)
   int teams = (MAX_WARPS - GEMM_WARPS) / kp.nw;
-  while (teams > 1 && smem_bytes(A, kp.nb, kp.nw, teams, kp.stage_bytes, nullptr) > 227 * 1024) --teams;
+  size_t smem = 0;
+  for (; teams >= 1; --teams) {
+    smem = smem_bytes(A, kp.nb, kp.nw, teams, kp.stage_bytes, &kp.prod_off);
+    if (smem > 227 * 1024) continue;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) continue;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, (GEMM_WARPS + teams * kp.nw) * 32, smem) ==
+            cudaSuccess &&
+        per_sm >= 1)
+      break;
+  }
+  cudaGetLastError();   // a refused configuration above is not an error of this call
+  if (teams < 1) return OQ_ERR_UNSUPPORTED;
   kp.teams = teams;
-  const size_t smem = smem_bytes(A, kp.nb, kp.nw, teams, kp.stage_bytes, &kp.prod_off);
-  if (smem > 227 * 1024) return OQ_ERR_UNSUPPORTED;
 
   oq_status st = encode_operand_map(&kp.a_map, a.out16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.M, g.K, RM,
                                     "the fp16 A operand");
   if (st == OQ_OK)
     st = encode_operand_map(&kp.b_map, g.b_f16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.N, g.K, RN, "the fp16 B operand");
-  if (st == OQ_OK) st = encode_y_map(&kp.y_map, g.y, g.M, g.N);
+  if (st == OQ_OK) st = encode_y_map(&kp.y_map, g.y, g.M, g.N, g.y_bf16);
   if (st != OQ_OK) return st;
 
-  auto kern = A == 32 ? fused_kernel<32> : fused_kernel<16>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) {
-    set_error(std::string("cudaFuncSetAttribute(fused): ") + cudaGetErrorString(e));
-    return OQ_ERR_CUDA;
-  }
+  cudaError_t e = cudaSuccess;
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -467,10 +467,17 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* str
     set_error(std::string("clear fused flags: ") + cudaGetErrorString(e));
     return OQ_ERR_CUDA;
   }
-  kern<<<(unsigned)grid, (unsigned)((GEMM_WARPS + teams * kp.nw) * 32), smem, s>>>(kp);
+  const unsigned threads = (unsigned)((GEMM_WARPS + teams * kp.nw) * 32);
+  kern<<<(unsigned)grid, threads, smem, s>>>(kp);
   e = cudaGetLastError();
   if (e != cudaSuccess) {
-    set_error(std::string("fused kernel launch: ") + cudaGetErrorString(e));
+    cudaFuncAttributes fa;
+    std::memset(&fa, 0, sizeof(fa));
+    cudaFuncGetAttributes(&fa, kern);
+    set_error(std::string("fused kernel launch: ") + cudaGetErrorString(e) + " (threads " + std::to_string(threads) +
+              ", dynamic shared memory " + std::to_string(smem) + ", registers " + std::to_string(fa.numRegs) +
+              ", max threads " + std::to_string(fa.maxThreadsPerBlock) + ", static shared " +
+              std::to_string(fa.sharedSizeBytes) + ")");
     return OQ_ERR_CUDA;
   }
   return OQ_OK;

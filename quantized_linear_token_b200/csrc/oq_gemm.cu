@@ -23,6 +23,7 @@
 
 #include "oq_decode.cuh"
 #include "oq_internal.h"
+#include "oq_epilogue.cuh"
 #include "oq_ptx.cuh"
 
 namespace oq {
@@ -41,7 +42,8 @@ struct GemmKParams {
   const float* a_scale;
   const float* b_scale;
   float out_scale;
-  float* y;
+  bool y_bf16;         // y is bf16 (else fp32)
+  void* y;             // [M, N] fp32, or bf16 with y_bf16
   int64_t M;
   int N, K, a_wpr, b_wpr;
   int n_tiles, nkb;
@@ -201,8 +203,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
         tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * BN + cc * 32), v);
         tmem_wait_ld();
         const int nb = n0 + cc * 32;
-        if (row < p.M && nb < p.N) {
-          float* dst = p.y + row * p.N + nb;
+        if (row < p.M && nb < p.N && !p.y_bf16) {
+          float* dst = static_cast<float*>(p.y) + row * p.N + nb;
           if (nb + 32 <= p.N) {
 #pragma unroll
             for (int k4 = 0; k4 < 8; ++k4) {
@@ -218,6 +220,31 @@ __global__ void __launch_bounds__(NTHREADS, 1) gemm_kernel(const __grid_constant
 #pragma unroll
             for (int k1 = 0; k1 < 32; ++k1)
               if (nb + k1 < p.N) dst[k1] = __uint_as_float(v[k1]) * srow * __ldg(p.b_scale + nb + k1);
+          }
+        } else if (row < p.M && nb < p.N) {
+          // bf16 y: pairs rounded to nearest even; 32 columns are 64
+          // contiguous, 16-byte aligned bytes (N % 16 == 0)
+          uint16_t* dst = static_cast<uint16_t*>(p.y) + row * p.N + nb;
+          if (nb + 32 <= p.N) {
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8) {
+              const float4 r0 = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + 2 * k8);
+              const float4 r1 = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + 2 * k8 + 1);
+              const uint32_t* w = v + 8 * k8;
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(w[0]) * srow * r0.x, __uint_as_float(w[1]) * srow * r0.y);
+              o.y = pack_bf16x2(__uint_as_float(w[2]) * srow * r0.z, __uint_as_float(w[3]) * srow * r0.w);
+              o.z = pack_bf16x2(__uint_as_float(w[4]) * srow * r1.x, __uint_as_float(w[5]) * srow * r1.y);
+              o.w = pack_bf16x2(__uint_as_float(w[6]) * srow * r1.z, __uint_as_float(w[7]) * srow * r1.w);
+              reinterpret_cast<uint4*>(dst)[k8] = o;
+            }
+          } else {
+#pragma unroll
+            for (int k1 = 0; k1 < 32; ++k1)
+              if (nb + k1 < p.N) {
+                const __nv_bfloat16 b = __float2bfloat16_rn(__uint_as_float(v[k1]) * srow * __ldg(p.b_scale + nb + k1));
+                dst[k1] = *reinterpret_cast<const uint16_t*>(&b);
+              }
           }
         }
       }
@@ -356,6 +383,7 @@ oq_status gemm_launch(const GemmArgs& g, void* stream) {
   kp.a_scale = g.a_scale;
   kp.b_scale = g.b_scale;
   kp.out_scale = g.out_scale;
+  kp.y_bf16 = g.y_bf16;
   kp.y = g.y;
   kp.M = g.M;
   kp.N = g.N;

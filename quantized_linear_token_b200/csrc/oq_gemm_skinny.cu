@@ -416,7 +416,8 @@ oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream) {
   kp.a_scale = g.a_scale;
   kp.b_scale = g.b_scale;
   kp.out_scale = g.out_scale;
-  kp.y = g.y;
+  if (g.y_bf16) return OQ_ERR_UNSUPPORTED;   // the splits add in fp32 in y itself
+  kp.y = static_cast<float*>(g.y);
   kp.counters = counters;
   kp.err = g.err;
   kp.T = (int)g.M;

@@ -24,6 +24,7 @@
 #include <cstring>
 
 #include "oq_internal.h"
+#include "oq_epilogue.cuh"
 #include "oq_ptx.cuh"
 #include "oq_tmap.cuh"
 
@@ -53,6 +54,7 @@ struct W16Params {
   const float* a_scale;
   const float* b_scale;
   float out_scale;
+  bool y_bf16;         // y is bf16 (else fp32)
   int64_t M;
   int N, K, n_tiles, nkb;
   int64_t tiles;
@@ -160,17 +162,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
         // the store that last read this buffer (two chunks ago) must be done
         if (lane == 0) bulk_wait_read<1>();
         __syncwarp();
-        const uint32_t rb = smem_u32(buf) + (uint32_t)lane * 128u;
-#pragma unroll
-        for (int k4 = 0; k4 < 8; ++k4) {
-          const float4 rr = __ldg(reinterpret_cast<const float4*>(p.b_scale + nb) + k4);
-          uint4 o;
-          o.x = __float_as_uint(__uint_as_float(v[4 * k4 + 0]) * srow * rr.x);
-          o.y = __float_as_uint(__uint_as_float(v[4 * k4 + 1]) * srow * rr.y);
-          o.z = __float_as_uint(__uint_as_float(v[4 * k4 + 2]) * srow * rr.z);
-          o.w = __float_as_uint(__uint_as_float(v[4 * k4 + 3]) * srow * rr.w);
-          st_shared_v4(rb + ((uint32_t)(k4 ^ (lane & 7)) << 4), o);
-        }
+        stage_y_chunk(v, srow, p.b_scale + nb, smem_u32(buf), lane, p.y_bf16);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -251,6 +243,7 @@ oq_status gemm_w16_launch(const GemmArgs& g, void* stream) {
   kp.a_scale = g.a_scale;
   kp.b_scale = g.b_scale;
   kp.out_scale = g.out_scale;
+  kp.y_bf16 = g.y_bf16;
   kp.M = g.M;
   kp.N = g.N;
   kp.K = g.K;
@@ -260,7 +253,7 @@ oq_status gemm_w16_launch(const GemmArgs& g, void* stream) {
   if (st == OQ_OK)
     st = encode_operand_map(&kp.b_map, g.b_f16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.N, g.K, RN,
                             "the fp16 B operand");
-  if (st == OQ_OK) st = encode_y_map(&kp.y_map, g.y, g.M, g.N);
+  if (st == OQ_OK) st = encode_y_map(&kp.y_map, g.y, g.M, g.N, g.y_bf16);
   if (st != OQ_OK) return st;
 
   const size_t smem = 1024 + (size_t)OS * STAGE_BYTES + EPI_BYTES + 8 * (2 * OS + 4) + 16;

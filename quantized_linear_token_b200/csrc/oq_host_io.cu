@@ -123,11 +123,12 @@ size_t oq_linear_fused_host_workspace_size(const oq_layer* L, int32_t x_dtype, i
 }
 
 oq_status oq_linear_fused_host(const oq_layer* layer, const void* x_host, int32_t x_dtype, int64_t T,
-                               const uint32_t* Wcodes, const float* r, float* y_host, void* workspace,
+                               const uint32_t* Wcodes, const float* r, void* y_host, int32_t y_dtype, void* workspace,
                                size_t workspace_bytes, void* stream) {
   // the copy streams and events are a cache inside the layer
   oq_layer* L = const_cast<oq_layer*>(layer);
-  oq_status st = fused_check_args(L, x_host, x_dtype, T, Wcodes, r, y_host, workspace, "oq_linear_fused_host");
+  oq_status st =
+      fused_check_args(L, x_host, x_dtype, T, Wcodes, r, y_host, y_dtype, workspace, "oq_linear_fused_host");
   if (st != OQ_OK || T == 0) return st;
   if (L->int4_only) {
     set_error("oq_linear_fused_host: not available on an INT4 weight-only layer");
@@ -147,7 +148,8 @@ oq_status oq_linear_fused_host(const oq_layer* layer, const void* x_host, int32_
   // ev[0]: start (caller's stream); ev[1 + k]: x slot k filled; ev[3 + k]:
   // chunk in slot k computed; ev[5 + k]: y slot k copied out; ev[7]: done
   unsigned char* ws = static_cast<unsigned char*>(workspace);
-  const size_t xrow = x_row_bytes(L, x_dtype), yrow = (size_t)L->d_out * 4;
+  const bool y_bf16 = y_dtype == OQ_DTYPE_BF16;
+  const size_t xrow = x_row_bytes(L, x_dtype), yrow = (size_t)L->d_out * (y_bf16 ? 2 : 4);
   const unsigned char* xh = static_cast<const unsigned char*>(x_host);
   unsigned char* yh = reinterpret_cast<unsigned char*>(y_host);
 
@@ -166,7 +168,7 @@ oq_status oq_linear_fused_host(const oq_layer* layer, const void* x_host, int32_
     const int k = (int)(i & 1);
     const int64_t t0 = i * lay.chunk, tc = std::min(lay.chunk, T - t0);
     void* xd = ws + lay.x_off[k];
-    float* yd = reinterpret_cast<float*>(ws + lay.y_off[k]);
+    void* yd = ws + lay.y_off[k];
     // x slot k is free once chunk i - 2 has been computed
     if (i >= 2 && (st = cu(cudaStreamWaitEvent(s_in, ev[3 + k], 0), "wait slot")) != OQ_OK) return st;
     if ((st = cu(cudaMemcpyAsync(xd, xh + (size_t)t0 * xrow, (size_t)tc * xrow, cudaMemcpyHostToDevice, s_in),
@@ -176,7 +178,7 @@ oq_status oq_linear_fused_host(const oq_layer* layer, const void* x_host, int32_
     // compute once x has arrived and y slot k has been copied out (chunk i - 2)
     if ((st = cu(cudaStreamWaitEvent(comp, ev[1 + k], 0), "wait x")) != OQ_OK) return st;
     if (i >= 2 && (st = cu(cudaStreamWaitEvent(comp, ev[5 + k], 0), "wait y slot")) != OQ_OK) return st;
-    st = fused_run(L, xd, x_dtype, tc, Wcodes, r, yd, ws, lay.fused_bytes, comp, w16);
+    st = fused_run(L, xd, x_dtype, tc, Wcodes, r, yd, y_bf16, ws, lay.fused_bytes, comp, w16);
     if (st != OQ_OK) return st;
     if ((st = cu(cudaEventRecord(ev[3 + k], comp), "record compute")) != OQ_OK) return st;
     if ((st = cu(cudaStreamWaitEvent(s_out, ev[3 + k], 0), "wait compute")) != OQ_OK) return st;

@@ -119,7 +119,8 @@ struct GemmArgs {
   const uint16_t* a_levels_host;  // host copies (register decode tables)
   const uint16_t* b_levels_host;
   float out_scale;           // 1 / (alpha_a alpha_w)
-  float* y;                  // [M, N] fp32
+  void* y;                   // [M, N] fp32, or bf16 with y_bf16
+  bool y_bf16;
   int64_t M;
   int N, K, a_bits, b_bits;
   int* err;
@@ -157,9 +158,10 @@ size_t fused_min_workspace(const oq_layer* L, int64_t T);
 size_t fused_w16_workspace(const oq_layer* L, int64_t T);
 bool fused_decodes_weights(const oq_layer* L, int32_t x_dtype, int64_t T);
 oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                           const float* r, const float* y, const void* workspace, const char* who);
+                           const float* r, const void* y, int32_t y_dtype, const void* workspace, const char* who);
 oq_status fused_run(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
-                    const float* r, float* y, void* ws, size_t ws_bytes, void* stream, const uint16_t* w16_ready);
+                    const float* r, void* y, bool y_bf16, void* ws, size_t ws_bytes, void* stream,
+                    const uint16_t* w16_ready);
 oq_status decode_weight_levels(const oq_layer* L, const uint32_t* Wcodes, uint16_t* w16, void* stream);
 // a one-warp kernel whose bounded wait (limit_ns) runs out (oq_diag.cu)
 oq_status wait_timeout_launch(int* err, uint64_t limit_ns, void* stream);

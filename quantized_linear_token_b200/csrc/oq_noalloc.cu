@@ -88,5 +88,5 @@ extern "C" oq_status oq_linear_fused_static(const oq_layer* layer, const void* x
   void* scratch = nullptr;
   const oq_status st = scratch_address(&scratch);
   if (st != OQ_OK) return st;
-  return oq_linear_fused(layer, x, x_dtype, T, Wcodes, r, y, scratch, need, stream);
+  return oq_linear_fused(layer, x, x_dtype, T, Wcodes, r, y, OQ_DTYPE_F32, scratch, need, stream);
 }

@@ -53,18 +53,20 @@ inline oq_status encode_operand_map(CUtensorMap* map, const void* base, CUtensor
   return OQ_OK;
 }
 
-// fp32 y [M, N] written by the contraction epilogues in 128B-swizzled boxes
-// of 32 x 32 (TMA stores clip rows past M)
-inline oq_status encode_y_map(CUtensorMap* map, float* y, int64_t M, int N) {
+// y [M, N] written by the contraction epilogues in boxes of 32 x 32: fp32 in
+// the 128-byte swizzle (128-byte box rows), bf16 in the 64-byte swizzle
+// (64-byte box rows); TMA stores clip rows past M
+inline oq_status encode_y_map(CUtensorMap* map, void* y, int64_t M, int N, bool bf16 = false) {
   EncodeTiledFn fn = nullptr;
   const oq_status st = tmap_encode_fn(&fn);
   if (st != OQ_OK) return st;
   const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-  const cuuint64_t strides[1] = {(cuuint64_t)N * 4};
+  const cuuint64_t strides[1] = {(cuuint64_t)N * (bf16 ? 2 : 4)};
   const cuuint32_t box[2] = {32, 32};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+  const CUresult r = fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, y, dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_error("cuTensorMapEncodeTiled failed for y (code " + std::to_string((int)r) + ")");

@@ -98,10 +98,10 @@ def test_argument_checks(lib):
     assert lib.oq_layer_create(256, 256, 0, 4, 4, 64, ctypes.byref(h)) == 1     # unknown flag
     assert lib.oq_layer_create(256, 256, 0, 4, 4, 0, None) == 1
     assert lib.oq_rotate_quantize(None, None, 1, 4, None, None, None) == 1
-    assert lib.oq_linear(None, None, None, 4, None, None, None, None) == 1
+    assert lib.oq_linear(None, None, None, 4, None, None, None, 0, None) == 1
     assert lib.oq_linear_fused_workspace_size(None, 10) == 0
     assert lib.oq_linear_fused_host_workspace_size(None, 0, 10) == 0
-    assert lib.oq_linear_fused_host(None, None, 0, 4, None, None, None, None, 0, None) == 1
+    assert lib.oq_linear_fused_host(None, None, 0, 4, None, None, None, 0, None, 0, None) == 1
     assert lib.oq_rotation_build(0, 0, 0, None, None) == 1
     assert lib.oq_check_wait_timeout(None, 1000, None) == 1
     assert b"" != lib.oq_status_string(2)

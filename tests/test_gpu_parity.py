@@ -504,6 +504,71 @@ def test_prepared_weight_file(env, tmp_path):
     B.oq_poll_error(layer)
 
 
+BF16_Y = [
+    # d_in, d_out, a, w, T: the fused kernel (bf16 x, h = 1024, T >= 1024), the
+    # CTA pair with weights decoded in the contraction, a small batch (which
+    # takes the CTA pair for bf16 y), the one-SM kernel (d_out = 80), and the
+    # packed-code route (fp32 x)
+    (3072, 768, 4, 4, 1300, "bf16"),
+    (2048, 512, 4, 2, 1100, "bf16"),
+    (3072, 512, 4, 4, 300, "bf16"),
+    (640, 512, 3, 3, 100, "bf16"),
+    (192, 80, 3, 3, 129, "bf16"),
+    (256, 256, 4, 4, 70, "f32"),
+]
+
+
+@pytest.mark.parametrize("d_in,d_out,a_bits,w_bits,T,xdt", BF16_Y)
+def test_bf16_output(env, d_in, d_out, a_bits, w_bits, T, xdt):
+    # y written as bf16 (round to nearest even in the epilogue): within the
+    # parity bound of the oracle widened by the output rounding, |dy| <=
+    # 1e-3 * bound + 2^-8 |y|; where the bf16 and fp32 calls take the same
+    # kernel, bit for bit the bf16 rounding of the fp32 y; and the same through
+    # the host-buffer call
+    torch, B = env
+    x_np = W.custom_activations(T, d_in, seed=d_in + 3 * T)
+    if xdt == "f32":
+        x_np = W.bf16_bits_to_f32(x_np)
+    Wm = W.custom_weights(d_out, d_in, seed=d_out + 5)
+    layer = B.oq_layer_create(d_in, d_out, 0, a_bits, w_bits, 0)
+    x_t, x64 = _x_tensor(torch, x_np)
+    Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(Wm).cuda())
+    y32 = B.oq_linear_fused(layer, x_t, Wc, r)
+    y16 = B.oq_linear_fused(layer, x_t, Wc, r, y_dtype=torch.bfloat16)
+    codes, s = B.oq_rotate_quantize(layer, x_t)
+    y16c = B.oq_linear(layer, codes, s, Wc, r, y_dtype=torch.bfloat16)
+    y32c = B.oq_linear(layer, codes, s, Wc, r)
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+    assert y16.dtype == torch.bfloat16 and y16.shape == (T, d_out)
+    same_kernel = T > 256 or d_out % 256 != 0 or xdt == "f32"
+    if same_kernel:
+        assert torch.equal(y16.view(torch.int16), y32.to(torch.bfloat16).view(torch.int16))
+    assert torch.equal(y16c.view(torch.int16), y32c.to(torch.bfloat16).view(torch.int16))
+    # against the oracle on the codes of the route that ran (the packed-code
+    # kernel's codes; on the fp16-level route the fused call's operand)
+    if x_np.dtype == np.uint16 and d_out % 256 == 0:
+        a16, s2 = B.oq_rotate_quantize_levels(layer, x_t)
+        cb_a = O.lloyd_max(d_in, a_bits)
+        lv = (layer.a_scale * np.asarray(cb_a.levels)).astype(np.float16).view(np.uint16)
+        ca = levels_to_codes(a16.cpu().numpy().view(np.uint16), lv, "bf16 y")
+        s_np = s2.cpu().numpy()
+    else:
+        ca = O.unpack_codes(to_numpy_u32(codes), a_bits, d_in)
+        s_np = s.cpu().numpy()
+    cw = O.unpack_codes(to_numpy_u32(Wc), w_bits, d_in)
+    y_or, bound = O.linear_from_codes(ca, s_np.astype(np.float64), cw, r.cpu().numpy().astype(np.float64),
+                                      O.lloyd_max(d_in, a_bits).levels, O.lloyd_max(d_in, w_bits).levels)
+    err = np.abs(y16.float().cpu().numpy().astype(np.float64) - y_or)
+    assert np.all(err <= 1e-3 * bound + 2.0 ** -8 * np.abs(y_or) + 1e-30)
+    # host buffers
+    x_host = x_t.cpu().pin_memory()
+    y_host = torch.empty((T, d_out), dtype=torch.bfloat16).pin_memory()
+    B.oq_linear_fused_host(layer, x_host, Wc, r, y_host)
+    torch.cuda.current_stream().synchronize()
+    assert torch.equal(y_host.view(torch.int16), y16.cpu().view(torch.int16))
+
+
 def test_empty_batch(env):
     torch, B = env
     layer = B.oq_layer_create(256, 256, 0, 4, 4, 0)
