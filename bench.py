@@ -45,7 +45,7 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's token count (profiling)")
     ap.add_argument("--layer", default="", help="layer of the workload by name (default: its first)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--route", choices=["levels", "levels_wdec", "codes"], default="levels",
+    ap.add_argument("--route", choices=["levels", "staged", "levels_wdec", "codes"], default="levels",
                     help="hot-path route of the timed step (the others are reported beside it)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true",
@@ -340,8 +340,21 @@ def run_ours(args):
     #   levels_wdec: oq_rotate_quantize_levels -> oq_linear_levels at any size
     #   codes:       oq_rotate_quantize -> oq_linear (packed codes between them)
     decoded = T >= B.W16_MIN_T and dout % 256 == 0
+    ws_fd = torch.empty((max(B.oq_linear_fused_decoded_workspace_size(layer, T), 1),), dtype=torch.uint8,
+                        device=dev)
+    # the fused call's large-batch route runs one kernel for rotate-quantize
+    # and the contraction where the block size is 1024 or 512 with at most 12
+    # warps per token row (bf16 x, no Rademacher signs)
+    h_blk = d & -d
+    fused_kernel = decoded and ((h_blk == 1024 and d // h_blk <= 8) or (h_blk == 512 and d // h_blk <= 12))
     stages = {
-        "levels": [("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s))]
+        # the stages of oq_linear_fused at this batch size
+        "levels": ([("wlevels", lambda: B.oq_weight_levels(layer, Wc, w16)),
+                    ("fused", lambda: B.oq_linear_fused_decoded(layer, x, w16, r, y, ws_fd))] if decoded else
+                   [("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s)),
+                    ("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]),
+        # the same route with rotate-quantize and the contraction as two kernels
+        "staged": [("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s))]
         + ([("wlevels", lambda: B.oq_weight_levels(layer, Wc, w16)),
             ("gemm", lambda: B.oq_linear_decoded(layer, a16, s, w16, r, y))] if decoded else
            [("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]),
@@ -386,7 +399,7 @@ def run_ours(args):
 
     K = args.steps
     route = args.route
-    others = [o for o in ("levels", "levels_wdec", "codes") if o != route]
+    others = [o for o in ("levels", "staged", "levels_wdec", "codes") if o != route]
     # the step: one oq_linear_fused call (the whole hot path, x -> y; from
     # W16_MIN_T tokens on it also decodes the weight levels once)
     for _ in range(args.warmup):
@@ -442,6 +455,30 @@ def run_ours(args):
     e2e_ms = max_over_ranks(sum(t_e2e), dev)
     B.oq_poll_error(layer)
 
+    # the same step and the same end-to-end call with bf16 y (half the output
+    # bytes: the epilogue's write and the copy out)
+    y_b = torch.empty((T, dout), dtype=torch.bfloat16, device=dev)
+    y_host_b = torch.empty((T, dout), dtype=torch.bfloat16).pin_memory()
+    evb = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for _ in range(max(2, args.warmup // 2)):
+        flush.zero_()
+        B.oq_linear_fused(layer, x, Wc, r, y_b, ws)
+        B.oq_linear_fused_host(layer, x_host, Wc, r, y_host_b, ws_host)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()
+        evb[i][0].record(stream)
+        B.oq_linear_fused(layer, x, Wc, r, y_b, ws)
+        evb[i][1].record(stream)
+    for i in range(K):
+        evb[i][2].record(stream)
+        B.oq_linear_fused_host(layer, x_host, Wc, r, y_host_b, ws_host)
+        evb[i][3].record(stream)
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+    bf16_ms = max_over_ranks(sum(evb[i][0].elapsed_time(evb[i][1]) for i in range(K)), dev)
+    bf16_e2e_ms = max_over_ranks(sum(evb[i][2].elapsed_time(evb[i][3]) for i in range(K)), dev)
+
     peaks = load_peaks()
     flops = 2.0 * T * d * dout
 
@@ -454,16 +491,25 @@ def run_ours(args):
     # writes: bf16 x read, packed codes and the norm written
     rq_alg_bytes = T * (2 * d + d * lay.a_bits / 8 + 4)
 
-    def route_decoded(rt):
-        return rt == "levels" and decoded
+    def contraction_key(pr):
+        return "fused" if "fused" in pr else "gemm"
 
+    # the stand-alone rotate-quantize kernel: in this route, or else in the
+    # staged form of it (the fused kernel runs rotate-quantize inside the
+    # contraction, so it has no time of its own)
+    rq_src = per if "rq" in per else other_per.get("staged", other_per.get("levels_wdec"))
+    rq_route = route if "rq" in per else "staged"
     wl_bytes = dout * d * (lay.w_bits / 8 + 2)     # weight codes read + fp16 levels written
-    mm_ms = statistics.mean(per["gemm"])
-    rq_ms = statistics.mean(per["rq"])
-    rq_bytes = rq_bytes_per_launch(route)
+    ckey = contraction_key(per)
+    mm_ms = statistics.mean(per[ckey])
+    rq_ms = statistics.mean(rq_src["rq"])
+    rq_bytes = rq_bytes_per_launch(rq_route)
     gemm_tf = flops / (mm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
     gemm_desc = {
+        "fused": ("fused layer kernel: rotate-quantize warps (norm, gather, tensor-core block FWHT, Lloyd-Max "
+                  "codes as fp16 levels) feeding the tcgen05 CTA-pair contraction of the decoded weights, "
+                  "fp32 TMEM accumulate", "fused"),
         "decoded": ("codebook GEMM on fp16 levels of both operands, both by TMA "
                     "(tcgen05 CTA pair, fp32 TMEM accumulate)", "gemm_decoded"),
         "levels_wdec": ("codebook GEMM, fp16 A operand by TMA, weight codes decoded to fp16 in shared memory "
@@ -471,19 +517,37 @@ def run_ours(args):
         "codes": ("codebook GEMM, both operands' codes decoded to fp16 in shared memory "
                   "(tcgen05 CTA pair, fp32 TMEM accumulate)", None),
     }
-    gkey = "decoded" if route_decoded(route) else ("codes" if route == "codes" else "levels_wdec")
+    gkey = ("fused" if ckey == "fused" else "decoded" if (decoded and route in ("levels", "staged")) else
+            "codes" if route == "codes" else "levels_wdec")
     rq_desc = {
         "levels": "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes) writing the codes' fp16 levels",
         "codes": "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes, pack)",
     }
     steps_desc = {
-        "levels": ("oq_rotate_quantize_levels + oq_weight_levels + oq_linear_decoded" if decoded else
+        "levels": ("oq_weight_levels + oq_linear_fused_decoded" if decoded else
                    "oq_rotate_quantize_levels + oq_linear_levels")
         + " (the stages of oq_linear_fused at this batch size; weights prepared once, offline)",
+        "staged": ("oq_rotate_quantize_levels + oq_weight_levels + oq_linear_decoded" if decoded else
+                   "oq_rotate_quantize_levels + oq_linear_levels")
+        + " (the same route, rotate-quantize and the contraction as separate kernels)",
         "levels_wdec": "oq_rotate_quantize_levels + oq_linear_levels (weight codes decoded inside the contraction)",
         "codes": "oq_rotate_quantize + oq_linear (weights prepared once, offline)",
     }
+
+    def route_summary(o):
+        pr = other_per[o]
+        c = contraction_key(pr)
+        row = {"route": o, "step": steps_desc[o], "value": whole_job_rate(world, T, K, other_ms[o]), "unit": UNIT,
+               "ms_per_step": other_ms[o] / K, "contraction": c,
+               "gemm_tflops": flops / (statistics.mean(pr[c]) * 1e-3) / 1e12, "gemm_ms": statistics.mean(pr[c])}
+        if "rq" in pr:
+            row.update({"rq_gbs": rq_alg_bytes / (statistics.mean(pr["rq"]) * 1e-3) / 1e9,
+                        "rq_route_gbs": rq_bytes_per_launch(o) / (statistics.mean(pr["rq"]) * 1e-3) / 1e9,
+                        "rq_ms": statistics.mean(pr["rq"])})
+        return row
+
     full_size = T == wl.tokens
+    launches_per_step = (2 if fused_kernel else 3) if decoded else 2
     out = {
         "metric": METRIC,
         "value": whole_job_rate(world, T, K, total_ms),
@@ -500,7 +564,7 @@ def run_ours(args):
         "config": {
             **workload_config(args, wl, lay, T, world),
             "l2": "flushed (256 MiB write) before every step, outside the timed events",
-            "step": "one oq_linear_fused call (x -> y: " + steps_desc[route].split(" (")[0] + ")",
+            "step": "one oq_linear_fused call (x -> y: " + steps_desc["levels"].split(" (")[0] + ")",
         },
         "roofline": {
             "kernel": gemm_desc[gkey][0],
@@ -512,18 +576,19 @@ def run_ours(args):
             "flops_per_launch": flops, "ms_per_launch": mm_ms,
         },
         "roofline_rotate_quantize": {
-            "kernel": rq_desc["codes" if route == "codes" else "levels"],
+            "kernel": rq_desc["codes" if rq_route == "codes" else "levels"]
+            + ("" if rq_route == route else " (the stand-alone kernel of the staged route)"),
             "bound": "hbm", "achieved": rq_alg_bytes / (rq_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": rq_alg_bytes / (rq_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
             "bytes_per_launch": rq_alg_bytes,
             "bytes_rule": "algorithmic: 2 d (bf16 x) + d a_bits / 8 (packed codes) + 4 (norm) per token",
-            "traffic": measured_traffic("rq_levels" if route != "codes" else "rq_codes") if full_size else None,
+            "traffic": measured_traffic("rq_levels" if rq_route != "codes" else "rq_codes") if full_size else None,
             "peak_source": f"{peaks['source']} HBM copy bandwidth",
             "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum per launch, profiles/traffic.json",
             "ms_per_launch": rq_ms,
             "route_bytes_per_launch": rq_bytes, "route_achieved": rq_gbs, "route_frac": rq_gbs / peaks["hbm_gbs"],
             "route_bytes_rule": ("the bytes this route's kernel moves: its A operand is written as fp16 levels, "
-                                 "2 d bytes per token" if route != "codes" else "same as algorithmic"),
+                                 "2 d bytes per token" if rq_route != "codes" else "same as algorithmic"),
         },
         **({"roofline_weight_levels": {
             "kernel": "weight codes -> fp16 levels (once per call)",
@@ -535,19 +600,18 @@ def run_ours(args):
         }} if "wlevels" in per else {}),
         "stages": {"value": whole_job_rate(world, T, K, stage_ms), "unit": UNIT, "ms_per_step": stage_ms / K,
                    "step": steps_desc[route] + "; separate calls on one stream, one event per kernel"},
-        "other_routes": [{"route": o, "step": steps_desc[o],
-                          "value": whole_job_rate(world, T, K, other_ms[o]), "unit": UNIT,
-                          "ms_per_step": other_ms[o] / K,
-                          "gemm_tflops": flops / (statistics.mean(other_per[o]["gemm"]) * 1e-3) / 1e12,
-                          "gemm_ms": statistics.mean(other_per[o]["gemm"]),
-                          "rq_gbs": rq_alg_bytes / (statistics.mean(other_per[o]["rq"]) * 1e-3) / 1e9,
-                          "rq_route_gbs": rq_bytes_per_launch(o) / (statistics.mean(other_per[o]["rq"]) * 1e-3) / 1e9,
-                          "rq_ms": statistics.mean(other_per[o]["rq"])} for o in others],
+        "other_routes": [route_summary(o) for o in others],
         "e2e": {"value": whole_job_rate(world, T, K, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size()),
                 "path": "oq_linear_fused_host: pinned host x -> device, fused call, y -> pinned host, overlapped in chunks of 1024 tokens"},
-        "gpu_launches": len(stages[route]) * K,
+        "bf16_y": {"value": whole_job_rate(world, T, K, bf16_ms), "unit": UNIT, "ms_per_step": bf16_ms / K,
+                   "step": "one oq_linear_fused call writing bf16 y",
+                   "e2e": {"value": whole_job_rate(world, T, K, bf16_e2e_ms), "unit": UNIT,
+                           "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                           "d2h_bytes_per_step": int(y_b.numel() * y_b.element_size()),
+                           "path": "oq_linear_fused_host with bf16 y_host"}},
+        "gpu_launches": launches_per_step * K,
         "wall_s_timed_region": wall,
         "clocks": clk,
     }
@@ -658,6 +722,10 @@ def run_sweep(args):
             else:
                 stages += [("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]
             runs = {"step": [("step", lambda: B.oq_linear_fused(layer, x, Wc, r, y, ws))], "stages": stages}
+            if decoded:
+                ws_fd = torch.empty((max(B.oq_linear_fused_decoded_workspace_size(layer, T), 1),),
+                                    dtype=torch.uint8, device=dev)
+                runs["fused"] = [("fused", lambda: B.oq_linear_fused_decoded(layer, x, w16, r, y, ws_fd))]
             times = {}
             for name, st in runs.items():
                 for _ in range(warm):
@@ -678,6 +746,9 @@ def run_sweep(args):
             B.oq_poll_error(layer)
             flops = 2.0 * T * d * dout
             rq_alg = T * (2 * d + d * lay.a_bits / 8 + 4)
+            # the step's dominant kernel: the fused kernel where the step runs
+            # one, else the contraction
+            ck = "fused" if "fused" in times else "gemm"
             line = {
                 "metric": METRIC, "sweep_point": True, "value": T / (times["step"] * 1e-3), "unit": UNIT,
                 "n_gpus": 1, "steps": K, "warmup": warm, "ms_per_step": times["step"],
@@ -688,10 +759,14 @@ def run_sweep(args):
                            "l2": "flushed (256 MiB write) before every step, outside the timed events",
                            "contraction": "decoded weights, both operands by TMA" if decoded else
                            ("small-batch split-K kernel" if T <= 256 else "CTA pair, weights decoded in the GEMM")},
-                "roofline": {"bound": "tensor", "achieved": flops / (times["gemm"] * 1e-3) / 1e12,
+                "roofline": {"kernel": "fused rotate-quantize + contraction" if ck == "fused" else "contraction",
+                             "bound": "tensor", "achieved": flops / (times[ck] * 1e-3) / 1e12,
                              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                             "frac": flops / (times["gemm"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
-                             "traffic": None, "ms_per_launch": times["gemm"]},
+                             "frac": flops / (times[ck] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                             "traffic": None, "ms_per_launch": times[ck]},
+                "contraction_alone": {"achieved": flops / (times["gemm"] * 1e-3) / 1e12,
+                                      "frac": flops / (times["gemm"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                      "ms_per_launch": times["gemm"]},
                 "roofline_rotate_quantize": {"bound": "hbm", "achieved": rq_alg / (times["rq"] * 1e-3) / 1e9,
                                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
                                              "frac": rq_alg / (times["rq"] * 1e-3) / 1e9 / peaks["hbm_gbs"],

@@ -324,6 +324,34 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  * (different streams or host threads).  With bf16 y those batches take the
  * CTA-pair kernel instead (the splits add in fp32 in y itself).
  */
+/*
+ * oq_linear_fused_decoded -- oq_linear_fused with the weights' fp16 levels
+ * already decoded (w16 from oq_weight_levels, kept by the caller across
+ * calls or decoded just before): the large-batch route of oq_linear_fused
+ * without its first step.  Where the block size is 1024 or 512 (at most 12
+ * warps per token row) one kernel rotates, quantizes and contracts: its
+ * rotate-quantize warps claim groups of 4 token rows from a queue, write
+ * their fp16 levels and norms to the workspace and publish each group with a
+ * flag, while its contraction warps load a tile's rows as soon as their
+ * groups are published (gecl notes Method 2: the codes of R x meet the
+ * pre-rotated weight codes in one pass).  Elsewhere the rotate-quantize
+ * kernel and oq_linear_decoded's kernel run in turn.  Either way y is that of
+ * oq_rotate_quantize_levels + oq_linear_decoded, bit for bit.
+ *   x          device [T, d_in] bf16 (else OQ_ERR_UNSUPPORTED).
+ *   w16        device [d_out, d_in] fp16 levels, 16-byte aligned.
+ *   r          device [d_out] fp32, 16-byte aligned.
+ *   y          device [T, d_out], fp32 or bf16 as y_dtype says.
+ *   workspace  device scratch of oq_linear_fused_decoded_workspace_size(layer,
+ *              T) bytes (0 when the call is not available for the layer),
+ *              256-byte aligned; reusable between calls on one stream.
+ * Needs d_out % 256 == 0.  Calls that share a workspace must not overlap on
+ * the GPU.  Errors: as oq_linear_fused.
+ */
+size_t oq_linear_fused_decoded_workspace_size(const oq_layer* layer, int64_t T);
+oq_status oq_linear_fused_decoded(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
+                                  const uint16_t* w16, const float* r, void* y, int32_t y_dtype, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
 oq_status oq_rotate_quantize_levels(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
                                     uint16_t* a16, float* s, void* stream);
 oq_status oq_linear_levels(const oq_layer* layer, const uint16_t* a16, const float* s, int64_t T,

@@ -32,7 +32,8 @@ EXPORTS = (
     "oq_codebook_build", "oq_rotation_build", "oq_layer_create", "oq_layer_destroy", "oq_layer_get_info", "oq_layer_get_perm",
     "oq_rotate_quantize", "oq_weight_prepare", "oq_weight_save", "oq_weight_load", "oq_linear",
     "oq_linear_fused_workspace_size",
-    "oq_linear_fused", "oq_rotate_quantize_levels", "oq_linear_levels", "oq_weight_levels", "oq_linear_decoded",
+    "oq_linear_fused", "oq_linear_fused_decoded_workspace_size", "oq_linear_fused_decoded",
+    "oq_rotate_quantize_levels", "oq_linear_levels", "oq_weight_levels", "oq_linear_decoded",
     "oq_linear_fused_static", "oq_linear_fused_host_workspace_size", "oq_linear_fused_host",
     "oq_poll_error", "oq_check_wait_timeout", "oq_last_error", "oq_status_string",
 )
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH):
         "oq_linear_fused_host_workspace_size": (ctypes.c_size_t, [vp, i32, i64]),
         "oq_linear_fused_host": (i32, [vp, vp, i32, i64, vp, vp, vp, i32, vp, ctypes.c_size_t, vp]),
         "oq_linear_decoded": (i32, [vp, vp, vp, i64, vp, vp, vp, i32, vp]),
+        "oq_linear_fused_decoded_workspace_size": (sz, [vp, i64]),
+        "oq_linear_fused_decoded": (i32, [vp, vp, i32, i64, vp, vp, vp, i32, vp, sz, vp]),
         "oq_linear_fused_static": (i32, [vp, vp, i32, i64, vp, vp, vp, vp]),
         "oq_weight_save": (i32, [vp, vp, vp, ctypes.c_char_p]),
         "oq_weight_load": (i32, [vp, ctypes.c_char_p, vp, vp]),
@@ -315,6 +318,27 @@ def oq_linear_decoded(layer: Layer, a16, s, w16, r, y=None, y_dtype=None):
     y, ycode = _y_out(y, T, layer.d_out, y_dtype, a16.device)
     _check(load_library().oq_linear_decoded(layer.handle, _dev(a16, "a16"), _dev(s, "s"), T, _dev(w16, "w16"),
                                             _dev(r, "r"), _dev(y, "y"), ycode, _stream(a16)), "oq_linear_decoded")
+    return y
+
+
+def oq_linear_fused_decoded_workspace_size(layer: Layer, T: int) -> int:
+    return int(load_library().oq_linear_fused_decoded_workspace_size(layer.handle, T))
+
+
+def oq_linear_fused_decoded(layer: Layer, x, w16, r, y=None, workspace=None, y_dtype=None):
+    """x [T, d_in] bf16 and the weights' fp16 levels w16 -> y [T, d_out]: the
+    fused call's large-batch route after its weight decode (one kernel
+    rotating, quantizing and contracting where the block size allows)."""
+    torch = _torch()
+    T = x.shape[0]
+    y, ycode = _y_out(y, T, layer.d_out, y_dtype, x.device)
+    if workspace is None:
+        workspace = torch.empty((max(oq_linear_fused_decoded_workspace_size(layer, T), 1),), dtype=torch.uint8,
+                                device=x.device)
+    _check(load_library().oq_linear_fused_decoded(layer.handle, _dev(x, "x"), _dtype_code(x), T, _dev(w16, "w16"),
+                                                  _dev(r, "r"), _dev(y, "y"), ycode, _dev(workspace, "workspace"),
+                                                  workspace.numel() * workspace.element_size(), _stream(x)),
+           "oq_linear_fused_decoded")
     return y
 
 

@@ -438,10 +438,10 @@ static bool fused_w16_route(const oq_layer* L, int32_t x_dtype, int64_t T) {
 
 static size_t fused_w16_bytes(const oq_layer* L) { return round256((size_t)L->d_out * (size_t)L->d_in * 2); }
 
-// the workspace of the large-batch route: the least workspace, the decoded
-// weights, and the fused kernel's row-group flags
+// the workspace of the large-batch route: the least workspace, the fused
+// kernel's row-group flags, and the decoded weights
 static size_t full_workspace(const oq_layer* L, int64_t T, size_t base) {
-  return round256(base) + fused_w16_bytes(L) + round256(fused_flag_bytes(T));
+  return round256(base) + round256(fused_flag_bytes(T)) + fused_w16_bytes(L);
 }
 
 // the least workspace oq_linear_fused accepts (without the decoded weights)
@@ -450,6 +450,11 @@ static size_t min_workspace(const oq_layer* L, int64_t T) {
   size_t a = fused_codes_bytes(L, T);
   if (L->d_out % 256 == 0) a = std::max(a, fused_f16_bytes(L, T));
   return round256(a) + (size_t)T * 4;
+}
+
+// the workspace of oq_linear_fused_decoded: the least workspace and the flags
+static size_t decoded_workspace(const oq_layer* L, int64_t T) {
+  return round256(min_workspace(L, T)) + round256(fused_flag_bytes(T));
 }
 
 size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
@@ -606,6 +611,25 @@ static oq_status int4_linear(const oq_layer* L, const void* x, int32_t x_dtype, 
   return OQ_OK;
 }
 
+// x -> y with the weights' fp16 levels already decoded: the fused kernel
+// where it applies, else the rotate-quantize kernel and the decoded-weight
+// contraction in turn.  ws: [A operand | norms | row-group flags].
+static oq_status fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint16_t* w16,
+                               const float* r, void* y, bool y_bf16, unsigned char* ws, void* stream) {
+  if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
+  const size_t need = min_workspace(L, T);
+  uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
+  float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
+  const RQArgs ra = rq_levels_args(L, x, x_dtype, T, a16, s);
+  if (fused_kernel_supported(ra, L->d_out)) {
+    int* flags = reinterpret_cast<int*>(ws + round256(need));
+    const oq_status st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), flags, stream);
+    if (st != OQ_ERR_UNSUPPORTED) return st;
+  }
+  const oq_status st = rq_levels(L, x, x_dtype, T, a16, s, stream);
+  return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16, r, y, y_bf16, stream);
+}
+
 // The fused call's body on checked arguments.  w16_ready: the weights' fp16
 // levels, already decoded by the caller (oq_linear_fused_host decodes them
 // once for all its chunks), or null.
@@ -626,18 +650,11 @@ static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype,
     // write the A operand while the contraction runs, where it applies;
     // otherwise decode weights inside the contraction
     if (fused_w16_route(L, x_dtype, T) && workspace_bytes >= full_workspace(L, T, need)) {
-      if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
-      uint16_t* w16 = reinterpret_cast<uint16_t*>(ws + round256(need));
+      // workspace: [A operand | norms | row-group flags | decoded weights]
+      uint16_t* w16 = reinterpret_cast<uint16_t*>(ws + decoded_workspace(L, T));
       st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
       if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_fused: unsupported shape") : st;
-      const RQArgs ra = rq_levels_args(L, x, x_dtype, T, a16, s);
-      if (fused_kernel_supported(ra, L->d_out)) {
-        int* flags = reinterpret_cast<int*>(ws + round256(need) + fused_w16_bytes(L));
-        st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), flags, stream);
-        if (st != OQ_ERR_UNSUPPORTED) return st;
-      }
-      st = rq_levels(L, x, x_dtype, T, a16, s, stream);
-      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16, r, y, y_bf16, stream);
+      return fused_decoded(L, x, x_dtype, T, w16, r, y, y_bf16, ws, stream);
     }
     st = rq_levels(L, x, x_dtype, T, a16, s, stream);
     if (st != OQ_OK) return st;
@@ -679,6 +696,29 @@ oq_status oq_linear_fused(const oq_layer* L, const void* x, int32_t x_dtype, int
   if (workspace_bytes < min_workspace(L, T)) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused: workspace too small");
   return fused_device(L, x, x_dtype, T, Wcodes, r, y, y_dtype == OQ_DTYPE_BF16,
                       static_cast<unsigned char*>(workspace), workspace_bytes, stream, nullptr);
+}
+
+size_t oq_linear_fused_decoded_workspace_size(const oq_layer* L, int64_t T) {
+  if (!L || T <= 0 || L->int4_only || L->fp8 || L->d_out % 256) return 0;
+  return decoded_workspace(L, T);
+}
+
+oq_status oq_linear_fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint16_t* w16,
+                                  const float* r, void* y, int32_t y_dtype, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  const char* who = "oq_linear_fused_decoded";
+  if (!L) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused_decoded: layer is null");
+  if (L->int4_only) return not_for_int4(L, who);
+  if (L->fp8) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_fused_decoded: the fp16-level route is not used in the FP8 mode");
+  if (L->d_out % 256 != 0) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_fused_decoded: needs d_out % 256 == 0");
+  oq_status st = fused_checks(L, x, x_dtype, T, reinterpret_cast<const uint32_t*>(w16), r, y, y_dtype, workspace, who);
+  if (st != OQ_OK || T == 0) return st;
+  if (x_dtype != OQ_DTYPE_BF16) return fail(OQ_ERR_UNSUPPORTED, "oq_linear_fused_decoded: bf16 input only");
+  if (!aligned(w16, 16)) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused_decoded: w16 must be 16-byte aligned");
+  if (workspace_bytes < decoded_workspace(L, T))
+    return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused_decoded: workspace too small");
+  return fused_decoded(L, x, x_dtype, T, w16, r, y, y_dtype == OQ_DTYPE_BF16, static_cast<unsigned char*>(workspace),
+                       stream);
 }
 
 oq_status oq_poll_error(const oq_layer* L) {

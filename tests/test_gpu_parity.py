@@ -362,7 +362,11 @@ def test_decoded_weight_route(env, d_in, d_out, a_bits, w_bits, T):
     assert full >= d_out * d_in * 2 + T * d_in * 2
     y_full = B.oq_linear_fused(layer, x_t, Wc, r)
     a16, s = B.oq_rotate_quantize_levels(layer, x_t)
-    y_stage = B.oq_linear_decoded(layer, a16, s, B.oq_weight_levels(layer, Wc), r)
+    w16 = B.oq_weight_levels(layer, Wc)
+    y_stage = B.oq_linear_decoded(layer, a16, s, w16, r)
+    # the same route after its weight decode: where the block size allows, the
+    # kernel that rotates, quantizes and contracts in one launch
+    y_fd = B.oq_linear_fused_decoded(layer, x_t, w16, r)
     # the least workspace: the fp16 A operand (rounded up to 256 bytes) and the norms
     least = (T * d_in * 2 + 255) // 256 * 256 + T * 4
     ws = torch.empty((least,), dtype=torch.uint8, device="cuda")
@@ -371,6 +375,7 @@ def test_decoded_weight_route(env, d_in, d_out, a_bits, w_bits, T):
     torch.cuda.synchronize()
     B.oq_poll_error(layer)
     np.testing.assert_array_equal(y_full.cpu().numpy(), y_stage.cpu().numpy())
+    np.testing.assert_array_equal(y_fd.cpu().numpy(), y_stage.cpu().numpy())
     np.testing.assert_array_equal(y_least.cpu().numpy(), y_lv.cpu().numpy())
     np.testing.assert_array_equal(y_full.cpu().numpy(), y_lv.cpu().numpy())
     with pytest.raises(B.OrbitQuantError):
