@@ -21,7 +21,7 @@ LIB = os.path.join(HERE, "liborbitquant.so")
 
 SOURCES = ["oq_api.cu", "oq_rotate_quantize.cu", "oq_rotate_quantize_tc.cu", "oq_gemm.cu", "oq_gemm_pair.cu", "oq_gemm_skinny.cu", "oq_gemm_w16.cu",
            "oq_levels.cu", "oq_host_io.cu", "oq_int4.cu",
-           "oq_noalloc.cu", "oq_diag.cu", "oq_fused.cu", "oq_weight_io.cpp", "oq_host.cpp"]
+           "oq_noalloc.cu", "oq_diag.cu", "oq_fused.cu", "oq_gemv.cu", "oq_weight_io.cpp", "oq_host.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17"]
 

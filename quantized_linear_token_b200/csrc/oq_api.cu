@@ -389,6 +389,10 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
   // a few hundred tokens or fewer: the small-batch kernel (weight rows as the
   // MMA's M, split K, its splits added in fp32 in y itself, so fp32 y only);
   // larger batches and bf16 y: the CTA-pair kernel
+  if (a_f16 && T <= GEMV_MAX_T && !L->fp8) {
+    const oq_status st = gemv_launch(g, stream);
+    if (st != OQ_ERR_UNSUPPORTED) return st;
+  }
   if (a_f16 && T <= SKINNY_MAX_T && L->d_counters && !y_bf16) return gemm_skinny_launch(g, L->d_counters, stream);
   return gemm_launch(g, stream);
 }

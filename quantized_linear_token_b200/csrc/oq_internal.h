@@ -131,6 +131,11 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream);
 // small-batch contraction (oq_gemm_skinny.cu): fp16 A operand, T <= SKINNY_MAX_T,
 // N % 128 == 0; `counters` holds N / 32 zeroed ints
 constexpr int SKINNY_MAX_T = 256;
+// GEMV contraction for up to GEMV_MAX_T tokens (oq_gemv.cu): fp16 A operand,
+// weight codes of 2-4 bits decoded in registers, warp MMAs, no split across
+// CTAs; N % 16 == 0, K % 32 == 0
+constexpr int GEMV_MAX_T = 8;
+oq_status gemv_launch(const GemmArgs& g, void* stream);
 oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream);
 // INT4 weight-only round-to-nearest of weight rows (oq_int4.cu): per-row
 // scale max|w| / 7 and 4-bit codes of q in [-7, 7] (q >= 0 -> q + 8, else q + 7)

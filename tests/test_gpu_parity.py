@@ -230,6 +230,26 @@ def test_small_batch_sweep(env, T):
     _run_layer(env, 13824, 5120, 4, 4, x_np, Wm, w_rows=w_rows, label=f"small{T}")
 
 
+GEMV = [
+    # d_in, d_out, a, w, T: batches of up to 8 tokens take the GEMV kernel
+    # (weights streamed once, warp MMAs, K split over a CTA's warps): every
+    # weight width, a K that is not a multiple of the 128-position chunk, 8-bit
+    # activations, and the largest batch it takes
+    (96, 256, 4, 2, 3),
+    (3072, 512, 4, 4, 1),
+    (3072, 512, 3, 3, 8),
+    (5120, 256, 4, 2, 2),
+    (13824, 512, 8, 4, 5),
+]
+
+
+@pytest.mark.parametrize("d_in,d_out,a_bits,w_bits,T", GEMV)
+def test_gemv_batches(env, d_in, d_out, a_bits, w_bits, T):
+    x_np = W.custom_activations(T, d_in, seed=d_in + 11 * T)
+    Wm = W.custom_weights(d_out, d_in, seed=d_out + 13)
+    _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, label=f"gemv {d_in}x{d_out} T={T}")
+
+
 @pytest.mark.parametrize("T,d_in,d_out,w_bf16", [(2, 3072, 18432, False), (7, 1024, 256, True),
                                                    (300, 512, 384, False)])
 def test_int4_weight_only_layer(env, T, d_in, d_out, w_bf16):
