@@ -96,6 +96,7 @@ void oq_layer_destroy(oq_layer* L) {
   cudaFree(L->bins_w.d_codes);
   cudaFree(L->bins_w.d_levels);
   cudaFree(L->bins_a_full.d_levels);
+  cudaFree(L->bins_a_full.d_codes);
   cudaFree(L->d_counters);
   cudaFree(L->d_error);
   delete L;
@@ -259,7 +260,10 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
   upload(&L->bins_a.d_levels, ta_levels);
   upload(&L->bins_w.d_codes, tw_codes);
   upload(&L->bins_w.d_levels, tw_levels);
-  if (full_table) upload(&L->bins_a_full.d_levels, taf_levels);
+  if (full_table) {
+    upload(&L->bins_a_full.d_levels, taf_levels);
+    upload(&L->bins_a_full.d_codes, taf_codes);
+  }
   if (st == OQ_OK && d_out % 128 == 0) {
     const size_t cb = (size_t)(d_out / 32) * sizeof(int);
     st = cuda_check(cudaMalloc(&L->d_counters, cb), "cudaMalloc(split counters)");
@@ -327,6 +331,18 @@ static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t row
   a.codes = codes;
   a.norms = norms;
   a.err = L->d_error;
+  // activation rows in bf16 at a block size of 1024 or 512: the tensor-core
+  // block transform, writing the packed codes
+  if (&bins == &L->bins_a && L->d_gather_tc) {
+    a.gather_tc = L->d_gather_tc;
+    a.bins_full = L->bins_a_full.d_codes;
+    a.nb_full = L->bins_a_full.nb;
+    a.b0_full = L->bins_a_full.b0;
+    if (rqtc_supported(a)) {
+      const oq_status st = rqtc_launch(a, stream);
+      if (st != OQ_ERR_UNSUPPORTED) return st;
+    }
+  }
   return rq_launch(a, stream);
 }
 

@@ -65,14 +65,35 @@ struct TCParams {
   int d, nw;           // nw = d / h warps per CTA
   int stage_bytes;     // per row buffer
   const uint16_t* gather;
-  uint16_t* out16;     // fp16 levels [rows, d]
+  uint16_t* out16;     // fp16 levels [rows, d], or
+  uint32_t* codes;     // packed codes [rows, d * bits / 32]
+  int bits;
   float* norms;
   int* err;
-  const uint2* bins;   // {threshold bits, fp16 level pair}
+  const uint2* bins;   // {threshold bits, fp16 level pair} (or {threshold bits, base code} for codes)
   int nb, b0;
   int full;            // the table spans every g of a token with a normal fp32 norm
   float kscale;
 };
+
+// packed-code output at the layer's activation width
+template <int MT2>
+__device__ __forceinline__ void store_codes(int bits, bool unclamped, const float (&D2)[MT2][4][4], float ks,
+                                            float magic, int bin_lo, int bin_hi, uint32_t tbl_shift, uint32_t* grp,
+                                            int g, int q) {
+#define OQ_STORE_CODES(B)                                                                                  \
+  if (unclamped)                                                                                           \
+    rqtc::quantize_store_codes<false, MT2, B>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, grp, g, q);         \
+  else                                                                                                     \
+    rqtc::quantize_store_codes<true, MT2, B>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, grp, g, q);
+  switch (bits) {
+    case 2: OQ_STORE_CODES(2) break;
+    case 3: OQ_STORE_CODES(3) break;
+    case 4: OQ_STORE_CODES(4) break;
+    default: OQ_STORE_CODES(8) break;
+  }
+#undef OQ_STORE_CODES
+}
 
 // A = rows of the block matrix (h / 32): MT2 = A / 16 pass-2 row tiles
 template <int A>
@@ -152,15 +173,21 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
     // ---- quantize: Z[a'][b'] for a' = 16 mt + g + 8 half, b' = 8 nt + 2q + {0, 1}
     // (the bin-table search of rq_kernel), fp16 level pairs stored as words
     const float ks = (s > 0.f) ? p.kscale / s : 0.f;
-    uint16_t* rowout = p.out16 + (size_t)t * p.d + (size_t)warp * H + 2 * q;
     // With a full-range table every finite g of a token whose squared norm is
     // a normal fp32 number lies inside it (|g| <= K sqrt(d) up to rounding),
     // so the bin index needs no clamp.  Other tokens (a norm that under- or
     // overflowed in fp32, non-finite values, zero) take the clamped search.
-    if (p.full && s2 >= 1e-30f && s2 <= 1e30f)
-      rqtc::quantize_store<false, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
-    else
-      rqtc::quantize_store<true, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+    const bool unclamped = p.full && s2 >= 1e-30f && s2 <= 1e30f;
+    if (p.codes) {
+      uint32_t* grp = p.codes + (size_t)t * ((size_t)p.d * p.bits / 32) + (size_t)warp * A * p.bits;
+      store_codes<MT2>(p.bits, unclamped, D2, ks, magic, bin_lo, bin_hi, tbl_shift, grp, g, q);
+    } else {
+      uint16_t* rowout = p.out16 + (size_t)t * p.d + (size_t)warp * H + 2 * q;
+      if (unclamped)
+        rqtc::quantize_store<false, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+      else
+        rqtc::quantize_store<true, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+    }
     if (tid == 0) p.norms[t] = s;
   }
 }
@@ -168,7 +195,8 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
 }  // namespace
 
 bool rqtc_supported(const RQArgs& a) {
-  return a.out16 && (a.h == 1024 || a.h == 512) && a.src_dtype == OQ_DTYPE_BF16 && !a.signmask && a.gather_tc &&
+  return (a.out16 || (a.codes && (a.bits == 2 || a.bits == 3 || a.bits == 4 || a.bits == 8))) &&
+         (a.h == 1024 || a.h == 512) && a.src_dtype == OQ_DTYPE_BF16 && !a.signmask && a.gather_tc &&
          a.d % a.h == 0 && a.d / a.h >= 1 && a.d / a.h <= (a.h == 1024 ? 8 : 32) && a.nb >= 1 &&
          a.nb <= OQ_MAX_BINS;
 }
@@ -214,6 +242,8 @@ oq_status rqtc_launch(const RQArgs& a, void* stream) {
   p.stage_bytes = (a.d * 2 + 127) & ~127;
   p.gather = a.gather_tc;
   p.out16 = a.out16;
+  p.codes = a.out16 ? nullptr : a.codes;
+  p.bits = a.bits;
   p.norms = a.norms;
   p.err = a.err;
   if (a.bins_full) {

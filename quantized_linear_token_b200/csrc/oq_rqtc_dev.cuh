@@ -104,6 +104,60 @@ __device__ __forceinline__ void quantize_store(const float (&D2)[MT2][4][4], flo
       }
 }
 
+// The same quantization writing packed codes (the format of oq_rotate_quantize:
+// each group of 32 positions is a little-endian stream of 32 BITS bits in BITS
+// words).  Row a' of the block is positions [32 a', 32 a' + 32): one group.
+// A lane holds 8 of its codes (positions 8 nt + 2q + {0, 1}), placed at bits
+// BITS (8 nt + 2q + j) of the group's stream; the four lanes of the quad OR
+// their words together and lane q stores words q, q + 4 (BITS words in all,
+// one 4 BITS-byte run per group).  `grp` points to group 0 of the block.
+template <bool CLAMP, int MT2, int BITS>
+__device__ __forceinline__ void quantize_store_codes(const float (&D2)[MT2][4][4], float ks, float magic, int bin_lo,
+                                                     int bin_hi, uint32_t tbl_shift, uint32_t* grp, int g, int q) {
+#pragma unroll
+  for (int mt = 0; mt < MT2; ++mt)
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t w[BITS];
+#pragma unroll
+      for (int i = 0; i < BITS; ++i) w[i] = 0u;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        float g0, g1, t0, t1;
+        mul2(g0, g1, D2[mt][nt][2 * half], D2[mt][nt][2 * half + 1], ks);
+        add2(t0, t1, g0, g1, magic);
+        int m0 = __float_as_int(t0), m1 = __float_as_int(t1);
+        if (CLAMP) {
+          m0 = min(max(m0, bin_lo), bin_hi);
+          m1 = min(max(m1, bin_lo), bin_hi);
+        }
+        const uint2 e0 = lds_v2(tbl_shift + 8u * (uint32_t)m0);
+        const uint2 e1 = lds_v2(tbl_shift + 8u * (uint32_t)m1);
+        // code = the bin's base code, plus one above the bin's threshold
+        const uint32_t c0 = e0.y + (g0 > __uint_as_float(e0.x) ? 1u : 0u);
+        const uint32_t c1 = e1.y + (g1 > __uint_as_float(e1.x) ? 1u : 0u);
+        // both codes of the pair: 2 BITS bits starting at bit BITS (8 nt + 2q)
+        const uint32_t pair = c0 | (c1 << BITS);
+        const int bit = BITS * (8 * nt + 2 * q);
+#pragma unroll
+        for (int i = 0; i < BITS; ++i) {
+          const int lo = bit - 32 * i;     // the pair's offset within word i
+          if (lo >= 0 && lo < 32) w[i] |= pair << lo;
+          if (lo < 0 && lo > -2 * BITS) w[i] |= pair >> (-lo);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < BITS; ++i) {
+        w[i] |= __shfl_xor_sync(0xffffffffu, w[i], 1);
+        w[i] |= __shfl_xor_sync(0xffffffffu, w[i], 2);
+      }
+      uint32_t* out = grp + (16 * mt + g + 8 * half) * BITS;
+#pragma unroll
+      for (int i = 0; i < BITS; ++i)
+        if ((i & 3) == q) out[i] = w[i];
+    }
+}
+
 // Per-lane constants of the two passes: the pass-1 A fragments of H_32 (hp,
 // and hn = the negated tile) and the four values that make up every pass-2 A
 // fragment of H_A.
