@@ -409,7 +409,10 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
     const oq_status st = gemv_launch(g, stream);
     if (st != OQ_ERR_UNSUPPORTED) return st;
   }
-  if (a_f16 && T <= SKINNY_MAX_T && L->d_counters && !y_bf16) return gemm_skinny_launch(g, L->d_counters, stream);
+  if (a_f16 && T <= SKINNY_MAX_T && L->d_counters && !y_bf16) {
+    const oq_status st = gemm_skinny_launch(g, L->d_counters, stream);
+    if (st != OQ_ERR_UNSUPPORTED) return st;
+  }
   return gemm_launch(g, stream);
 }
 

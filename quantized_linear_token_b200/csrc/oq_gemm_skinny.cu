@@ -8,7 +8,9 @@
 // the workload sweep).  Every weight row is decoded once per call.  With few
 // weight-row tiles the K range is split so that every SM gets work; the splits
 // of a tile add into y one after another (split s waits for split s - 1 on a
-// per-tile counter), so the result does not depend on timing.
+// per-tile counter), so the result does not depend on timing.  The waits need
+// every CTA of the grid resident at once, which the cooperative launch
+// guarantees.
 //
 // Warps: 0-15 decode weight codes (two groups on alternate K blocks), 16-19
 // epilogue (TMEM lane quarters 0-3), 20 issues the MMAs (M 128, N = padded T,
@@ -395,8 +397,27 @@ oq_status launch_skinny(const SkinnyParams& kp_in, void* stream) {
   kp.ks = (kp.nkb + kp.kps - 1) / kp.kps;
   kp.items = kp.n_tiles * kp.ks;
   const int grid = std::min(kp.items, sms);
-  kern<<<grid, NTHREADS, smem, static_cast<cudaStream_t>(stream)>>>(kp);
-  e = cudaGetLastError();
+  // the splits of a tile hand over through counters, so every CTA of the grid
+  // must be resident at once: a cooperative launch guarantees that, or fails
+  // (and the caller takes another kernel) when the GPU cannot hold the grid
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, kp);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    cudaGetLastError();
+    set_error("gemm skinny: the GPU cannot hold the whole grid at once");
+    return OQ_ERR_UNSUPPORTED;
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("gemm skinny launch: ") + cudaGetErrorString(e));
     return OQ_ERR_CUDA;
