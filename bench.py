@@ -722,7 +722,9 @@ def run_sweep(args):
             else:
                 stages += [("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]
             runs = {"step": [("step", lambda: B.oq_linear_fused(layer, x, Wc, r, y, ws))], "stages": stages}
-            if decoded:
+            h_blk = d & -d
+            if decoded and ((h_blk == 1024 and d // h_blk <= 8) or (h_blk == 512 and d // h_blk <= 12)):
+                # the step runs the fused kernel: time it on its own
                 ws_fd = torch.empty((max(B.oq_linear_fused_decoded_workspace_size(layer, T), 1),),
                                     dtype=torch.uint8, device=dev)
                 runs["fused"] = [("fused", lambda: B.oq_linear_fused_decoded(layer, x, w16, r, y, ws_fd))]
