@@ -70,6 +70,11 @@ oq_status oq_rotation_build(int32_t d, uint64_t seed, int32_t flags, uint32_t* p
   return OQ_OK;
 }
 
+// Blocks of 1024 take the block transform on the CUDA cores (oq_rqcc_dev.cuh)
+// rather than on the warp MMAs, in the stand-alone rotate-quantize kernel and
+// in the fused kernel's producer warps.
+constexpr bool kCudaCoreBlockTransform = true;
+
 static oq_status check_shape(int32_t d_in, int32_t d_out, int32_t a_bits, int32_t w_bits) {
   if (d_in <= 0 || d_out <= 0) return fail(OQ_ERR_INVALID_ARG, "dimensions must be positive");
   if (d_in % 32) return fail(OQ_ERR_UNSUPPORTED, "d_in must be a multiple of 32");
@@ -88,6 +93,7 @@ void oq_layer_destroy(oq_layer* L) {
   io_release(L);
   cudaFree(L->d_gather_a);
   cudaFree(L->d_gather_tc);
+  cudaFree(L->d_gather_cc);
   cudaFree(L->d_signmask);
   cudaFree(L->d_levels_a);
   cudaFree(L->d_levels_w);
@@ -241,6 +247,14 @@ oq_status oq_layer_create(int32_t d_in, int32_t d_out, uint64_t seed, int32_t a_
     if (st == OQ_OK)
       st = cuda_check(cudaMemcpy(L->d_gather_tc, gather_tc.data(), gather_tc.size() * sizeof(uint16_t),
                                  cudaMemcpyHostToDevice), "upload gather");
+    if (st == OQ_OK && L->h == 1024 && kCudaCoreBlockTransform) {
+      std::vector<uint16_t> gather_cc;
+      rqcc_build_gather(d_in, L->perm_host, gather_cc);
+      st = cuda_check(cudaMalloc(&L->d_gather_cc, gather_cc.size() * sizeof(uint16_t)), "cudaMalloc(gather)");
+      if (st == OQ_OK)
+        st = cuda_check(cudaMemcpy(L->d_gather_cc, gather_cc.data(), gather_cc.size() * sizeof(uint16_t),
+                                   cudaMemcpyHostToDevice), "upload gather");
+    }
   }
   if (st == OQ_OK && signed_rot) {
     st = cuda_check(cudaMalloc(&L->d_signmask, signmask.size() * sizeof(uint32_t)), "cudaMalloc(signs)");
@@ -335,6 +349,7 @@ static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t row
   // block transform, writing the packed codes
   if (&bins == &L->bins_a && L->d_gather_tc) {
     a.gather_tc = L->d_gather_tc;
+    a.gather_cc = L->d_gather_cc;
     a.bins_full = L->bins_a_full.d_codes;
     a.nb_full = L->bins_a_full.nb;
     a.b0_full = L->bins_a_full.b0;
@@ -506,6 +521,7 @@ static RQArgs rq_levels_args(const oq_layer* L, const void* x, int32_t x_dtype, 
   a.norms = s;
   a.err = L->d_error;
   a.gather_tc = L->d_gather_tc;
+  a.gather_cc = L->d_gather_cc;
   a.bins_full = L->bins_a_full.d_levels;
   a.nb_full = L->bins_a_full.nb;
   a.b0_full = L->bins_a_full.b0;

@@ -34,6 +34,7 @@
 #include "oq_internal.h"
 #include "oq_epilogue.cuh"
 #include "oq_ptx.cuh"
+#include "oq_rqcc_dev.cuh"
 #include "oq_rqtc_dev.cuh"
 #include "oq_tmap.cuh"
 
@@ -108,7 +109,11 @@ __device__ __forceinline__ bool wait_flags(const int* f, int cnt, int lane, int*
   }
 }
 
-template <int A>
+// CC: the producers' block transform runs on the CUDA cores (h = 1024,
+// oq_rqcc_dev.cuh: no warp MMAs, so they never wait behind the contraction's
+// tcgen05 MMAs), with a 4 KB transpose tile per producer warp; otherwise on
+// the warp MMAs (oq_rqtc_dev.cuh)
+template <int A, bool CC>
 __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
     fused_kernel(const __grid_constant__ FusedParams p) {
   constexpr int MT2 = A / 16, H = 32 * A;
@@ -128,7 +133,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
   const int gtab_off = (8 * p.nb + 15) & ~15;
   uint4* gtab = reinterpret_cast<uint4*>(prod + gtab_off);
   const int teams_off = (gtab_off + 2 * A * team_threads + 127) & ~127;
-  const int team_bytes = TEAM_HDR + 2 * p.stage_bytes;
+  const int team_bytes = TEAM_HDR + (CC ? p.nw * 4096 : 0) + 2 * p.stage_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -178,9 +183,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
     uint64_t* mbar = reinterpret_cast<uint64_t*>(tbase);
     float* red = reinterpret_cast<float*>(tbase + 16);
     volatile int* slot = reinterpret_cast<volatile int*>(tbase + 16 + 256);
-    unsigned char* stage = tbase + TEAM_HDR;
+    float* tile = reinterpret_cast<float*>(tbase + TEAM_HDR + w * 4096);   // CC only
+    unsigned char* stage = tbase + TEAM_HDR + (CC ? p.nw * 4096 : 0);
     const uint32_t stage_addr0 = smem_u32(stage);
-    const rqtc::Lane lc = rqtc::make_lane(lane);
+    const rqtc::Lane lc = rqtc::make_lane(lane);   // tensor-core transform only
     const uint32_t row_bytes = (uint32_t)p.K * 2u;
     const float magic = 12582912.0f + (float)p.b0;
     const int bin_lo = 0x4B400000, bin_hi = 0x4B400000 + p.nb - 1;
@@ -222,7 +228,12 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
         const bool ok = mbar_wait(&mbar[buf], (uint32_t)(it >> 1) & 1u, p.err);
         const uint32_t sa = stage_addr0 + (uint32_t)(buf * p.stage_bytes);
         float D2[MT2][4][4];
-        const float ss = rqtc::transform_block<A>(lc, gtab, team_threads, ttid, sa, D2);
+        float zc[32];
+        float ss;
+        if constexpr (CC)
+          ss = rqcc::transform_block(gtab, team_threads, ttid, sa, tile, lane, zc);
+        else
+          ss = rqtc::transform_block<A>(lc, gtab, team_threads, ttid, sa, D2);
         if (lane == 0) red[buf * 32 + w] = ss;
         if (named_bar_or(bar_id, team_threads, !ok)) {
           if (issued) mbar_wait(&mbar[buf ^ 1], (uint32_t)((it + 1) >> 1) & 1u, p.err);
@@ -231,13 +242,23 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
         }
         float s2 = 0.f;
         for (int v = 0; v < p.nw; ++v) s2 += red[buf * 32 + v];
-        const float s = sqrtf(s2 * (1.0f / 32.0f));
+        // the tensor-core transform's partials are 32 sum y^2 (from P)
+        const float s = CC ? sqrtf(s2) : sqrtf(s2 * (1.0f / 32.0f));
         const float ks = (s > 0.f) ? p.kscale / s : 0.f;
-        uint16_t* rowout = p.a16 + (size_t)t * p.K + (size_t)w * H + 2 * q;
-        if (p.full && s2 >= 1e-30f && s2 <= 1e30f)
-          rqtc::quantize_store<false, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
-        else
-          rqtc::quantize_store<true, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+        const bool unclamped = p.full && s2 >= 1e-30f && s2 <= 1e30f;
+        if constexpr (CC) {
+          uint16_t* out = p.a16 + (size_t)t * p.K + (size_t)w * H + 32 * lane;
+          if (unclamped)
+            rqcc::quantize_levels<false>(zc, ks, magic, bin_lo, bin_hi, tbl_shift, out);
+          else
+            rqcc::quantize_levels<true>(zc, ks, magic, bin_lo, bin_hi, tbl_shift, out);
+        } else {
+          uint16_t* rowout = p.a16 + (size_t)t * p.K + (size_t)w * H + 2 * q;
+          if (unclamped)
+            rqtc::quantize_store<false, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+          else
+            rqtc::quantize_store<true, MT2>(D2, ks, magic, bin_lo, bin_hi, tbl_shift, rowout, g);
+        }
         if (leader) p.norms[t] = s;
       }
       if (failed) break;
@@ -371,13 +392,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
   }
 }
 
-size_t smem_bytes(int A, int nb, int nw, int teams, int stage_bytes, int* prod_off) {
+size_t smem_bytes(int A, bool cc, int nb, int nw, int teams, int stage_bytes, int* prod_off) {
   const int off = OS * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
   const int team_threads = nw * 32;
   const int gtab_off = (8 * nb + 15) & ~15;
   const int teams_off = (gtab_off + 2 * A * team_threads + 127) & ~127;
   if (prod_off) *prod_off = off;
-  return 1024 + (size_t)off + teams_off + (size_t)teams * (TEAM_HDR + 2 * (size_t)stage_bytes);
+  return 1024 + (size_t)off + teams_off + (size_t)teams * (TEAM_HDR + (cc ? (size_t)nw * 4096 : 0) +
+                                                           2 * (size_t)stage_bytes);
 }
 
 }  // namespace
@@ -390,7 +412,7 @@ bool fused_kernel_supported(const RQArgs& a, int N) {
   if (GEMM_WARPS + nw > MAX_WARPS) return false;
   const int stage_bytes = (a.d * 2 + 127) & ~127;
   const int nb = a.bins_full ? a.nb_full : a.nb;
-  return smem_bytes(A, nb, nw, 1, stage_bytes, nullptr) <= 227 * 1024;
+  return smem_bytes(A, A == 32 && a.gather_cc, nb, nw, 1, stage_bytes, nullptr) <= 227 * 1024;
 }
 
 oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream) {
@@ -411,7 +433,8 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* str
   kp.n_items = (int)((g.M + RG - 1) / RG);
   kp.flags = flags;
   kp.counter = flags + kp.n_items + 32;   // its own line, away from the flags
-  kp.gather = a.gather_tc;
+  const bool cc = a.h == 1024 && a.gather_cc;
+  kp.gather = cc ? a.gather_cc : a.gather_tc;
   if (a.bins_full) {
     kp.bins = reinterpret_cast<const uint2*>(a.bins_full);
     kp.nb = a.nb_full;
@@ -426,13 +449,13 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* str
   const int A = a.h / 32;
   kp.nw = a.d / a.h;
   kp.stage_bytes = (a.d * 2 + 127) & ~127;
-  auto kern = A == 32 ? fused_kernel<32> : fused_kernel<16>;
+  auto kern = cc ? fused_kernel<32, true> : (A == 32 ? fused_kernel<32, false> : fused_kernel<16, false>);
   // as many teams as the warp budget, shared memory and the SM's registers
   // allow (the occupancy query says whether one CTA of that shape fits)
   int teams = (MAX_WARPS - GEMM_WARPS) / kp.nw;
   size_t smem = 0;
   for (; teams >= 1; --teams) {
-    smem = smem_bytes(A, kp.nb, kp.nw, teams, kp.stage_bytes, &kp.prod_off);
+    smem = smem_bytes(A, cc, kp.nb, kp.nw, teams, kp.stage_bytes, &kp.prod_off);
     if (smem > 227 * 1024) continue;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) continue;
     int per_sm = 0;

@@ -38,6 +38,7 @@ struct oq_layer {
   // device tables (owned)
   uint16_t* d_gather_a;               // rotate-quantize gather offsets, kernel order
   uint16_t* d_gather_tc;              // the same for the tensor-core FWHT kernel (h = 1024 or 512), or null
+  uint16_t* d_gather_cc;              // the same for the CUDA-core block kernel (h = 1024), or null
   uint32_t* d_signmask;               // sign bits in kernel order, or null
   uint16_t* d_levels_a;               // fp16 bits of a_scale * activation levels
   uint16_t* d_levels_w;               // fp16 bits of w_scale * weight levels
@@ -80,6 +81,7 @@ struct RQArgs {
   int d, h, log_h, bits;
   const uint16_t* gather;    // per-thread gather offsets (kernel order)
   const uint16_t* gather_tc; // offsets in the tensor-core kernel's order, or null
+  const uint16_t* gather_cc; // offsets in the CUDA-core block kernel's order (h = 1024), or null
   const uint32_t* bins_full; // full-range levels table (no clamping needed), or null
   int nb_full, b0_full;
   const uint32_t* signmask;  // or null
@@ -99,6 +101,8 @@ oq_status rq_launch(const RQArgs& a, void* stream);
 // rotate-quantize with the block FWHT on the tensor cores (h = 1024 or 512,
 // bf16 input, fp16-level output, no signs; oq_rotate_quantize_tc.cu)
 void rqtc_build_gather(int d, int h, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather);
+// the same for the CUDA-core block transform (h = 1024; rqcc_kernel and the fused kernel)
+void rqcc_build_gather(int d, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather);
 bool rqtc_supported(const RQArgs& a);
 oq_status rqtc_launch(const RQArgs& a, void* stream);
 
