@@ -70,9 +70,10 @@ oq_status oq_rotation_build(int32_t d, uint64_t seed, int32_t flags, uint32_t* p
   return OQ_OK;
 }
 
-// Blocks of 1024 take the block transform on the CUDA cores (oq_rqcc_dev.cuh)
-// rather than on the warp MMAs, in the stand-alone rotate-quantize kernel and
-// in the fused kernel's producer warps.
+// The fused kernel's producer warps run the block transform of h = 1024 on the
+// CUDA cores (oq_rqcc_dev.cuh): beside the tcgen05 contraction, warp MMAs
+// would wait behind it.  (The stand-alone kernels keep the warp-MMA transform,
+// which is faster on its own.)
 constexpr bool kCudaCoreBlockTransform = true;
 
 static oq_status check_shape(int32_t d_in, int32_t d_out, int32_t a_bits, int32_t w_bits) {
@@ -349,7 +350,6 @@ static oq_status rq(const oq_layer* L, const void* x, int32_t dtype, int64_t row
   // block transform, writing the packed codes
   if (&bins == &L->bins_a && L->d_gather_tc) {
     a.gather_tc = L->d_gather_tc;
-    a.gather_cc = L->d_gather_cc;
     a.bins_full = L->bins_a_full.d_codes;
     a.nb_full = L->bins_a_full.nb;
     a.b0_full = L->bins_a_full.b0;

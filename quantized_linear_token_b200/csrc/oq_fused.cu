@@ -45,7 +45,7 @@ constexpr int RM = 128;            // A rows per CTA (pair M = 256)
 constexpr int PN = 256;            // output columns per pair tile
 constexpr int RN = 128;            // B rows per CTA
 constexpr int BK = 64;             // K elements per stage
-constexpr int OS = 4;              // operand stages
+constexpr int MAX_OS = 6;          // operand stages (the launch picks 3 to 6)
 constexpr int A_TILE = RM * BK * 2;
 constexpr int B_TILE = RN * BK * 2;
 constexpr int STAGE_BYTES = A_TILE + B_TILE;
@@ -81,10 +81,17 @@ struct FusedParams {
   float kscale;
   int nw, teams;             // warps per team (d / h), teams per CTA
   int stage_bytes;           // one staged row, 128-byte multiple
+  int row_bufs;              // staged rows per team: 2 (the next row loads during this one) or 1
+  int os;                    // operand stages of the contraction
   int prod_off;              // byte offset of the producer region in shared memory
 };
 
 constexpr int RG = 4;              // token rows per queue group: 32 groups per 128-row tile
+// the contraction's operand stages and the producer teams' staged rows: the
+// shared memory left by the stages holds the teams, so these trade the
+// contraction's latency cover against the number of producer warps
+constexpr int kStages = 4;
+constexpr int kRowBuffers = 2;
 
 // Waits (bounded) until the `cnt` (<= 32) flags at f are all set, polling
 // with every lane of the warp.  Each lane turns the relaxed read that saw its
@@ -120,10 +127,11 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
       reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int OS = p.os;
   unsigned char* epi = smem + OS * STAGE_BYTES;
   uint64_t* op_full = reinterpret_cast<uint64_t*>(epi + EPI_BYTES);
-  uint64_t* op_empty = op_full + OS;
-  uint64_t* acc_full = op_empty + OS;
+  uint64_t* op_empty = op_full + MAX_OS;
+  uint64_t* acc_full = op_empty + MAX_OS;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   // producer region: threshold table | gather offsets (transposed, uint4) | teams
@@ -133,7 +141,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
   const int gtab_off = (8 * p.nb + 15) & ~15;
   uint4* gtab = reinterpret_cast<uint4*>(prod + gtab_off);
   const int teams_off = (gtab_off + 2 * A * team_threads + 127) & ~127;
-  const int team_bytes = TEAM_HDR + (CC ? p.nw * 4096 : 0) + 2 * p.stage_bytes;
+  const int team_bytes = TEAM_HDR + (CC ? p.nw * 4096 : 0) + p.row_bufs * p.stage_bytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -205,27 +213,32 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
     int item = slot[0];
     int it = 0, done = 0;
     bool failed = false;
+    // two row buffers: the next row's copy starts with this row; one: it
+    // starts once every warp of the team has gathered this row
+    const bool dbl = p.row_bufs == 2;
+    // the row after t: the next in its group, or the first of a newly
+    // claimed group (whose index the team reads from slot after the group)
+    auto next_row = [&](int64_t t, int64_t r1) -> int64_t {
+      if (t + 1 < r1) return t + 1;
+      const int nitem = atomicAdd(p.counter, 1);
+      slot[(done + 1) & 1] = nitem;
+      return nitem < p.n_items ? (int64_t)nitem * RG : -1;
+    };
     while (item < p.n_items && !failed) {
       const int64_t r0 = (int64_t)item * RG, r1 = (r0 + RG < p.M) ? r0 + RG : p.M;
       for (int64_t t = r0; t < r1; ++t, ++it) {
-        const int buf = it & 1;
+        const int buf = dbl ? (it & 1) : 0;
+        const uint32_t parity = dbl ? (uint32_t)(it >> 1) & 1u : (uint32_t)it & 1u;
         bool issued = false;
-        if (leader) {
-          int64_t next = -1;
-          if (t + 1 < r1) {
-            next = t + 1;
-          } else {
-            const int nitem = atomicAdd(p.counter, 1);
-            slot[(done + 1) & 1] = nitem;
-            if (nitem < p.n_items) next = (int64_t)nitem * RG;
-          }
+        if (leader && dbl) {
+          const int64_t next = next_row(t, r1);
           if (next >= 0) {
             issued = true;
             mbar_arrive_expect_tx(&mbar[buf ^ 1], row_bytes);
             bulk_g2s(stage + (buf ^ 1) * p.stage_bytes, p.x + (size_t)next * row_bytes, row_bytes, &mbar[buf ^ 1]);
           }
         }
-        const bool ok = mbar_wait(&mbar[buf], (uint32_t)(it >> 1) & 1u, p.err);
+        const bool ok = mbar_wait(&mbar[buf], parity, p.err);
         const uint32_t sa = stage_addr0 + (uint32_t)(buf * p.stage_bytes);
         float D2[MT2][4][4];
         float zc[32];
@@ -239,6 +252,14 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
           if (issued) mbar_wait(&mbar[buf ^ 1], (uint32_t)((it + 1) >> 1) & 1u, p.err);
           failed = true;
           break;
+        }
+        if (leader && !dbl) {
+          // every warp of the team is past its gather: the buffer is free
+          const int64_t next = next_row(t, r1);
+          if (next >= 0) {
+            mbar_arrive_expect_tx(&mbar[0], row_bytes);
+            bulk_g2s(stage, p.x + (size_t)next * row_bytes, row_bytes, &mbar[0]);
+          }
         }
         float s2 = 0.f;
         for (int v = 0; v < p.nw; ++v) s2 += red[buf * 32 + v];
@@ -392,17 +413,29 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
   }
 }
 
-size_t smem_bytes(int A, bool cc, int nb, int nw, int teams, int stage_bytes, int* prod_off) {
-  const int off = OS * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
+size_t smem_bytes(int A, bool cc, int nb, int nw, int teams, int stage_bytes, int os, int row_bufs, int* prod_off) {
+  const int off = os * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
   const int team_threads = nw * 32;
   const int gtab_off = (8 * nb + 15) & ~15;
   const int teams_off = (gtab_off + 2 * A * team_threads + 127) & ~127;
   if (prod_off) *prod_off = off;
   return 1024 + (size_t)off + teams_off + (size_t)teams * (TEAM_HDR + (cc ? (size_t)nw * 4096 : 0) +
-                                                           2 * (size_t)stage_bytes);
+                                                           (size_t)row_bufs * (size_t)stage_bytes);
 }
 
 }  // namespace
+
+// Gather table of the producers' CUDA-core block transform (h = 1024): entry
+// (w * 32 + lane) * 32 + a is the byte offset (2 x the input channel) of
+// in-block position 32 a + lane of block w, the order in which a lane gathers
+// its column.
+void rqcc_build_gather(int d, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather) {
+  gather.assign((size_t)d, 0);
+  for (int w = 0; w < d / 1024; ++w)
+    for (int lane = 0; lane < 32; ++lane)
+      for (int a = 0; a < 32; ++a)
+        gather[((size_t)w * 32 + lane) * 32 + a] = (uint16_t)(2 * perm[(size_t)w * 1024 + 32 * a + lane]);
+}
 
 size_t fused_flag_bytes(int64_t T) { return (size_t)((T + RG - 1) / RG + 64) * sizeof(int); }
 
@@ -412,7 +445,7 @@ bool fused_kernel_supported(const RQArgs& a, int N) {
   if (GEMM_WARPS + nw > MAX_WARPS) return false;
   const int stage_bytes = (a.d * 2 + 127) & ~127;
   const int nb = a.bins_full ? a.nb_full : a.nb;
-  return smem_bytes(A, A == 32 && a.gather_cc, nb, nw, 1, stage_bytes, nullptr) <= 227 * 1024;
+  return smem_bytes(A, A == 32 && a.gather_cc, nb, nw, 1, stage_bytes, 3, 1, nullptr) <= 227 * 1024;
 }
 
 oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream) {
@@ -452,10 +485,12 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* str
   auto kern = cc ? fused_kernel<32, true> : (A == 32 ? fused_kernel<32, false> : fused_kernel<16, false>);
   // as many teams as the warp budget, shared memory and the SM's registers
   // allow (the occupancy query says whether one CTA of that shape fits)
+  kp.os = kStages;
+  kp.row_bufs = kRowBuffers;
   int teams = (MAX_WARPS - GEMM_WARPS) / kp.nw;
   size_t smem = 0;
   for (; teams >= 1; --teams) {
-    smem = smem_bytes(A, cc, kp.nb, kp.nw, teams, kp.stage_bytes, &kp.prod_off);
+    smem = smem_bytes(A, cc, kp.nb, kp.nw, teams, kp.stage_bytes, kp.os, kp.row_bufs, &kp.prod_off);
     if (smem > 227 * 1024) continue;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) continue;
     int per_sm = 0;

@@ -101,7 +101,7 @@ oq_status rq_launch(const RQArgs& a, void* stream);
 // rotate-quantize with the block FWHT on the tensor cores (h = 1024 or 512,
 // bf16 input, fp16-level output, no signs; oq_rotate_quantize_tc.cu)
 void rqtc_build_gather(int d, int h, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather);
-// the same for the CUDA-core block transform (h = 1024; rqcc_kernel and the fused kernel)
+// the same for the fused kernel's CUDA-core block transform (h = 1024; oq_fused.cu)
 void rqcc_build_gather(int d, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather);
 bool rqtc_supported(const RQArgs& a);
 oq_status rqtc_launch(const RQArgs& a, void* stream);

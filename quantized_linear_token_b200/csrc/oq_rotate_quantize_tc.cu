@@ -32,7 +32,6 @@
 
 #include "oq_internal.h"
 #include "oq_ptx.cuh"
-#include "oq_rqcc_dev.cuh"
 #include "oq_rqtc_dev.cuh"
 
 namespace oq {
@@ -193,115 +192,7 @@ __global__ void __launch_bounds__(A == 32 ? 256 : 1024) rqtc_kernel(const __grid
   }
 }
 
-// The same contract with the block transform on the CUDA cores (h = 1024,
-// oq_rqcc_dev.cuh): lane l of a block's warp gathers column l of the 32 x 32
-// block matrix, and after the two in-register passes holds the block's 32
-// consecutive positions 32 l .. 32 l + 31, which it quantizes and stores as
-// one group (64 bytes of fp16 levels, or 4 b bytes of codes).
-__global__ void __launch_bounds__(256) rqcc_kernel(const __grid_constant__ TCParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int nw = p.nw, nthreads = nw * 32;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  // shared memory: mbarriers | norm partials [2][32] | threshold table |
-  // gather offsets [4][threads] (uint4) | per-warp 32 x 32 fp32 tiles | two row buffers
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem);
-  float* red = reinterpret_cast<float*>(smem + 16);
-  uint2* tbl = reinterpret_cast<uint2*>(smem + 272);
-  const int gtab_off = (272 + 8 * p.nb + 15) & ~15;
-  uint4* gtab = reinterpret_cast<uint4*>(smem + gtab_off);
-  const int tiles_off = (gtab_off + 64 * nthreads + 127) & ~127;
-  float* tile = reinterpret_cast<float*>(smem + tiles_off + warp * 4096);
-  unsigned char* stage = smem + tiles_off + nw * 4096;
-  const uint32_t stage_addr0 = smem_u32(stage);
-
-  for (int i = tid; i < 4 * nthreads; i += nthreads) {
-    const int t = i % nthreads, qq = i / nthreads;
-    gtab[i] = __ldg(reinterpret_cast<const uint4*>(p.gather) + (size_t)t * 4 + qq);
-  }
-  for (int i = tid; i < p.nb; i += nthreads) tbl[i] = __ldg(p.bins + i);
-  if (tid == 0) {
-    mbar_init(&mbar[0], 1);
-    mbar_init(&mbar[1], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  const uint32_t row_bytes = (uint32_t)p.d * 2u;
-  const unsigned char* src = static_cast<const unsigned char*>(p.src);
-  const float magic = 12582912.0f + (float)p.b0;
-  const int bin_lo = 0x4B400000, bin_hi = 0x4B400000 + p.nb - 1;
-  const uint32_t tbl_shift = smem_u32(tbl) - 0x4B400000u * 8u;
-  if (tid == 0 && (int64_t)blockIdx.x < p.rows) {
-    mbar_arrive_expect_tx(&mbar[0], row_bytes);
-    bulk_g2s(stage, src + (size_t)blockIdx.x * row_bytes, row_bytes, &mbar[0]);
-  }
-
-  int it = 0;
-  for (int64_t t = blockIdx.x; t < p.rows; t += gridDim.x, ++it) {
-    const int buf = it & 1;
-    bool issued = false;
-    if (tid == 0) {
-      const int64_t tn = t + gridDim.x;
-      if (tn < p.rows) {
-        issued = true;
-        mbar_arrive_expect_tx(&mbar[buf ^ 1], row_bytes);
-        bulk_g2s(stage + (buf ^ 1) * p.stage_bytes, src + (size_t)tn * row_bytes, row_bytes, &mbar[buf ^ 1]);
-      }
-    }
-    const bool ok = mbar_wait(&mbar[buf], (uint32_t)(it >> 1) & 1u, p.err);
-    const uint32_t sa = stage_addr0 + (uint32_t)(buf * p.stage_bytes);
-    float z[32];
-    const float ss = rqcc::transform_block(gtab, nthreads, tid, sa, tile, lane, z);
-    if (lane == 0) red[buf * 32 + warp] = ss;
-    const int failed = __syncthreads_or(!ok);
-    if (failed) {
-      if (issued) mbar_wait(&mbar[buf ^ 1], (uint32_t)((it + 1) >> 1) & 1u, p.err);
-      break;
-    }
-    float s2 = 0.f;
-    for (int w = 0; w < nw; ++w) s2 += red[buf * 32 + w];
-    const float s = sqrtf(s2);
-    const float ks = (s > 0.f) ? p.kscale / s : 0.f;
-    const bool unclamped = p.full && s2 >= 1e-30f && s2 <= 1e30f;
-    const size_t grp = (size_t)warp * 32 + lane;   // this lane's code group in the row
-    if (p.codes) {
-      uint32_t* out = p.codes + (size_t)t * ((size_t)p.d * p.bits / 32) + grp * p.bits;
-#define OQ_CC_CODES(B)                                                                            \
-  if (unclamped)                                                                                  \
-    rqcc::quantize_codes<false, B>(z, ks, magic, bin_lo, bin_hi, tbl_shift, out);                 \
-  else                                                                                            \
-    rqcc::quantize_codes<true, B>(z, ks, magic, bin_lo, bin_hi, tbl_shift, out);
-      switch (p.bits) {
-        case 2: OQ_CC_CODES(2) break;
-        case 3: OQ_CC_CODES(3) break;
-        case 4: OQ_CC_CODES(4) break;
-        default: OQ_CC_CODES(8) break;
-      }
-#undef OQ_CC_CODES
-    } else {
-      uint16_t* out = p.out16 + (size_t)t * p.d + grp * 32;
-      if (unclamped)
-        rqcc::quantize_levels<false>(z, ks, magic, bin_lo, bin_hi, tbl_shift, out);
-      else
-        rqcc::quantize_levels<true>(z, ks, magic, bin_lo, bin_hi, tbl_shift, out);
-    }
-    if (tid == 0) p.norms[t] = s;
-  }
-}
-
 }  // namespace
-
-// Gather table of the CUDA-core kernel (h = 1024): entry (w * 32 + lane) * 32
-// + a is the byte offset (2 x the input channel) of in-block position
-// 32 a + lane of block w, the order in which a lane gathers its column.
-void rqcc_build_gather(int d, const std::vector<uint32_t>& perm, std::vector<uint16_t>& gather) {
-  gather.assign((size_t)d, 0);
-  for (int w = 0; w < d / 1024; ++w)
-    for (int lane = 0; lane < 32; ++lane)
-      for (int a = 0; a < 32; ++a)
-        gather[((size_t)w * 32 + lane) * 32 + a] = (uint16_t)(2 * perm[(size_t)w * 1024 + 32 * a + lane]);
-}
 
 bool rqtc_supported(const RQArgs& a) {
   return (a.out16 || (a.codes && (a.bits == 2 || a.bits == 3 || a.bits == 4 || a.bits == 8))) &&
@@ -339,35 +230,6 @@ static oq_status rqtc_launch_t(const TCParams& p, void* stream) {
   return OQ_OK;
 }
 
-static oq_status rqcc_launch(const TCParams& p, void* stream) {
-  const int threads = p.nw * 32;
-  const size_t gtab_off = (272 + 8 * (size_t)p.nb + 15) & ~(size_t)15;
-  const size_t smem = ((gtab_off + 64 * (size_t)threads + 127) & ~(size_t)127) + (size_t)p.nw * 4096 +
-                      2 * (size_t)p.stage_bytes;
-  if (smem > 227 * 1024) return OQ_ERR_UNSUPPORTED;
-  cudaError_t e = cudaFuncSetAttribute(rqcc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(rqcc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) {
-    set_error(std::string("cudaFuncSetAttribute: ") + cudaGetErrorString(e));
-    return OQ_ERR_CUDA;
-  }
-  int dev = 0, sms = 0, per_sm = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rqcc_kernel, threads, smem);
-  if (per_sm < 1) per_sm = 1;
-  const int64_t grid = std::min<int64_t>(p.rows, (int64_t)sms * per_sm);
-  rqcc_kernel<<<(unsigned)grid, threads, smem, static_cast<cudaStream_t>(stream)>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    set_error(std::string("rotate_quantize (CUDA-core FWHT) launch: ") + cudaGetErrorString(e));
-    return OQ_ERR_CUDA;
-  }
-  return OQ_OK;
-}
-
 oq_status rqtc_launch(const RQArgs& a, void* stream) {
   if (a.rows == 0) return OQ_OK;
   if (!rqtc_supported(a)) return OQ_ERR_UNSUPPORTED;
@@ -395,10 +257,6 @@ oq_status rqtc_launch(const RQArgs& a, void* stream) {
     p.b0 = a.b0;
   }
   p.kscale = a.kscale;
-  if (a.h == 1024 && a.gather_cc) {
-    p.gather = a.gather_cc;
-    return rqcc_launch(p, stream);
-  }
   return a.h == 1024 ? rqtc_launch_t<32>(p, stream) : rqtc_launch_t<16>(p, stream);
 }
 
