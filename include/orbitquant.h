@@ -259,8 +259,16 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
  * size: 2 T d_in bytes rounded up to a multiple of 256, plus 4 T, on the
  * fp16-level route) is accepted and decodes the weights inside the
  * contraction instead; the y values are the same up to fp32 summation
- * order.  Errors: OQ_ERR_INVALID_ARG when the workspace is below that least
- * size.
+ * order.  On the fp16-level route the workspace starts with the A operand
+ * (fp16 levels [T, d_in] as oq_rotate_quantize_levels writes them, 2 T d_in
+ * bytes rounded up to a multiple of 256) followed by the norms s [T] fp32:
+ * after the call they hold the codes' levels and norms that gave y.  Where
+ * the fused kernel runs with the block transform on the CUDA cores (h =
+ * 1024), its fp32 rounding differs from oq_rotate_quantize_levels', so a code
+ * may differ from that call's where the coordinate lies within rounding of a
+ * decision threshold, and s in the last bits; y is then oq_linear_decoded's
+ * on the workspace's operands, bit for bit.  Errors: OQ_ERR_INVALID_ARG when
+ * the workspace is below that least size.
  */
 size_t oq_linear_fused_workspace_size(const oq_layer* layer, int64_t T);
 oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype, int64_t T,
@@ -335,8 +343,12 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  * flag, while its contraction warps load a tile's rows as soon as their
  * groups are published (gecl notes Method 2: the codes of R x meet the
  * pre-rotated weight codes in one pass).  Elsewhere the rotate-quantize
- * kernel and oq_linear_decoded's kernel run in turn.  Either way y is that of
- * oq_rotate_quantize_levels + oq_linear_decoded, bit for bit.
+ * kernel and oq_linear_decoded's kernel run in turn.  The workspace then holds
+ * the A operand and the norms as for oq_linear_fused, and y is that of
+ * oq_linear_decoded on them, bit for bit (and that of
+ * oq_rotate_quantize_levels + oq_linear_decoded where the transform is the
+ * same: every case but h = 1024 inside the fused kernel, see
+ * oq_linear_fused).
  *   x          device [T, d_in] bf16 (else OQ_ERR_UNSUPPORTED).
  *   w16        device [d_out, d_in] fp16 levels, 16-byte aligned.
  *   r          device [d_out] fp32, 16-byte aligned.

@@ -479,7 +479,7 @@ static size_t fused_w16_bytes(const oq_layer* L) { return round256((size_t)L->d_
 // the workspace of the large-batch route: the least workspace, the fused
 // kernel's row-group flags, and the decoded weights
 static size_t full_workspace(const oq_layer* L, int64_t T, size_t base) {
-  return round256(base) + round256(fused_flag_bytes(T)) + fused_w16_bytes(L);
+  return round256(base) + round256(fused_flag_bytes(T, L->d_out)) + fused_w16_bytes(L);
 }
 
 // the least workspace oq_linear_fused accepts (without the decoded weights)
@@ -492,7 +492,7 @@ static size_t min_workspace(const oq_layer* L, int64_t T) {
 
 // the workspace of oq_linear_fused_decoded: the least workspace and the flags
 static size_t decoded_workspace(const oq_layer* L, int64_t T) {
-  return round256(min_workspace(L, T)) + round256(fused_flag_bytes(T));
+  return round256(min_workspace(L, T)) + round256(fused_flag_bytes(T, L->d_out));
 }
 
 size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
@@ -653,8 +653,11 @@ static oq_status int4_linear(const oq_layer* L, const void* x, int32_t x_dtype, 
 // x -> y with the weights' fp16 levels already decoded: the fused kernel
 // where it applies, else the rotate-quantize kernel and the decoded-weight
 // contraction in turn.  ws: [A operand | norms | row-group flags].
-static oq_status fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint16_t* w16,
-                               const float* r, void* y, bool y_bf16, unsigned char* ws, void* stream) {
+// Wcodes: the weight codes, decoded into w16 here (by the fused kernel's own
+// producers where it runs, else by the level kernel first), or null when w16
+// already holds their levels.
+static oq_status fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
+                               uint16_t* w16, const float* r, void* y, bool y_bf16, unsigned char* ws, void* stream) {
   if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
   const size_t need = min_workspace(L, T);
   uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
@@ -662,10 +665,16 @@ static oq_status fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype
   const RQArgs ra = rq_levels_args(L, x, x_dtype, T, a16, s);
   if (fused_kernel_supported(ra, L->d_out)) {
     int* flags = reinterpret_cast<int*>(ws + round256(need));
-    const oq_status st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), flags, stream);
+    const oq_status st =
+        fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), Wcodes, L->lv_w, flags, stream);
     if (st != OQ_ERR_UNSUPPORTED) return st;
   }
-  const oq_status st = rq_levels(L, x, x_dtype, T, a16, s, stream);
+  oq_status st = OQ_OK;
+  if (Wcodes) {
+    st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
+    if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_fused: unsupported shape") : st;
+  }
+  st = rq_levels(L, x, x_dtype, T, a16, s, stream);
   return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16, r, y, y_bf16, stream);
 }
 
@@ -691,9 +700,7 @@ static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype,
     if (fused_w16_route(L, x_dtype, T) && workspace_bytes >= full_workspace(L, T, need)) {
       // workspace: [A operand | norms | row-group flags | decoded weights]
       uint16_t* w16 = reinterpret_cast<uint16_t*>(ws + decoded_workspace(L, T));
-      st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
-      if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_fused: unsupported shape") : st;
-      return fused_decoded(L, x, x_dtype, T, w16, r, y, y_bf16, ws, stream);
+      return fused_decoded(L, x, x_dtype, T, Wcodes, w16, r, y, y_bf16, ws, stream);
     }
     st = rq_levels(L, x, x_dtype, T, a16, s, stream);
     if (st != OQ_OK) return st;
@@ -756,8 +763,8 @@ oq_status oq_linear_fused_decoded(const oq_layer* L, const void* x, int32_t x_dt
   if (!aligned(w16, 16)) return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused_decoded: w16 must be 16-byte aligned");
   if (workspace_bytes < decoded_workspace(L, T))
     return fail(OQ_ERR_INVALID_ARG, "oq_linear_fused_decoded: workspace too small");
-  return fused_decoded(L, x, x_dtype, T, w16, r, y, y_dtype == OQ_DTYPE_BF16, static_cast<unsigned char*>(workspace),
-                       stream);
+  return fused_decoded(L, x, x_dtype, T, nullptr, const_cast<uint16_t*>(w16), r, y, y_dtype == OQ_DTYPE_BF16,
+                       static_cast<unsigned char*>(workspace), stream);
 }
 
 oq_status oq_poll_error(const oq_layer* L) {

@@ -1,13 +1,13 @@
 """GPU parity at the workloads' full sizes, in the launch configuration the
-benchmark times (one oq_linear_fused call with the workspace it asks for: the
-rotate-quantize kernel writes the fp16 levels of the activation codes, the
-weight codes are decoded once into fp16 levels, and the two operands are
-contracted on CTA pairs).  Needs a B200.
+benchmark times: one oq_linear_fused call with the workspace it asks for
+(the weight codes decoded once into fp16 levels, then the fused kernel --
+rotate-quantize producer warps inside the CTA-pair contraction -- where the
+block size allows, else the rotate-quantize kernel and the contraction in
+turn).  Needs a B200.
 
-For every case:
-* the fused call's y equals, bit for bit, the y of its three stage calls
-  (oq_rotate_quantize_levels, oq_weight_levels, oq_linear_decoded), whose
-  intermediate operands are then checked;
+For every case, on the call's own operands (its workspace starts with the A
+operand and the norms that gave y):
+* y is the decoded-weight contraction of those operands, bit for bit;
 * every activation code (read back from the fp16 A operand) and every norm
   against the fp64 oracle, with the bounds of tests/parity.py (codes exact
   outside a band of 1e-5/sqrt(d) around each threshold, excused mismatches
@@ -90,14 +90,20 @@ def test_full_size_parity(env, pool, wl_key, layer_name, T, gelu, stream):
     Wm = W.weights(wl, lay)
     layer = B.oq_layer_create(d, dout, W.ROTATION_SEED, lay.a_bits, lay.w_bits)
     Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(Wm).cuda())
-    y = B.oq_linear_fused(layer, x_t, Wc, r)
-    a16, s = B.oq_rotate_quantize_levels(layer, x_t)
+    # the benchmarked call, with its own workspace: it starts with the call's A
+    # operand (fp16 levels [T, d], rounded up to 256 bytes) and its norms
+    ws = torch.empty((B.oq_linear_fused_workspace_size(layer, T),), dtype=torch.uint8, device="cuda")
+    y = B.oq_linear_fused(layer, x_t, Wc, r, workspace=ws)
+    a_bytes = (T * d * 2 + 255) // 256 * 256
+    a16 = ws[:T * d * 2].view(torch.float16).view(T, d)
+    s = ws[a_bytes:a_bytes + 4 * T].view(torch.float32)
     w16 = B.oq_weight_levels(layer, Wc)
+    # y is the decoded-weight contraction of those operands, bit for bit
     y2 = B.oq_linear_decoded(layer, a16, s, w16, r)
     torch.cuda.synchronize()
     B.oq_poll_error(layer)
     del x_t
-    assert torch.equal(y.view(torch.int32), y2.view(torch.int32)), "fused call differs from its stage calls"
+    assert torch.equal(y.view(torch.int32), y2.view(torch.int32)), "fused y differs from its operands' contraction"
     del y2
 
     cb_a, cb_w = O.lloyd_max(d, lay.a_bits), O.lloyd_max(d, lay.w_bits)
