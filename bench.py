@@ -346,7 +346,8 @@ def run_ours(args):
     # and the contraction where the block size is 1024 or 512 with at most 12
     # warps per token row (bf16 x, no Rademacher signs)
     h_blk = d & -d
-    fused_kernel = decoded and ((h_blk == 1024 and d // h_blk <= 8) or (h_blk == 512 and d // h_blk <= 12))
+    fused_kernel = decoded and dout <= d and ((h_blk == 1024 and d // h_blk <= 8) or
+                                                (h_blk == 512 and d // h_blk <= 12))
     stages = {
         # the stages of oq_linear_fused at this batch size: where the fused
         # kernel runs, the call is that one kernel (it decodes the weights too)
@@ -726,7 +727,8 @@ def run_sweep(args):
                 stages += [("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]
             runs = {"step": [("step", lambda: B.oq_linear_fused(layer, x, Wc, r, y, ws))], "stages": stages}
             h_blk = d & -d
-            fused_kernel = decoded and ((h_blk == 1024 and d // h_blk <= 8) or (h_blk == 512 and d // h_blk <= 12))
+            fused_kernel = decoded and dout <= d and ((h_blk == 1024 and d // h_blk <= 8) or
+                                                (h_blk == 512 and d // h_blk <= 12))
             times = {}
             for name, st in runs.items():
                 for _ in range(warm):

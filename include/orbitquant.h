@@ -337,7 +337,9 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  * already decoded (w16 from oq_weight_levels, kept by the caller across
  * calls or decoded just before): the large-batch route of oq_linear_fused
  * without its first step.  Where the block size is 1024 or 512 (at most 12
- * warps per token row) one kernel rotates, quantizes and contracts: its
+ * warps per token row) and d_out <= d_in (where rotate-quantize is a share of
+ * the work large enough for the overlap to pay) one kernel rotates, quantizes
+ * and contracts: its
  * rotate-quantize warps claim groups of 4 token rows from a queue, write
  * their fp16 levels and norms to the workspace and publish each group with a
  * flag, while its contraction warps load a tile's rows as soon as their

@@ -479,7 +479,7 @@ static size_t fused_w16_bytes(const oq_layer* L) { return round256((size_t)L->d_
 // the workspace of the large-batch route: the least workspace, the fused
 // kernel's row-group flags, and the decoded weights
 static size_t full_workspace(const oq_layer* L, int64_t T, size_t base) {
-  return round256(base) + round256(fused_flag_bytes(T, L->d_out)) + fused_w16_bytes(L);
+  return round256(base) + round256(fused_flag_bytes(T)) + fused_w16_bytes(L);
 }
 
 // the least workspace oq_linear_fused accepts (without the decoded weights)
@@ -492,7 +492,7 @@ static size_t min_workspace(const oq_layer* L, int64_t T) {
 
 // the workspace of oq_linear_fused_decoded: the least workspace and the flags
 static size_t decoded_workspace(const oq_layer* L, int64_t T) {
-  return round256(min_workspace(L, T)) + round256(fused_flag_bytes(T, L->d_out));
+  return round256(min_workspace(L, T)) + round256(fused_flag_bytes(T));
 }
 
 size_t oq_linear_fused_workspace_size(const oq_layer* L, int64_t T) {
@@ -653,9 +653,15 @@ static oq_status int4_linear(const oq_layer* L, const void* x, int32_t x_dtype, 
 // x -> y with the weights' fp16 levels already decoded: the fused kernel
 // where it applies, else the rotate-quantize kernel and the decoded-weight
 // contraction in turn.  ws: [A operand | norms | row-group flags].
-// Wcodes: the weight codes, decoded into w16 here (by the fused kernel's own
-// producers where it runs, else by the level kernel first), or null when w16
-// already holds their levels.
+// Wcodes: the weight codes, decoded into w16 here first by the level kernel,
+// or null when w16 already holds their levels.
+// The fused kernel pays where rotate-quantize is a large share of the layer's
+// work: the contraction's work per token row grows with d_out, the producers'
+// with d_in.  (Measured: with d_out = d_in, 3-6 % below the two kernels in
+// turn; with d_out = 4 d_in, 16 % above them, the producers' warps and shared
+// memory slowing a contraction that runs long after they are done.)
+static bool fused_kernel_pays(const oq_layer* L) { return L->d_out <= L->d_in; }
+
 static oq_status fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
                                uint16_t* w16, const float* r, void* y, bool y_bf16, unsigned char* ws, void* stream) {
   if (T > MAX_TOKENS) return fail(OQ_ERR_UNSUPPORTED, "batch too large: at most 2^31 - 1024 tokens per call");
@@ -663,16 +669,15 @@ static oq_status fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype
   uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
   float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
   const RQArgs ra = rq_levels_args(L, x, x_dtype, T, a16, s);
-  if (fused_kernel_supported(ra, L->d_out)) {
-    int* flags = reinterpret_cast<int*>(ws + round256(need));
-    const oq_status st =
-        fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), Wcodes, L->lv_w, flags, stream);
-    if (st != OQ_ERR_UNSUPPORTED) return st;
-  }
   oq_status st = OQ_OK;
   if (Wcodes) {
     st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
     if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_fused: unsupported shape") : st;
+  }
+  if (fused_kernel_pays(L) && fused_kernel_supported(ra, L->d_out)) {
+    int* flags = reinterpret_cast<int*>(ws + round256(need));
+    st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), flags, stream);
+    if (st != OQ_ERR_UNSUPPORTED) return st;
   }
   st = rq_levels(L, x, x_dtype, T, a16, s, stream);
   return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16, r, y, y_bf16, stream);
@@ -689,10 +694,8 @@ static oq_status fused_device(const oq_layer* L, const void* x, int32_t x_dtype,
   if (fused_f16_route(L, x_dtype)) {
     uint16_t* a16 = reinterpret_cast<uint16_t*>(ws);
     float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
-    if (w16_ready) {
-      st = rq_levels(L, x, x_dtype, T, a16, s, stream);
-      return st != OQ_OK ? st : linear_w16(L, a16, s, T, w16_ready, r, y, y_bf16, stream);
-    }
+    if (w16_ready)   // the same kernels as the one-call route, weights given
+      return fused_decoded(L, x, x_dtype, T, nullptr, const_cast<uint16_t*>(w16_ready), r, y, y_bf16, ws, stream);
     // large batches with room for the decoded weights: decode them once, then
     // contract two fp16 operands -- in the fused kernel, whose producer teams
     // write the A operand while the contraction runs, where it applies;
@@ -794,6 +797,7 @@ oq_status oq_check_wait_timeout(const oq_layer* L, uint32_t limit_us, void* stre
 namespace oq {
 size_t fused_min_workspace(const oq_layer* L, int64_t T) { return min_workspace(L, T); }
 size_t fused_w16_workspace(const oq_layer* L, int64_t T) { return full_workspace(L, T, min_workspace(L, T)); }
+size_t fused_decoded_min_workspace(const oq_layer* L, int64_t T) { return decoded_workspace(L, T); }
 bool fused_decodes_weights(const oq_layer* L, int32_t x_dtype, int64_t T) { return fused_w16_route(L, x_dtype, T); }
 oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
                            const float* r, const void* y, int32_t y_dtype, const void* workspace, const char* who) {

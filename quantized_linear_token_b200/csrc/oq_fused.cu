@@ -32,7 +32,6 @@
 #include <cstring>
 
 #include "oq_internal.h"
-#include "oq_decode.cuh"
 #include "oq_epilogue.cuh"
 #include "oq_ptx.cuh"
 #include "oq_rqcc_dev.cuh"
@@ -74,16 +73,8 @@ struct FusedParams {
   uint16_t* a16;             // fp16 levels [M, K]
   float* norms;              // [M]
   int* flags;                // [n_items]: 1 once the group's rows are written
-  int* counter;              // the queue's next item (weight groups first, then token groups)
+  int* counter;              // the queue's next group
   int n_items;               // ceil(M / RG)
-  // weight decode inside the kernel (or none: n_witems = 0, weights given)
-  const uint32_t* wcodes;    // weight codes [N, K * w_bits / 32]
-  uint4* w16out;             // their fp16 levels [N, K] (the B operand)
-  int* wflags;               // [n_witems]: 1 once the group's rows are decoded
-  int n_witems;              // N / RWI
-  int w_bits;
-  uint32_t wtab[4];          // byte-permute decode tables of the weight codebook
-  DecK kc;
   const uint16_t* gather;    // tensor-core gather table (kernel order)
   const uint2* bins;         // {threshold bits, fp16 level pair}
   int nb, b0, full;
@@ -96,7 +87,6 @@ struct FusedParams {
 };
 
 constexpr int RG = 4;              // token rows per queue group: 32 groups per 128-row tile
-constexpr int RWI = 4;             // weight rows per queue group: 32 groups per 128-row B tile
 // the contraction's operand stages and the producer teams' staged rows: the
 // shared memory left by the stages holds the teams, so these trade the
 // contraction's latency cover against the number of producer warps
@@ -211,45 +201,17 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
     const uint32_t tbl_shift = smem_u32(tbl) - 0x4B400000u * 8u;
     const int g = lane >> 2, q = lane & 3;
 
-    int done = 0;
-    if (leader) slot[0] = atomicAdd(p.counter, 1);
+    if (leader) {
+      const int item = atomicAdd(p.counter, 1);
+      slot[0] = item;
+      if (item < p.n_items) {
+        mbar_arrive_expect_tx(&mbar[0], row_bytes);
+        bulk_g2s(stage, p.x + (size_t)item * RG * row_bytes, row_bytes, &mbar[0]);
+      }
+    }
     named_bar_sync(bar_id, team_threads);
     int item = slot[0];
-    // ---- weight groups (queue items 0 .. n_witems - 1): RWI rows of codes
-    // decoded into their fp16 levels, 8 values per thread and step
-    while (item < p.n_witems) {
-      const int64_t cpr = p.K / 8;                              // 8-value chunks per row
-      const int64_t c0 = (int64_t)item * RWI * cpr, c1 = c0 + RWI * cpr;
-      for (int64_t i = c0 + ttid; i < c1; i += team_threads) {
-        uint4 v, o;
-        if (p.w_bits == 4) {
-          v = __ldg(reinterpret_cast<const uint4*>(p.wcodes) + i / 4);
-          o = decode_chunk_k<4>(v, (int)(i % 4), p.wtab, nullptr, p.kc);
-        } else if (p.w_bits == 2) {
-          v = __ldg(reinterpret_cast<const uint4*>(p.wcodes) + i / 8);
-          o = decode_chunk_k<2>(v, (int)(i % 8), p.wtab, nullptr, p.kc);
-        } else {
-          const uint32_t* pw = p.wcodes + (i / 4) * 3;
-          v = make_uint4(__ldg(pw), __ldg(pw + 1), __ldg(pw + 2), 0u);
-          o = decode_chunk_k<3>(v, (int)(i % 4), p.wtab, nullptr, p.kc);
-        }
-        p.w16out[i] = o;
-      }
-      fence_proxy_async_global();
-      __threadfence();
-      if (leader) slot[(done + 1) & 1] = atomicAdd(p.counter, 1);
-      named_bar_sync(bar_id, team_threads);
-      if (leader) st_release_gpu(p.wflags + item, 1);
-      ++done;
-      item = slot[done & 1];
-    }
-    // ---- token groups (queue items n_witems ..): item is now a token group
-    item -= p.n_witems;
-    if (leader && item < p.n_items) {
-      mbar_arrive_expect_tx(&mbar[0], row_bytes);
-      bulk_g2s(stage, p.x + (size_t)item * RG * row_bytes, row_bytes, &mbar[0]);
-    }
-    int it = 0;
+    int it = 0, done = 0;
     bool failed = false;
     // two row buffers: the next row's copy starts with this row; one: it
     // starts once every warp of the team has gathered this row
@@ -258,7 +220,7 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
     // claimed group (whose index the team reads from slot after the group)
     auto next_row = [&](int64_t t, int64_t r1) -> int64_t {
       if (t + 1 < r1) return t + 1;
-      const int nitem = atomicAdd(p.counter, 1) - p.n_witems;
+      const int nitem = atomicAdd(p.counter, 1);
       slot[(done + 1) & 1] = nitem;
       return nitem < p.n_items ? (int64_t)nitem * RG : -1;
     };
@@ -343,8 +305,6 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
       const int first = (int)(m0 / RG);
       const int left = p.n_items - first, cnt = left < 0 ? 0 : (left < RM / RG ? left : RM / RG);
       ok = wait_flags(p.flags + first, cnt, lane, p.err);
-      // and this CTA's 128 B rows, where the kernel decodes the weights
-      if (ok && p.n_witems) ok = wait_flags(p.wflags + n0 / RWI, RN / RWI, lane, p.err);
       if (!ok) break;
       if (lane == 0) {
         fence_proxy_async_global();
@@ -477,9 +437,7 @@ void rqcc_build_gather(int d, const std::vector<uint32_t>& perm, std::vector<uin
         gather[((size_t)w * 32 + lane) * 32 + a] = (uint16_t)(2 * perm[(size_t)w * 1024 + 32 * a + lane]);
 }
 
-size_t fused_flag_bytes(int64_t T, int N) {
-  return (size_t)((T + RG - 1) / RG + N / RWI + 64) * sizeof(int);
-}
+size_t fused_flag_bytes(int64_t T) { return (size_t)((T + RG - 1) / RG + 64) * sizeof(int); }
 
 bool fused_kernel_supported(const RQArgs& a, int N) {
   if (!rqtc_supported(a) || N % PN != 0 || a.d % 64 != 0) return false;
@@ -490,8 +448,7 @@ bool fused_kernel_supported(const RQArgs& a, int N) {
   return smem_bytes(A, A == 32 && a.gather_cc, nb, nw, 1, stage_bytes, 3, 1, nullptr) <= 227 * 1024;
 }
 
-oq_status fused_launch(const RQArgs& a, const GemmArgs& g, const uint32_t* wcodes, const uint16_t* w_levels_host,
-                       int* flags, void* stream) {
+oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream) {
   if (g.M == 0) return OQ_OK;
   if (!fused_kernel_supported(a, g.N) || !g.b_f16) return OQ_ERR_UNSUPPORTED;
   FusedParams kp;
@@ -508,17 +465,7 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, const uint32_t* wcode
   kp.norms = a.norms;
   kp.n_items = (int)((g.M + RG - 1) / RG);
   kp.flags = flags;
-  if (wcodes) {
-    // the kernel decodes the weights into g.b_f16 itself
-    kp.wcodes = wcodes;
-    kp.w16out = reinterpret_cast<uint4*>(const_cast<uint16_t*>(g.b_f16));
-    kp.n_witems = g.N / RWI;
-    kp.w_bits = g.b_bits;
-    make_decode_tables(g.b_bits, w_levels_host, kp.wtab);
-    kp.kc = make_deck();
-  }
-  kp.wflags = flags + kp.n_items;
-  kp.counter = flags + kp.n_items + kp.n_witems + 32;   // its own line, away from the flags
+  kp.counter = flags + kp.n_items + 32;   // its own line, away from the flags
   const bool cc = a.h == 1024 && a.gather_cc;
   kp.gather = cc ? a.gather_cc : a.gather_tc;
   if (a.bins_full) {
@@ -573,7 +520,7 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, const uint32_t* wcode
   const int grid = sms & ~1;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the flags and the queue counter start at zero on every call
-  e = cudaMemsetAsync(flags, 0, fused_flag_bytes(g.M, g.N), s);
+  e = cudaMemsetAsync(flags, 0, fused_flag_bytes(g.M), s);
   if (e != cudaSuccess) {
     set_error(std::string("clear fused flags: ") + cudaGetErrorString(e));
     return OQ_ERR_CUDA;

@@ -41,11 +41,13 @@ IoLayout io_layout(const oq_layer* L, int32_t x_dtype, int64_t T) {
   IoLayout o{};
   o.chunk = std::min<int64_t>(T, CHUNK);
   o.w16 = fused_decodes_weights(L, x_dtype, T);
-  // one chunk's fused workspace; with pre-decoded weights the chunk needs
-  // only the least workspace, and the weights sit after it
+  // one chunk's fused workspace; with pre-decoded weights the chunk needs its
+  // operand, norms and the fused kernel's flags, and the weights sit after it
   o.fused_bytes = r256(fused_min_workspace(L, o.chunk));
   size_t at = o.fused_bytes;
   if (o.w16) {
+    o.fused_bytes = r256(fused_decoded_min_workspace(L, o.chunk));
+    at = o.fused_bytes;
     o.w16_off = at;
     at += r256(fused_w16_workspace(L, o.chunk) - fused_min_workspace(L, o.chunk));
   } else if (o.chunk == T) {

@@ -154,20 +154,18 @@ oq_status gemm_w16_launch(const GemmArgs& g, void* stream);
 // the fused call decodes the weights once per call from this many tokens on
 constexpr int64_t W16_MIN_T = 1024;
 // the fused layer kernel (oq_fused.cu): rotate-quantize producer teams inside
-// the CTA-pair contraction of the decoded weights.  With wcodes the kernel's
-// producers first decode the weight codes into g.b_f16 (levels from
-// w_levels_host); without, g.b_f16 already holds them.  `flags` is workspace
-// of fused_flag_bytes(T, N) bytes (cleared by the launch itself).
+// the CTA-pair contraction of the decoded weights.  `flags` is zeroed
+// workspace of fused_flag_bytes(T) bytes (cleared by the launch itself).
 bool fused_kernel_supported(const RQArgs& a, int N);
-size_t fused_flag_bytes(int64_t T, int N);
-oq_status fused_launch(const RQArgs& a, const GemmArgs& g, const uint32_t* wcodes, const uint16_t* w_levels_host,
-                       int* flags, void* stream);
+size_t fused_flag_bytes(int64_t T);
+oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream);
 // the fused call's pieces for the host-buffer pipeline (oq_api.cu): the least
 // workspace; the workspace with the decoded weights after it; whether the
 // fused call decodes the weights once at this batch size; argument checks;
 // the call on checked arguments (w16_ready: weights already decoded, or null)
 size_t fused_min_workspace(const oq_layer* L, int64_t T);
 size_t fused_w16_workspace(const oq_layer* L, int64_t T);
+size_t fused_decoded_min_workspace(const oq_layer* L, int64_t T);   // operand, norms and fused-kernel flags
 bool fused_decodes_weights(const oq_layer* L, int32_t x_dtype, int64_t T);
 oq_status fused_check_args(const oq_layer* L, const void* x, int32_t x_dtype, int64_t T, const uint32_t* Wcodes,
                            const float* r, const void* y, int32_t y_dtype, const void* workspace, const char* who);

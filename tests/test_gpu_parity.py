@@ -127,7 +127,7 @@ def fused_kernel_cc(d_in, d_out, T, flags, x_bf16=True):
     on the CUDA cores (h = 1024), whose rounding differs from the stand-alone
     rotate-quantize kernel's."""
     h = d_in & -d_in
-    return (x_bf16 and d_out % 256 == 0 and T >= W16_MIN_T and h == 1024 and d_in // h <= 8
+    return (x_bf16 and d_out % 256 == 0 and d_out <= d_in and T >= W16_MIN_T and h == 1024 and d_in // h <= 8
             and not flags & 1)
 
 
