@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true",
                     help="the stress workload's sweep (every token count x every layer): one JSON line per point")
+    ap.add_argument("--sweep-small", default="1,8",
+                    help="batch sizes of the batch-1 / GEMV end added to the sweep (comma list, empty for none)")
     return ap.parse_args()
 
 
@@ -699,7 +701,8 @@ def run_sweep(args):
     B.load_library()
     peaks = load_peaks()
     wl = W.WORKLOADS["stress"]
-    sweep = wl.token_sweep
+    small = [int(v) for v in args.sweep_small.split(",") if v.strip()]
+    sweep = tuple(sorted(set(small) | set(wl.token_sweep)))
     d = wl.layers[0].d_in
     # the recipe does not depend on the batch size, so every smaller batch is
     # the first rows of the largest one
@@ -761,8 +764,9 @@ def run_sweep(args):
                            "x_bytes": T * d * 2,
                            "l2": "flushed (256 MiB write) before every step, outside the timed events",
                            "contraction": "decoded weights, both operands by TMA" if decoded else
-                           ("small-batch split-K kernel" if T <= 256 else "CTA pair, weights decoded in the GEMM")},
-                "roofline": {"kernel": "fused layer kernel (weight decode, rotate-quantize, contraction)"
+                           ("GEMV kernel (warp MMAs, weight codes decoded in registers)" if T <= 8 else
+                            "small-batch split-K kernel" if T <= 256 else "CTA pair, weights decoded in the GEMM")},
+                "roofline": {"kernel": "fused layer kernel (rotate-quantize and contraction)"
                              if fused_kernel else "contraction",
                              "bound": "tensor", "achieved": flops / (times[ck] * 1e-3) / 1e12,
                              "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -778,6 +782,18 @@ def run_sweep(args):
                 "step_tflops": flops / (times["step"] * 1e-3) / 1e12,
                 "step_frac": flops / (times["step"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
             }
+            if T <= 8:
+                # the batch-1 / GEMV end: the contraction streams the weight
+                # codes once; its floor is their bytes at HBM speed
+                gb = dout * d * lay.w_bits / 8 + T * d * 2 + dout * 4 + T * dout * 4
+                line["roofline_tensor"] = line["roofline"]
+                line["roofline"] = {
+                    "kernel": "small-batch contraction (warp MMAs, weight codes decoded in registers)",
+                    "bound": "hbm", "achieved": gb / (times["gemm"] * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": gb / (times["gemm"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                    "bytes_per_launch": gb, "ms_per_launch": times["gemm"],
+                    "floor_ms": gb / (peaks["hbm_gbs"] * 1e9) * 1e3,
+                    "bytes_rule": "weight codes + fp16 activation levels + r + fp32 y"}
             if decoded:
                 wb = dout * d * (lay.w_bits / 8 + 2)
                 line["roofline_weight_levels"] = {"bound": "hbm", "achieved": wb / (times["wlevels"] * 1e-3) / 1e9,
