@@ -351,11 +351,14 @@ def run_ours(args):
     fused_kernel = decoded and dout <= d and ((h_blk == 1024 and d // h_blk <= 8) or
                                                 (h_blk == 512 and d // h_blk <= 12))
     stages = {
-        # the stages of oq_linear_fused at this batch size: where the fused
-        # kernel runs, the call is that one kernel (it decodes the weights too)
-        "levels": ([("fused", lambda: B.oq_linear_fused(layer, x, Wc, r, y, ws))] if fused_kernel else
+        # the stages of oq_linear_fused at this batch size: the weight decode,
+        # then the fused kernel where it runs, else rotate-quantize and the
+        # contraction in turn
+        "levels": ([("wlevels", lambda: B.oq_weight_levels(layer, Wc, w16)),
+                    ("fused", lambda: B.oq_linear_fused_decoded(layer, x, w16, r, y, ws_fd))] if fused_kernel else
                    [("wlevels", lambda: B.oq_weight_levels(layer, Wc, w16)),
-                    ("gemm", lambda: B.oq_linear_fused_decoded(layer, x, w16, r, y, ws_fd))] if decoded else
+                    ("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s)),
+                    ("gemm", lambda: B.oq_linear_decoded(layer, a16, s, w16, r, y))] if decoded else
                    [("rq", lambda: B.oq_rotate_quantize_levels(layer, x, a16, s)),
                     ("gemm", lambda: B.oq_linear_levels(layer, a16, s, Wc, r, y))]),
         # the same route with rotate-quantize and the contraction as two kernels
@@ -512,9 +515,9 @@ def run_ours(args):
     gemm_tf = flops / (mm_ms * 1e-3) / 1e12
     rq_gbs = rq_bytes / (rq_ms * 1e-3) / 1e9
     gemm_desc = {
-        "fused": ("fused layer kernel: producer warps decode the weight codes and rotate-quantize the tokens "
-                  "(norm, gather, block FWHT on the CUDA cores, Lloyd-Max codes as fp16 levels) for the "
-                  "tcgen05 CTA-pair contraction, fp32 TMEM accumulate", "fused"),
+        "fused": ("fused layer kernel: producer warps rotate-quantize the tokens (norm, gather, block FWHT on "
+                  "the CUDA cores, Lloyd-Max codes as fp16 levels) for the tcgen05 CTA-pair contraction of the "
+                  "decoded weights, fp32 TMEM accumulate", "fused"),
         "decoded": ("codebook GEMM on fp16 levels of both operands, both by TMA "
                     "(tcgen05 CTA pair, fp32 TMEM accumulate)", "gemm_decoded"),
         "levels_wdec": ("codebook GEMM, fp16 A operand by TMA, weight codes decoded to fp16 in shared memory "
@@ -529,8 +532,8 @@ def run_ours(args):
         "codes": "rotate + quantize (norm, gather, block FWHT, Lloyd-Max codes, pack)",
     }
     steps_desc = {
-        "levels": ("oq_linear_fused (one kernel: weight decode, rotate-quantize and contraction)" if fused_kernel
-                   else "oq_weight_levels + oq_linear_fused_decoded" if decoded else
+        "levels": ("oq_weight_levels + oq_linear_fused_decoded (the fused kernel)" if fused_kernel
+                   else "oq_weight_levels + oq_rotate_quantize_levels + oq_linear_decoded" if decoded else
                    "oq_rotate_quantize_levels + oq_linear_levels")
         + " (the stages of oq_linear_fused at this batch size; weights prepared once, offline)",
         "staged": ("oq_rotate_quantize_levels + oq_weight_levels + oq_linear_decoded" if decoded else
@@ -553,7 +556,7 @@ def run_ours(args):
         return row
 
     full_size = T == wl.tokens
-    launches_per_step = (1 if fused_kernel else 3) if decoded else 2
+    launches_per_step = (2 if fused_kernel else 3) if decoded else 2
     out = {
         "metric": METRIC,
         "value": whole_job_rate(world, T, K, total_ms),
@@ -732,6 +735,12 @@ def run_sweep(args):
             h_blk = d & -d
             fused_kernel = decoded and dout <= d and ((h_blk == 1024 and d // h_blk <= 8) or
                                                 (h_blk == 512 and d // h_blk <= 12))
+            if fused_kernel:
+                # the step runs the weight decode and the fused kernel: time
+                # the fused kernel on its own
+                ws_fd = torch.empty((max(B.oq_linear_fused_decoded_workspace_size(layer, T), 1),),
+                                    dtype=torch.uint8, device=dev)
+                runs["fused"] = [("fused", lambda: B.oq_linear_fused_decoded(layer, x, w16, r, y, ws_fd))]
             times = {}
             for name, st in runs.items():
                 for _ in range(warm):
@@ -752,9 +761,9 @@ def run_sweep(args):
             B.oq_poll_error(layer)
             flops = 2.0 * T * d * dout
             rq_alg = T * (2 * d + d * lay.a_bits / 8 + 4)
-            # the step's dominant kernel: where the step is the fused kernel
-            # (with its flag memset), the step; else the contraction
-            ck = "step" if fused_kernel else "gemm"
+            # the step's dominant kernel: the fused kernel where the step runs
+            # one, else the contraction
+            ck = "fused" if fused_kernel else "gemm"
             line = {
                 "metric": METRIC, "sweep_point": True, "value": T / (times["step"] * 1e-3), "unit": UNIT,
                 "n_gpus": 1, "steps": K, "warmup": warm, "ms_per_step": times["step"],
