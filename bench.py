@@ -33,6 +33,8 @@ UNIT = "tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
+# batches of up to this many tokens take the GEMV kernel (the library's routing)
+GEMV_MAX_T = 24
 
 
 def parse_args():
@@ -50,7 +52,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--sweep", action="store_true",
                     help="the stress workload's sweep (every token count x every layer): one JSON line per point")
-    ap.add_argument("--sweep-small", default="1,8",
+    ap.add_argument("--sweep-small", default="1,8,16,24",
                     help="batch sizes of the batch-1 / GEMV end added to the sweep (comma list, empty for none)")
     return ap.parse_args()
 
@@ -773,7 +775,7 @@ def run_sweep(args):
                            "x_bytes": T * d * 2,
                            "l2": "flushed (256 MiB write) before every step, outside the timed events",
                            "contraction": "decoded weights, both operands by TMA" if decoded else
-                           ("GEMV kernel (warp MMAs, weight codes decoded in registers)" if T <= 8 else
+                           ("GEMV kernel (warp MMAs, weight codes decoded in registers)" if T <= GEMV_MAX_T else
                             "small-batch split-K kernel" if T <= 256 else "CTA pair, weights decoded in the GEMM")},
                 "roofline": {"kernel": "fused layer kernel (rotate-quantize and contraction)"
                              if fused_kernel else "contraction",
@@ -791,7 +793,7 @@ def run_sweep(args):
                 "step_tflops": flops / (times["step"] * 1e-3) / 1e12,
                 "step_frac": flops / (times["step"] * 1e-3) / 1e12 / peaks["bf16_tflops"],
             }
-            if T <= 8:
+            if T <= GEMV_MAX_T:
                 # the batch-1 / GEMV end: the contraction streams the weight
                 # codes once; its floor is their bytes at HBM speed
                 gb = dout * d * lay.w_bits / 8 + T * d * 2 + dout * 4 + T * dout * 4

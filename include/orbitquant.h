@@ -324,13 +324,18 @@ oq_status oq_linear_fused(const oq_layer* layer, const void* x, int32_t x_dtype,
  * oq_linear_decoded exactly its y for T >= 1024 with the full workspace (and
  * the y of oq_rotate_quantize + oq_linear up to fp32 summation order).
  *
- * Small batches (T <= 256, d_out % 128 == 0) take a kernel whose M dimension
- * is 128 weight rows and whose N is the padded batch, with the K range split
- * across the SMs (the batch-1 / GEMV end of the workload sweep); the splits of
- * a tile add into y in a fixed order through per-layer counters, so results
- * repeat bit for bit, and calls on one layer must not overlap on the GPU
- * (different streams or host threads).  With bf16 y those batches take the
- * CTA-pair kernel instead (the splits add in fp32 in y itself).
+ * Batches of up to 24 tokens (d_out % 16 == 0, d_in % 32 == 0; the batch-1 /
+ * GEMV end of the workload sweep) take a kernel that streams the weight codes
+ * once, decodes them in registers and multiplies them with warp MMAs; each
+ * CTA owns 16 weight rows and adds its warps' partial sums in a fixed order,
+ * so results repeat bit for bit, for fp32 and bf16 y alike.  Larger small
+ * batches (T <= 256, d_out % 128 == 0) take a kernel whose M dimension is 128
+ * weight rows and whose N is the padded batch, with the K range split across
+ * the SMs; the splits of a tile add into y in a fixed order through per-layer
+ * counters, so results repeat bit for bit, and calls on one layer must not
+ * overlap on the GPU (different streams or host threads).  With bf16 y those
+ * batches take the CTA-pair kernel instead (the splits add in fp32 in y
+ * itself).
  */
 /*
  * oq_linear_fused_decoded -- oq_linear_fused with the weights' fp16 levels

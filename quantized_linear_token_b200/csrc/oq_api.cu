@@ -417,9 +417,10 @@ static oq_status linear_impl(const oq_layer* L, const uint32_t* codes, const flo
   g.a_bits = L->a_bits;
   g.b_bits = L->w_bits;
   g.err = L->d_error;
-  // a few hundred tokens or fewer: the small-batch kernel (weight rows as the
-  // MMA's M, split K, its splits added in fp32 in y itself, so fp32 y only);
-  // larger batches and bf16 y: the CTA-pair kernel
+  // up to GEMV_MAX_T tokens: the GEMV kernel (weights streamed once, warp
+  // MMAs); a few hundred tokens or fewer: the small-batch kernel (weight rows
+  // as the MMA's M, split K, its splits added in fp32 in y itself, so fp32 y
+  // only); larger batches and bf16 y: the CTA-pair kernel
   if (a_f16 && T <= GEMV_MAX_T && !L->fp8) {
     const oq_status st = gemv_launch(g, stream);
     if (st != OQ_ERR_UNSUPPORTED) return st;

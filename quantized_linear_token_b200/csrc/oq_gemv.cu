@@ -1,11 +1,12 @@
 // Codebook contraction for the batch-1 / GEMV end of the workload sweep
-// (T <= 8 tokens): y[t, o] = a_scale[t] b_scale[o] out_scale sum_k A[t, k]
+// (T <= 24 tokens): y[t, o] = a_scale[t] b_scale[o] out_scale sum_k A[t, k]
 // C_w[Wc[o, k]], with A the fp16 levels of the activation codes (gecl notes
 // Method 2; the weights are streamed once and are the whole cost, so the
 // kernel is built to read them at HBM speed).
 //
 // A CTA owns 16 weight rows; its 8 warps split K.  Each warp runs warp-level
-// MMAs (m16n8k16: M = 16 weight rows, N = 8 tokens, K = 16, fp32 accumulate)
+// MMAs (m16n8k16: M = 16 weight rows, N = a tile of 8 tokens, K = 16, fp32
+// accumulate; up to three token tiles share each decoded weight fragment)
 // with its own mapping of the MMA's K slots to positions, chosen so that a
 // lane's operands are contiguous in memory: in a chunk of 128 positions,
 // lane q of each quad owns positions [32 q, 32 q + 32), and MMA step s (of 8)
@@ -16,6 +17,12 @@
 // token's levels per chunk, and decodes the codes with byte-permute lookups in
 // registers.  The 8 warps' partial sums meet in shared memory and are added in
 // a fixed order, so results repeat bit for bit; no CTA waits on another.
+//
+// Streaming the weights at HBM speed takes several megabytes in flight across
+// the GPU (bandwidth times latency), so each warp keeps the weight groups of
+// its next chunks in registers (PREFETCH of them for one token tile, one
+// fewer for more tiles, whose MMAs take longer per chunk): the loads of chunk
+// i + PF are issued before chunk i is decoded and multiplied.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -31,6 +38,8 @@ namespace {
 constexpr int ROWS = 16;           // weight rows per CTA (the MMA's M)
 constexpr int NWARP = 8;           // warps per CTA, splitting K
 constexpr int CHUNK = 128;         // K positions per warp step (32 per quad lane)
+constexpr int PREFETCH = 3;        // chunks of weight codes in flight per warp
+constexpr int MIN_CTAS = 3;        // resident CTAs per SM the register budget allows
 
 struct GemvParams {
   const uint32_t* codes;           // weight codes [N, K * bits / 32]
@@ -73,59 +82,95 @@ __device__ __forceinline__ uint4 decode8(const uint4& v, int j, const uint32_t (
   return decode_chunk<BITS>(v, j, t, nullptr);
 }
 
-template <int BITS>
-__global__ void __launch_bounds__(NWARP * 32, 4) gemv_kernel(const __grid_constant__ GemvParams p) {
-  __shared__ __align__(16) float part[NWARP][32][4];
+template <int BITS, int NT>
+__global__ void __launch_bounds__(NWARP * 32, MIN_CTAS) gemv_kernel(const __grid_constant__ GemvParams p) {
+  __shared__ __align__(16) float part[NWARP][NT][32][4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
   const int o0 = blockIdx.x * ROWS;
   const uint32_t* row_lo = p.codes + (size_t)(o0 + g) * p.wpr;       // weight row g of the tile
   const uint32_t* row_hi = p.codes + (size_t)(o0 + g + 8) * p.wpr;   // weight row g + 8
-  const bool tok = g < p.T;                                          // this lane's token (B column g)
-  const uint16_t* arow = p.a16 + (size_t)(tok ? g : 0) * p.K;
+  // this lane's token in token tile n (B column g of tile n) is 8 n + g; its
+  // levels start at arow + 8 n K
+  const uint16_t* arow = p.a16 + (size_t)g * p.K;
   uint32_t t[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) t[i] = p.tab[i];
 
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // this warp's chunks are warp, warp + NWARP, ...: chunk i of the warp starts
+  // at position (warp + i NWARP) CHUNK, and the lane's 32 positions at 32 q
+  // past that (K % 32 == 0, so a lane's group lies wholly inside or past K)
   const int nchunks = (p.K + CHUNK - 1) / CHUNK;
+  const int nmine = warp < nchunks ? (nchunks - 1 - warp) / NWARP + 1 : 0;
+  auto pos_of = [&](int i) { return (warp + i * NWARP) * CHUNK + 32 * q; };
+  constexpr int PF = NT == 1 ? PREFETCH : PREFETCH - 1;
+  uint4 wl[PF], wh[PF];
+#pragma unroll
+  for (int u = 0; u < PF; ++u) {
+    const int pos = pos_of(u);
+    const bool valid = u < nmine && pos < p.K;
+    wl[u] = load_group<BITS>(row_lo, pos >> 5, valid);
+    wh[u] = load_group<BITS>(row_hi, pos >> 5, valid);
+  }
+
+  float acc[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
 #pragma unroll 1
-  for (int c = warp; c < nchunks; c += NWARP) {
-    const int pos0 = c * CHUNK + 32 * q;                              // this lane's 32 positions
-    const bool valid = pos0 < p.K;                                    // K % 32 == 0: whole groups
-    const uint4 wl = load_group<BITS>(row_lo, pos0 >> 5, valid);
-    const uint4 wh = load_group<BITS>(row_hi, pos0 >> 5, valid);
-    uint4 av[4];
+  for (int i0 = 0; i0 < nmine; i0 += PF) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      av[i] = (valid && tok) ? __ldg(reinterpret_cast<const uint4*>(arow + pos0) + i) : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t aw[16] = {av[0].x, av[0].y, av[0].z, av[0].w, av[1].x, av[1].y, av[1].z, av[1].w,
-                             av[2].x, av[2].y, av[2].z, av[2].w, av[3].x, av[3].y, av[3].z, av[3].w};
+    for (int u = 0; u < PF; ++u) {
+      const int i = i0 + u;
+      if (i >= nmine) break;                                          // warp-uniform
+      const int pos0 = pos_of(i);
+      const bool valid = pos0 < p.K;
+      const uint4 cl = wl[u], ch = wh[u];
+      // refill the slot with chunk i + PF before working on chunk i
+      const int posn = pos_of(i + PF);
+      const bool vn = i + PF < nmine && posn < p.K;
+      wl[u] = load_group<BITS>(row_lo, posn >> 5, vn);
+      wh[u] = load_group<BITS>(row_hi, posn >> 5, vn);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 dl = decode8<BITS>(wl, j, t), dh = decode8<BITS>(wh, j, t);
-      // step 2j: positions 8j .. 8j + 3; step 2j + 1: 8j + 4 .. 8j + 7
-      mma_f16_16816(acc, dl.x, dh.x, dl.y, dh.y, aw[4 * j], aw[4 * j + 1]);
-      mma_f16_16816(acc, dl.z, dh.z, dl.w, dh.w, aw[4 * j + 2], aw[4 * j + 3]);
+      for (int j = 0; j < 4; ++j) {
+        // positions 8j .. 8j + 7 of the lane's group: the weights decoded
+        // once, then step 2j (8j .. 8j + 3) and 2j + 1 (8j + 4 .. 8j + 7) for
+        // every token tile
+        const uint4 dl = decode8<BITS>(cl, j, t), dh = decode8<BITS>(ch, j, t);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          const uint4 a = (valid && 8 * n + g < p.T)
+                              ? __ldg(reinterpret_cast<const uint4*>(arow + (size_t)(8 * n) * p.K + pos0) + j)
+                              : make_uint4(0u, 0u, 0u, 0u);
+          mma_f16_16816(acc[n], dl.x, dh.x, dl.y, dh.y, a.x, a.y);
+          mma_f16_16816(acc[n], dl.z, dh.z, dl.w, dh.w, a.z, a.w);
+        }
+      }
     }
   }
   // the warps' partial sums, added in warp order
-  *reinterpret_cast<float4*>(part[warp][lane]) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+#pragma unroll
+  for (int n = 0; n < NT; ++n)
+    *reinterpret_cast<float4*>(part[warp][n][lane]) = make_float4(acc[n][0], acc[n][1], acc[n][2], acc[n][3]);
   __syncthreads();
-  if (warp != 0) return;
+  if (warp >= NT) return;
+  // warp n writes token tile n
+  const int n = warp;
   float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int w = 0; w < NWARP; ++w) {
-    const float4 v = *reinterpret_cast<const float4*>(part[w][lane]);
+    const float4 v = *reinterpret_cast<const float4*>(part[w][n][lane]);
     s[0] += v.x;
     s[1] += v.y;
     s[2] += v.z;
     s[3] += v.w;
   }
-  // accumulator (row m, column n): d0 = (g, 2q), d1 = (g, 2q + 1),
-  // d2 = (g + 8, 2q), d3 = (g + 8, 2q + 1); rows are weight rows, columns tokens
+  // accumulator (row m, column c): d0 = (g, 2q), d1 = (g, 2q + 1),
+  // d2 = (g + 8, 2q), d3 = (g + 8, 2q + 1); rows are weight rows, column c is
+  // token 8 n + c
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int o = o0 + g + 8 * (i >> 1), tk = 2 * q + (i & 1);
+    const int o = o0 + g + 8 * (i >> 1), tk = 8 * n + 2 * q + (i & 1);
     if (tk >= p.T) continue;
     const float v = s[i] * __ldg(p.a_scale + tk) * p.out_scale * __ldg(p.b_scale + o);
     const size_t at = (size_t)tk * p.N + o;
@@ -136,6 +181,16 @@ __global__ void __launch_bounds__(NWARP * 32, 4) gemv_kernel(const __grid_consta
       static_cast<float*>(p.y)[at] = v;
     }
   }
+}
+
+template <int BITS>
+cudaError_t launch_bits(const GemvParams& kp, unsigned grid, cudaStream_t s) {
+  switch ((kp.T + 7) / 8) {
+    case 1: gemv_kernel<BITS, 1><<<grid, NWARP * 32, 0, s>>>(kp); break;
+    case 2: gemv_kernel<BITS, 2><<<grid, NWARP * 32, 0, s>>>(kp); break;
+    default: gemv_kernel<BITS, 3><<<grid, NWARP * 32, 0, s>>>(kp); break;
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace
@@ -162,12 +217,12 @@ oq_status gemv_launch(const GemmArgs& g, void* stream) {
   make_decode_tables(g.b_bits, g.b_levels_host, kp.tab);
   const unsigned grid = (unsigned)(g.N / ROWS);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
   switch (g.b_bits) {
-    case 2: gemv_kernel<2><<<grid, NWARP * 32, 0, s>>>(kp); break;
-    case 3: gemv_kernel<3><<<grid, NWARP * 32, 0, s>>>(kp); break;
-    default: gemv_kernel<4><<<grid, NWARP * 32, 0, s>>>(kp); break;
+    case 2: e = launch_bits<2>(kp, grid, s); break;
+    case 3: e = launch_bits<3>(kp, grid, s); break;
+    default: e = launch_bits<4>(kp, grid, s); break;
   }
-  const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("gemv launch: ") + cudaGetErrorString(e));
     return OQ_ERR_CUDA;

@@ -136,9 +136,9 @@ oq_status gemm_pair_launch(const GemmArgs& g, void* stream);
 // N % 128 == 0; `counters` holds N / 32 zeroed ints
 constexpr int SKINNY_MAX_T = 256;
 // GEMV contraction for up to GEMV_MAX_T tokens (oq_gemv.cu): fp16 A operand,
-// weight codes of 2-4 bits decoded in registers, warp MMAs, no split across
-// CTAs; N % 16 == 0, K % 32 == 0
-constexpr int GEMV_MAX_T = 8;
+// weight codes of 2-4 bits decoded in registers, warp MMAs over up to three
+// tiles of 8 tokens, no split across CTAs; N % 16 == 0, K % 32 == 0
+constexpr int GEMV_MAX_T = 24;
 oq_status gemv_launch(const GemmArgs& g, void* stream);
 oq_status gemm_skinny_launch(const GemmArgs& g, int* counters, void* stream);
 // INT4 weight-only round-to-nearest of weight rows (oq_int4.cu): per-row

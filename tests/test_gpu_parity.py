@@ -282,15 +282,28 @@ def test_small_batch_sweep(env, T):
 
 
 GEMV = [
-    # d_in, d_out, a, w, T: batches of up to 8 tokens take the GEMV kernel
-    # (weights streamed once, warp MMAs, K split over a CTA's warps): every
-    # weight width, a K that is not a multiple of the 128-position chunk, 8-bit
-    # activations, and the largest batch it takes
+    # d_in, d_out, a, w, T: batches of up to 24 tokens take the GEMV kernel
+    # (weights streamed once, warp MMAs over one to three tiles of 8 tokens, K
+    # split over a CTA's warps): every weight width, a K that is not a
+    # multiple of the 128-position chunk, 8-bit activations, every tile count
+    # with ragged last tiles, the largest batch it takes, and the stress layer
+    # at batch 1, 8, 16 and 24 (25 tokens: the small-batch kernel)
     (96, 256, 4, 2, 3),
     (3072, 512, 4, 4, 1),
     (3072, 512, 3, 3, 8),
     (5120, 256, 4, 2, 2),
     (13824, 512, 8, 4, 5),
+    (13824, 5120, 4, 4, 1),
+    (13824, 5120, 4, 2, 8),
+    (5120, 5120, 3, 3, 7),
+    (96, 256, 4, 3, 9),
+    (3072, 512, 4, 4, 16),
+    (5120, 256, 4, 2, 21),
+    (3072, 768, 3, 3, 24),
+    (13824, 512, 8, 4, 23),
+    (13824, 5120, 4, 4, 16),
+    (13824, 5120, 4, 4, 24),
+    (13824, 5120, 4, 4, 25),
 ]
 
 
@@ -299,6 +312,25 @@ def test_gemv_batches(env, d_in, d_out, a_bits, w_bits, T):
     x_np = W.custom_activations(T, d_in, seed=d_in + 11 * T)
     Wm = W.custom_weights(d_out, d_in, seed=d_out + 13)
     _run_layer(env, d_in, d_out, a_bits, w_bits, x_np, Wm, label=f"gemv {d_in}x{d_out} T={T}")
+
+
+@pytest.mark.parametrize("T", [1, 8, 24])
+def test_gemv_repeats_bit_for_bit(env, T):
+    # repeated calls, on the level stages and through the fused call, give
+    # one y bit for bit
+    torch, B = env
+    d_in, d_out = 13824, 5120
+    x_np, Wm = _inputs("stress_w4a4", d_in, d_out, T)
+    layer = B.oq_layer_create(d_in, d_out, 0, 4, 4)
+    Wc, r = B.oq_weight_prepare(layer, torch.from_numpy(Wm).cuda())
+    x_t, _ = _x_tensor(torch, x_np)
+    a16, s = B.oq_rotate_quantize_levels(layer, x_t)
+    ys = [B.oq_linear_levels(layer, a16, s, Wc, r) for _ in range(3)]
+    ys += [B.oq_linear_fused(layer, x_t, Wc, r) for _ in range(3)]
+    torch.cuda.synchronize()
+    B.oq_poll_error(layer)
+    for y in ys[1:]:
+        assert torch.equal(y.view(torch.int32), ys[0].view(torch.int32))
 
 
 @pytest.mark.parametrize("T,d_in,d_out,w_bf16", [(2, 3072, 18432, False), (7, 1024, 256, True),
