@@ -273,8 +273,9 @@ def test_edge_shapes(env, d_in, d_out, a_bits, w_bits, T, flags):
 
 @pytest.mark.parametrize("T", [1, 16, 64, 200, 256, 257])
 def test_small_batch_sweep(env, T):
-    # the small-T end of the workload sweep (d 13824 -> 5120, W4A4): batches of
-    # up to 256 tokens take the split-K small-batch kernel, 257 the CTA pair
+    # the small-T end of the workload sweep (d 13824 -> 5120, W4A4): up to 24
+    # tokens take the GEMV kernel, up to 256 the split-K small-batch kernel,
+    # 257 the CTA pair
     x_np, Wm = _inputs("stress_w4a4", 13824, 5120, T)
     rng = np.random.default_rng(11)
     w_rows = np.unique(np.concatenate([np.arange(32), rng.choice(5120, 64, replace=False)]))
