@@ -671,13 +671,20 @@ static oq_status fused_decoded(const oq_layer* L, const void* x, int32_t x_dtype
   float* s = reinterpret_cast<float*>(ws + round256(fused_f16_bytes(L, T)));
   const RQArgs ra = rq_levels_args(L, x, x_dtype, T, a16, s);
   oq_status st = OQ_OK;
+  const bool fused = fused_kernel_pays(L) && fused_kernel_supported(ra, L->d_out);
+  int* flags = reinterpret_cast<int*>(ws + round256(need));
+  // with a weight decode, the fused kernel follows it directly as its
+  // programmatic dependent, so its flags are cleared before the decode
+  if (fused && Wcodes) {
+    st = fused_clear_flags(flags, T, stream);
+    if (st != OQ_OK) return st;
+  }
   if (Wcodes) {
     st = levels_launch(Wcodes, L->d_out, L->d_in, L->w_bits, L->lv_w, L->d_levels_w, w16, stream);
     if (st != OQ_OK) return st == OQ_ERR_UNSUPPORTED ? fail(st, "oq_linear_fused: unsupported shape") : st;
   }
-  if (fused_kernel_pays(L) && fused_kernel_supported(ra, L->d_out)) {
-    int* flags = reinterpret_cast<int*>(ws + round256(need));
-    st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), flags, stream);
+  if (fused) {
+    st = fused_launch(ra, w16_args(L, a16, s, T, w16, r, y, y_bf16), flags, stream, Wcodes != nullptr);
     if (st != OQ_ERR_UNSUPPORTED) return st;
   }
   st = rq_levels(L, x, x_dtype, T, a16, s, stream);

@@ -293,6 +293,10 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(112)
     }
   } else if (warp == TMA_WARP) {
     // ------------------------------------------------ TMA producer (both CTAs)
+    // the decoded weights may come from the kernel just before this one (a
+    // programmatic dependent launch): wait for that grid and its writes before
+    // the first B load (returns at once after an ordinary launch)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const uint32_t full0 = mapa_shared(smem_u32(&op_full[0]), 0);
     int s = 0;
     uint32_t n = 0;
@@ -448,7 +452,16 @@ bool fused_kernel_supported(const RQArgs& a, int N) {
   return smem_bytes(A, A == 32 && a.gather_cc, nb, nw, 1, stage_bytes, 3, 1, nullptr) <= 227 * 1024;
 }
 
-oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream) {
+oq_status fused_clear_flags(int* flags, int64_t T, void* stream) {
+  const cudaError_t e = cudaMemsetAsync(flags, 0, fused_flag_bytes(T), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    set_error(std::string("clear fused flags: ") + cudaGetErrorString(e));
+    return OQ_ERR_CUDA;
+  }
+  return OQ_OK;
+}
+
+oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream, bool after_levels) {
   if (g.M == 0) return OQ_OK;
   if (!fused_kernel_supported(a, g.N) || !g.b_f16) return OQ_ERR_UNSUPPORTED;
   FusedParams kp;
@@ -520,14 +533,24 @@ oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* str
   const int grid = sms & ~1;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   // the flags and the queue counter start at zero on every call
-  e = cudaMemsetAsync(flags, 0, fused_flag_bytes(g.M), s);
-  if (e != cudaSuccess) {
-    set_error(std::string("clear fused flags: ") + cudaGetErrorString(e));
-    return OQ_ERR_CUDA;
+  if (!after_levels) {
+    const oq_status cs = fused_clear_flags(flags, g.M, stream);
+    if (cs != OQ_OK) return cs;
   }
   const unsigned threads = (unsigned)((GEMM_WARPS + teams * kp.nw) * 32);
-  kern<<<(unsigned)grid, threads, smem, s>>>(kp);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = after_levels ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, kp);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     cudaFuncAttributes fa;
     std::memset(&fa, 0, sizeof(fa));

@@ -154,11 +154,15 @@ oq_status gemm_w16_launch(const GemmArgs& g, void* stream);
 // the fused call decodes the weights once per call from this many tokens on
 constexpr int64_t W16_MIN_T = 1024;
 // the fused layer kernel (oq_fused.cu): rotate-quantize producer teams inside
-// the CTA-pair contraction of the decoded weights.  `flags` is zeroed
-// workspace of fused_flag_bytes(T) bytes (cleared by the launch itself).
+// the CTA-pair contraction of the decoded weights.  `flags` is workspace of
+// fused_flag_bytes(T) bytes, cleared by the launch itself, or, with
+// after_levels, by fused_clear_flags before the weight-level kernel that the
+// fused kernel then follows directly as its programmatic dependent (its
+// producers start while the weights are decoded; its TMA warp waits for them).
 bool fused_kernel_supported(const RQArgs& a, int N);
 size_t fused_flag_bytes(int64_t T);
-oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream);
+oq_status fused_clear_flags(int* flags, int64_t T, void* stream);
+oq_status fused_launch(const RQArgs& a, const GemmArgs& g, int* flags, void* stream, bool after_levels = false);
 // the fused call's pieces for the host-buffer pipeline (oq_api.cu): the least
 // workspace; the workspace with the decoded weights after it; whether the
 // fused call decodes the weights once at this batch size; argument checks;

@@ -26,6 +26,9 @@ __global__ void __launch_bounds__(256) levels_flat_kernel(const uint32_t* __rest
                                                           uint4* __restrict__ out) {
   constexpr int UNROLL = 4;
   __shared__ uint16_t lut8[256];
+  // a kernel launched as this one's programmatic dependent (the fused layer
+  // kernel) may start now: it waits for this grid before it reads the levels
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if constexpr (BITS == 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = lut8_g[i];
     __syncthreads();
@@ -63,6 +66,7 @@ __global__ void __launch_bounds__(256) levels_kernel(const uint32_t* __restrict_
                                                      uint4 tabv, DecK kc, const uint16_t* lut8_g,
                                                      uint16_t* __restrict__ out) {
   __shared__ uint16_t lut8[256];
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if constexpr (BITS == 8) {
     for (int i = threadIdx.x; i < 256; i += blockDim.x) lut8[i] = lut8_g[i];
     __syncthreads();
