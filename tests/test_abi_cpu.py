@@ -115,3 +115,22 @@ def test_python_names_mirror_c_names():
                     "oq_layer_get_perm"):
             continue
         assert callable(getattr(B, name)), name
+
+
+def test_routing_thresholds_mirror_the_library():
+    # bench.py labels its sweep points and the tests pick their bounds by the
+    # batch sizes at which the library changes kernels; those copies must
+    # follow the library's own constants
+    import bench
+    src = open(os.path.join(Bld.CSRC, "oq_internal.h")).read()
+
+    def const(name):
+        m = re.search(r"constexpr\s+(?:int|int64_t)\s+" + name + r"\s*=\s*(\d+)\s*;", src)
+        assert m, name
+        return int(m.group(1))
+
+    assert bench.GEMV_MAX_T == const("GEMV_MAX_T")
+    assert B.W16_MIN_T == const("W16_MIN_T")
+    text = open(os.path.join(os.path.dirname(__file__), "test_gpu_parity.py")).read()
+    assert int(re.search(r"^SKINNY_MAX_T = (\d+)", text, re.M).group(1)) == const("SKINNY_MAX_T")
+    assert int(re.search(r"^W16_MIN_T = (\d+)", text, re.M).group(1)) == const("W16_MIN_T")
