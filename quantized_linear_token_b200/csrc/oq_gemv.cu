@@ -18,11 +18,11 @@
 // registers.  The 8 warps' partial sums meet in shared memory and are added in
 // a fixed order, so results repeat bit for bit; no CTA waits on another.
 //
-// Streaming the weights at HBM speed takes several megabytes in flight across
-// the GPU (bandwidth times latency), so each warp keeps the weight groups of
-// its next chunks in registers (PREFETCH of them for one token tile, one
-// fewer for more tiles, whose MMAs take longer per chunk): the loads of chunk
-// i + PF are issued before chunk i is decoded and multiplied.
+// Each warp keeps the weight groups of its next chunks in registers (PREFETCH
+// of them for one token tile, one fewer for more tiles, whose MMAs take longer
+// per chunk): the loads of chunk i + PF are issued before chunk i is decoded
+// and multiplied.  The kernel is bound by instruction issue (the decode) more
+// than by the loads in flight: depths of 1 to 6 chunks measured alike.
 #include <cuda_bf16.h>
 
 #include <algorithm>
