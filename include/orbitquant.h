@@ -251,10 +251,12 @@ oq_status oq_linear(const oq_layer* layer, const uint32_t* codes, const float* s
  * weights' fp16 levels, which are then decoded once per call
  * (oq_weight_levels), and about T bytes of row-group flags.  That route
  * contracts the two fp16 operands on CTA pairs; where the block size is 1024
- * or 512 (at most 12 warps per token row) one kernel does both steps, its
- * rotate-quantize warps writing the A operand while the contraction of
- * earlier tiles runs, otherwise oq_rotate_quantize_levels' kernel and
- * oq_linear_decoded's kernel run in turn; y is the same bit for bit.  A
+ * or 512 (at most 12 warps per token row) and d_out <= d_in one kernel does
+ * both steps, its rotate-quantize warps writing the A operand while the
+ * contraction of earlier tiles runs (it is launched as a programmatic
+ * dependent of the weight decode, whose output only its TMA warp waits for),
+ * otherwise oq_rotate_quantize_levels' kernel and oq_linear_decoded's kernel
+ * run in turn.  A
  * smaller workspace that still holds the A operand and the norms (the least
  * size: 2 T d_in bytes rounded up to a multiple of 256, plus 4 T, on the
  * fp16-level route) is accepted and decodes the weights inside the
