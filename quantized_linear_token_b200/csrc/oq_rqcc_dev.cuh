@@ -23,16 +23,32 @@
 namespace oq {
 namespace rqcc {
 
-// in-register butterflies on v[0..32): stride S pairs (i, i + S) for i & S == 0
+// (a0, a1), (b0, b1) -> (a0 + b0, a1 + b1), (a0 - b0, a1 - b1) on the paired
+// fp32 pipe (add.f32x2 / sub.f32x2: each lane of the pair rounds as a scalar
+// add or subtract would)
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
+  asm("{\n\t.reg .b64 A, B, S, D;\n\tmov.b64 A, {%0, %1};\n\tmov.b64 B, {%2, %3};\n\t"
+      "add.rn.f32x2 S, A, B;\n\tsub.rn.f32x2 D, A, B;\n\tmov.b64 {%0, %1}, S;\n\tmov.b64 {%2, %3}, D;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
+}
+
+// in-register butterflies on v[0..32): stride S pairs (i, i + S) for i & S == 0;
+// from stride 2 on, the pairs (i, i + S) and (i + 1, i + S + 1) go together
 template <int S>
 __device__ __forceinline__ void stage(float (&v)[32]) {
+  if constexpr (S >= 2) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if ((i & S) == 0) {
-      const float a = v[i], b = v[i + S];
-      v[i] = a + b;
-      v[i + S] = a - b;
-    }
+    for (int i = 0; i < 32; i += 2)
+      if ((i & S) == 0) bfly2(v[i], v[i + 1], v[i + S], v[i + S + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if ((i & S) == 0) {
+        const float a = v[i], b = v[i + S];
+        v[i] = a + b;
+        v[i + S] = a - b;
+      }
+  }
 }
 
 __device__ __forceinline__ void fwht32(float (&v)[32]) {
