@@ -6,7 +6,9 @@ warp MMAs, and feeds pass 1's accumulator registers to pass 2 as B
 fragments after choosing pass 2's K order to match.  This emulates those
 fragment layouts (the m16n8k16 and m16n8k8 register maps of the PTX warp MMA
 instructions) lane by lane in numpy and checks that the assembled result is
-the Sylvester transform of the flattened block.  It pins the derivation the
+the Sylvester transform of the flattened block, and that the packed-code
+output (each lane placing its code pairs in the group's bit stream, the quad
+OR-ing its words) assembles the packed group.  It pins the derivation the
 kernel's indexing follows; the kernel itself is checked on the GPU."""
 
 import numpy as np
@@ -66,3 +68,36 @@ def test_two_pass_fragment_transform(A):
                     for e2 in range(2):
                         a, b = 16 * mt2 + g + 8 * half, 8 * nt2 + 2 * q + e2
                         assert np.isclose(acc[g + 8 * half][2 * q + e2], z[32 * a + b])
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_packed_code_quad_or(bits):
+    # The tensor-core kernel's packed-code output: for one row a' of the block
+    # (a group of 32 positions b'), lane q of a quad holds the codes of
+    # b' = 8 nt + 2q + {0, 1} (nt = 0..3); it places each pair at bit
+    # bits * (8 nt + 2q) of the group's stream (bits words), the four lanes OR
+    # their words together (two xor shuffles) and lane q stores the words
+    # i with i % 4 == q.  The assembled words must be the packed group.
+    rng = np.random.default_rng(bits)
+    codes = rng.integers(0, 1 << bits, size=32)
+    lanes = []
+    for q in range(4):
+        w = [0] * bits
+        for nt in range(4):
+            c0, c1 = int(codes[8 * nt + 2 * q]), int(codes[8 * nt + 2 * q + 1])
+            pair = c0 | (c1 << bits)
+            bit = bits * (8 * nt + 2 * q)
+            for i in range(bits):
+                lo = bit - 32 * i                       # the pair's offset within word i
+                if 0 <= lo < 32:
+                    w[i] |= (pair << lo) & 0xFFFFFFFF
+                if -2 * bits < lo < 0:
+                    w[i] |= pair >> (-lo)
+        lanes.append(w)
+    ored = [lanes[0][i] | lanes[1][i] | lanes[2][i] | lanes[3][i] for i in range(bits)]
+    stored = [None] * bits
+    for q in range(4):
+        for i in range(bits):
+            if i % 4 == q:
+                stored[i] = ored[i]
+    np.testing.assert_array_equal(np.array(stored, dtype=np.uint32), O.pack_codes(codes, bits))
